@@ -1,0 +1,221 @@
+"""The oracle: a plain fp64 CPU restatement of sink-softmax attention.
+
+TEST INFRASTRUCTURE. Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package. The CUDA library never reaches it, and it imports nothing
+from the CUDA library: the two share no code. The arithmetic lives in ``sinkattn_oracle.c``
+(plain C, fp64); this module only compiles it with gcc and marshals arrays.
+
+Every function takes bf16 tensors (CPU, any layout; they are made contiguous here) and returns
+float64 tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sinkattn_oracle.c")
+_LIB_DIR = os.path.join(_HERE, "_build")
+_LIB = os.path.join(_LIB_DIR, "libsinkattn_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+# KV-cache kinds (same numbering as the library header; restated, not shared).
+KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (fp64, IEEE semantics, no fast-math, no FMA contraction)."""
+    os.makedirs(_LIB_DIR, exist_ok=True)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC",
+             "-std=c11", _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            # SINKATTN_ORACLE_LIB points the oracle at another build of the same source; the
+            # mutation test uses it to load deliberately broken copies of the oracle.
+            path = os.environ.get("SINKATTN_ORACLE_LIB") or build()
+            lib = ctypes.CDLL(path)
+            P = ctypes.c_void_p
+            i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+            lib.sinkattn_oracle_prefill.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                                    f64, P, i64, P, P, P]
+            lib.sinkattn_oracle_prefill.restype = i32
+            lib.sinkattn_oracle_decode.argtypes = [i32, P, P, P, P, P, P, P, i32, P, i32, P, i32,
+                                                   i32, P, i32, i32, i32, i32, i32, i32, i32, f64,
+                                                   P, i32, P, P, P]
+            lib.sinkattn_oracle_decode.restype = i32
+            lib.sinkattn_oracle_partial.argtypes = [P, P, P, i32, i32, i32, i32, f64, P, P, P]
+            lib.sinkattn_oracle_partial.restype = None
+            lib.sinkattn_oracle_merge.argtypes = [P, P, P, i32, i32, f64, P, P]
+            lib.sinkattn_oracle_merge.restype = None
+            lib.sinkattn_oracle_commit.argtypes = [i32, P, P, P, P, P, P, P, i32, P, i32, P, i32,
+                                                   i32, i32, i32, i32, i32, i32]
+            lib.sinkattn_oracle_commit.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    """bf16 tensor -> contiguous uint16 numpy array of its bit patterns."""
+    assert t.dtype == torch.bfloat16, t.dtype
+    return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy()).view(np.uint16)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _i32(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(t, dtype=np.int32))
+
+
+def _f32(t):
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        t = t.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(t, dtype=np.float32))
+
+
+def prefill(q, k, v, sink, scale, window=0, rows=None, want_wsink=False):
+    """Sink attention over a whole sequence (prefill).
+
+    q [B,L,Hq,dq], k [B,L,Hkv,dq], v [B,L,Hkv,dv] bf16; sink [Hq] fp32 or None (no sink);
+    window > 0 selects the sliding window (keys i-window < j <= i), 0 the full causal mask.
+    rows: optional [n, 2] int array of (b, i) pairs; then outputs are [n, Hq, ...].
+    Returns (o [B,L,Hq,dv] or [n,Hq,dv], lse [B,L,Hq] or [n,Hq], wsink or None), float64.
+    """
+    lib = _load()
+    B, L, Hq, dq = q.shape
+    Hkv, dv = k.shape[2], v.shape[3]
+    qb, kb, vb = _bits(q), _bits(k), _bits(v)
+    s = _f32(sink)
+    r = _i32(rows)
+    n = B * L if r is None else r.shape[0]
+    o = np.zeros((n, Hq, dv), np.float64)
+    lse = np.zeros((n, Hq), np.float64)
+    ws = np.zeros((n, Hq), np.float64) if want_wsink else None
+    rc = lib.sinkattn_oracle_prefill(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(s), B, L, Hq, Hkv, dq, dv,
+                                     int(window), float(scale), _ptr(r), 0 if r is None else n,
+                                     _ptr(o), _ptr(lse), _ptr(ws))
+    if rc != 0:
+        raise ValueError("oracle prefill: bad arguments")
+    if r is None:
+        o, lse = o.reshape(B, L, Hq, dv), lse.reshape(B, L, Hq)
+        ws = None if ws is None else ws.reshape(B, L, Hq)
+    return (torch.from_numpy(o), torch.from_numpy(lse),
+            None if ws is None else torch.from_numpy(ws))
+
+
+def decode(kind, q, k_new, v_new, k_cache, v_cache, sink, scale, window=0, *, ring_head=None,
+           ring_len=None, ctx_len=None, page_table=None, page_size=0, seqs=None,
+           want_wsink=False):
+    """Sink attention for T new tokens per sequence against a KV cache (decode / verify).
+
+    kind: KV_RING (k_cache [B,cap,Hkv,dq] + ring_head/ring_len), KV_CONTIG (k_cache
+    [B,max_ctx,Hkv,dq] + ctx_len) or KV_PAGED (k_cache [pages,page_size,Hkv,dq] + page_table
+    [B,max_pages] + ctx_len). seqs: optional list of sequence indices to evaluate.
+    Returns (o [n,T,Hq,dv], lse [n,T,Hq], wsink or None), float64.
+    """
+    lib = _load()
+    B, T, Hq, dq = q.shape
+    Hkv, dv = k_new.shape[2], v_new.shape[3]
+    qb, knb, vnb = _bits(q), _bits(k_new), _bits(v_new)
+    kcb, vcb = _bits(k_cache), _bits(v_cache)
+    s = _f32(sink)
+    rh, rl, cl, pt = _i32(ring_head), _i32(ring_len), _i32(ctx_len), _i32(page_table)
+    sq = _i32(seqs)
+    ring_cap = k_cache.shape[1] if kind == KV_RING else 0
+    max_ctx = k_cache.shape[1] if kind == KV_CONTIG else 0
+    max_pages = pt.shape[1] if pt is not None else 0
+    n = B if sq is None else sq.shape[0]
+    o = np.zeros((n, T, Hq, dv), np.float64)
+    lse = np.zeros((n, T, Hq), np.float64)
+    ws = np.zeros((n, T, Hq), np.float64) if want_wsink else None
+    rc = lib.sinkattn_oracle_decode(int(kind), _ptr(qb), _ptr(knb), _ptr(vnb), _ptr(kcb), _ptr(vcb),
+                                    _ptr(rh), _ptr(rl), ring_cap, _ptr(cl), max_ctx, _ptr(pt),
+                                    int(page_size), max_pages, _ptr(s), B, T, Hq, Hkv, dq, dv,
+                                    int(window), float(scale), _ptr(sq), n, _ptr(o), _ptr(lse),
+                                    _ptr(ws))
+    if rc != 0:
+        raise ValueError("oracle decode: bad arguments")
+    return (torch.from_numpy(o), torch.from_numpy(lse),
+            None if ws is None else torch.from_numpy(ws))
+
+
+def partial(q_row, k_rows, v_rows, j0, j1, scale):
+    """(O_P, m_P, l_P) of one query row over keys [j0, j1) without the sink.
+
+    q_row [dq], k_rows [n,dq], v_rows [n,dv] bf16."""
+    lib = _load()
+    qb, kb, vb = _bits(q_row), _bits(k_rows), _bits(v_rows)
+    dq, dv = q_row.shape[0], v_rows.shape[1]
+    o = np.zeros(dv, np.float64)
+    m = np.zeros(1, np.float64)
+    l = np.zeros(1, np.float64)
+    lib.sinkattn_oracle_partial(_ptr(qb), _ptr(kb), _ptr(vb), int(j0), int(j1), dq, dv,
+                                float(scale), _ptr(o), _ptr(m), _ptr(l))
+    return torch.from_numpy(o), float(m[0]), float(l[0])
+
+
+def merge(o_parts, m_parts, l_parts, sink):
+    """Merge span partials, counting the sink once. Returns (o [dv], lse)."""
+    lib = _load()
+    op = np.ascontiguousarray(np.asarray(o_parts, np.float64))
+    mp = np.ascontiguousarray(np.asarray(m_parts, np.float64))
+    lp = np.ascontiguousarray(np.asarray(l_parts, np.float64))
+    nparts, dv = op.shape
+    o = np.zeros(dv, np.float64)
+    lse = np.zeros(1, np.float64)
+    lib.sinkattn_oracle_merge(_ptr(op), _ptr(mp), _ptr(lp), nparts, dv, float(sink), _ptr(o),
+                              _ptr(lse))
+    return torch.from_numpy(o), float(lse[0])
+
+
+def commit(kind, k_new, v_new, n_accept, k_cache, v_cache, *, ring_head=None, ring_len=None,
+           ctx_len=None, page_table=None, page_size=0):
+    """Append the first n_accept[b] new tokens of each sequence to the cache.
+
+    Returns new (k_cache, v_cache, ring_head, ring_len, ctx_len); inputs are not modified."""
+    lib = _load()
+    B, T, Hkv, dq = k_new.shape
+    dv = v_new.shape[3]
+    knb, vnb = _bits(k_new), _bits(v_new)
+    kcb, vcb = _bits(k_cache).copy(), _bits(v_cache).copy()
+    na = _i32(n_accept)
+    rh = None if ring_head is None else _i32(ring_head).copy()
+    rl = None if ring_len is None else _i32(ring_len).copy()
+    cl = None if ctx_len is None else _i32(ctx_len).copy()
+    pt = _i32(page_table)
+    ring_cap = k_cache.shape[1] if kind == KV_RING else 0
+    max_ctx = k_cache.shape[1] if kind == KV_CONTIG else 0
+    max_pages = pt.shape[1] if pt is not None else 0
+    rc = lib.sinkattn_oracle_commit(int(kind), _ptr(knb), _ptr(vnb), _ptr(na), _ptr(kcb), _ptr(vcb),
+                                    _ptr(rh), _ptr(rl), ring_cap, _ptr(cl), max_ctx, _ptr(pt),
+                                    int(page_size), max_pages, B, T, Hkv, dq, dv)
+    if rc != 0:
+        raise ValueError("oracle commit: bad arguments")
+
+    def back(a, like):
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).reshape(like.shape)
+
+    to_t = (lambda a: None if a is None else torch.from_numpy(a))
+    return back(kcb, k_cache), back(vcb, v_cache), to_t(rh), to_t(rl), to_t(cl)

@@ -1,0 +1,70 @@
+"""The oracle pins must catch plausible mistakes in the oracle.
+
+Each mutant is a copy of the oracle's C source with one plausible slip planted in it (a dropped
+term, an off-by-one window, a wrong head mapping, ...). It is compiled on the CPU and the pin
+suite is run against it; every mutant must make at least one pin fail.
+"""
+import os
+import subprocess
+import sys
+import tempfile
+from concurrent.futures import ThreadPoolExecutor
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "sinkattn_oracle.c")
+
+# (name, original text, replacement, occurrence index to replace)
+MUTANTS = [
+    ("sink dropped from the denominator", "double D = exp(sink - m);", "double D = 0.0;", 0),
+    ("sink scaled like a logit", "    double m = sink;\n    for (int j = 0; j < nkeys; ++j) {",
+     "    sink = sink * scale;\n    double m = sink;\n    for (int j = 0; j < nkeys; ++j) {", 0),
+    ("window one key too wide", "i - window + 1 > 0) ? i - window + 1", "i - window > 0) ? i - window", 0),
+    ("causal mask excludes the diagonal", "for (int j = lo; j <= i; ++j)", "for (int j = lo; j < i; ++j)", 0),
+    ("GQA head mapping h mod Hkv", "const int g = h / G;", "const int g = h % Hkv;", 0),
+    ("LSE in log2", "*lse = m + log(D);", "*lse = m + log2(D);", 0),
+    ("weights renormalised without the sink", "double w = exp(a[j] - m) / D;",
+     "double w = exp(a[j] - m) / (D - exp(sink - m));", 0),
+    ("scale dropped", "a[j] = scale * dot;", "a[j] = dot;", 0),
+    ("ring slot off by one", "(ring_head[b] + c) % ring_cap", "(ring_head[b] + c + 1) % ring_cap", 0),
+    ("new tokens not causal", "for (int u = 0; u <= t; ++u)", "for (int u = 0; u < T; ++u)", 0),
+    ("decode window off by one", "if (p > t || (window > 0 && p <= t - window))",
+     "if (p > t || (window > 0 && p < t - window))", 0),
+    ("merge counts the sink per span", "D += l_p[p] * exp(m_p[p] - m);",
+     "D += l_p[p] * exp(m_p[p] - m) + exp(sink - m);", 0),
+    ("paged row ignores the page size", "*\n                                      page_size + c % page_size;",
+     "+ c % page_size;", 0),
+    ("commit ring overwrites the newest", "slot = ring_head[b];\n", "slot = (ring_head[b] + ring_cap - 1) % ring_cap;\n", 0),
+]
+
+
+def _replace_nth(text, old, new, n):
+    idx = -1
+    for _ in range(n + 1):
+        idx = text.find(old, idx + 1)
+        assert idx >= 0, f"mutation anchor not found: {old!r}"
+    return text[:idx] + new + text[idx + len(old):]
+
+
+def _run_mutant(tmp, i, name, old, new, n):
+    src = open(SRC).read()
+    path_c = os.path.join(tmp, f"m{i}.c")
+    path_so = os.path.join(tmp, f"m{i}.so")
+    open(path_c, "w").write(_replace_nth(src, old, new, n))
+    subprocess.check_call(["gcc", "-O2", "-ffp-contract=off", "-fopenmp", "-shared", "-fPIC",
+                           "-std=c11", path_c, "-o", path_so, "-lm"])
+    env = dict(os.environ, SINKATTN_ORACLE_LIB=path_so, OMP_NUM_THREADS="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                        os.path.join(ROOT, "tests", "test_oracle_pins.py")],
+                       env=env, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    return name, r.returncode
+
+
+def test_every_mutant_is_caught():
+    with tempfile.TemporaryDirectory() as tmp:
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            results = list(ex.map(lambda a: _run_mutant(tmp, *a),
+                                  [(i,) + m for i, m in enumerate(MUTANTS)]))
+    survivors = [name for name, rc in results if rc == 0]
+    assert not survivors, f"mutants not caught by any pin: {survivors}"

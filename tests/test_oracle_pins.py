@@ -1,0 +1,401 @@
+"""Pins for the fp64 oracle: it is checked against things other than itself.
+
+* the worked example printed on the page "MiMo-V2-Flash Technical Report" (paper notes), §4.3
+  (tests/golden/worked_example.json), plus its closed form;
+* a library attention routine (torch scaled_dot_product_attention, fp64, CPU) when the sink is
+  -inf, which the pages say reduces to standard softmax ("MiMo-V2-Flash 架构 QA", Q3.7);
+* the eager concat -> softmax -> drop formulation ("MiMo-V2-Flash 模型架构深度拆解", CH10.1 and
+  "MiMo-V2-Flash 架构 QA", Q3.8) built from library softmax / logsumexp;
+* invariants the mathematics fixes: weights + sink share = 1, shift invariance, SWA == GA when
+  the window covers the sequence, GQA == MHA with repeated K/V, decode == prefill of the
+  concatenated sequence, ring / paged caches == the contiguous cache, split + merge == direct.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from global_attention_sink_softmax_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_example.json")
+pytestmark = pytest.mark.filterwarnings("ignore")
+
+
+def bf(x):
+    return torch.as_tensor(x, dtype=torch.float32).to(torch.bfloat16)
+
+
+def rand_bf16(shape, g):
+    return torch.randn(shape, generator=g).to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------------------------
+# the worked example (paper notes §4.3)
+# ----------------------------------------------------------------------------------------------
+
+def worked_example_inputs(L, n_keys_logit, window):
+    """All logits equal 2 (scale 1: q = 2 e0, k_j = e0), sink 4, v_j = e_(j mod 128)."""
+    dq, dv = 192, 128
+    q = torch.zeros(1, L, 1, dq)
+    q[..., 0] = n_keys_logit
+    k = torch.zeros(1, L, 1, dq)
+    k[..., 0] = 1.0
+    v = torch.zeros(1, L, 1, dv)
+    for j in range(L):
+        v[0, j, 0, j % dv] = 1.0
+    return bf(q), bf(k), bf(v), torch.tensor([4.0])
+
+
+@pytest.mark.parametrize("L,row,window", [(128, 127, 128), (128, 127, 0), (256, 200, 128),
+                                          (300, 299, 128)])
+def test_worked_example_printed_numbers(L, row, window):
+    gold = json.load(open(GOLDEN))
+    p, tol = gold["printed"], gold["printed_half_ulp"]
+    q, k, v, sink = worked_example_inputs(L, gold["inputs"]["logit"], window)
+    o, lse, ws = oracle.prefill(q, k, v, sink, scale=1.0, window=window,
+                                rows=[[0, row]], want_wsink=True)
+    weights = o[0, 0]                     # v is one-hot, so O is the weight vector
+    lse = float(lse[0, 0])
+    m = 4.0                               # the page: m = max(max(0..2), 4) = 4
+    D = math.exp(lse - m)                 # LSE = m + ln D
+    nz = weights[weights > 0]
+    # exactly 128 keys are visible: the window holds 128 keys including the query
+    assert nz.numel() == gold["inputs"]["n_keys"]
+    checks = {
+        "denominator": D,
+        "per_key_weight": float(nz.max()),
+        "weights_sum": float(weights.sum()),
+        "sink_share": float(ws[0, 0]),
+        "per_key_numerator": float(nz.max()) * D,
+        "sink_numerator": float(ws[0, 0]) * D,
+        "m": m,
+    }
+    for key, val in checks.items():
+        assert abs(val - p[key]) <= tol[key] + 1e-12, (key, val, p[key])
+    # closed form: D = 1 + 128 e^-2, w_j = e^-2 / D, w_s = 1 / D
+    Dx = 1.0 + 128.0 * math.exp(-2.0)
+    assert abs(D - Dx) < 1e-12
+    assert torch.allclose(nz, torch.full_like(nz, math.exp(-2.0) / Dx), rtol=0, atol=1e-15)
+    assert abs(float(ws[0, 0]) - 1.0 / Dx) < 1e-15
+
+
+def test_worked_example_bound_for_logits_in_0_2():
+    """Logits anywhere in [0, 2] with sink 4: 1 + 128 e^-4 <= D <= 1 + 128 e^-2 (paper notes
+    §4.3 bounds each numerator term by exp(-2))."""
+    g = torch.Generator().manual_seed(7)
+    L, dq, dv = 128, 192, 128
+    u = torch.rand(L, generator=g) * 2.0
+    q = torch.zeros(1, L, 1, dq)
+    q[..., 0] = 1.0
+    k = torch.zeros(1, L, 1, dq)
+    k[0, :, 0, 0] = u
+    v = rand_bf16((1, L, 1, dv), g)
+    o, lse, ws = oracle.prefill(bf(q), bf(k), v, torch.tensor([4.0]), scale=1.0, window=128,
+                                rows=[[0, L - 1]], want_wsink=True)
+    D = math.exp(float(lse[0, 0]) - 4.0)
+    assert 1 + 128 * math.exp(-4) - 1e-12 <= D <= 1 + 128 * math.exp(-2) + 1e-12
+    # and it is exact for the drawn logits (they are bf16-rounded)
+    a = bf(u).double()
+    assert abs(D - (1 + torch.exp(a - 4).sum().item())) < 1e-12
+
+
+# ----------------------------------------------------------------------------------------------
+# library routines
+# ----------------------------------------------------------------------------------------------
+
+def band_mask(L, window):
+    i = torch.arange(L)[:, None]
+    j = torch.arange(L)[None, :]
+    keep = j <= i
+    if window > 0:
+        keep &= j > i - window
+    return keep
+
+
+def to_bhld(x):
+    return x.double().permute(0, 2, 1, 3)
+
+
+@pytest.mark.parametrize("B,L,Hq,Hkv,window", [(2, 37, 4, 2, 0), (1, 70, 8, 1, 16),
+                                               (2, 33, 6, 3, 5), (1, 129, 4, 4, 128)])
+def test_no_sink_equals_library_attention(B, L, Hq, Hkv, window):
+    """sink = -inf (and sink = NULL) reduce to standard softmax (QA Q3.7): compare with torch
+    scaled_dot_product_attention in fp64 (GQA via enable_gqa, head h -> KV head h // G)."""
+    g = torch.Generator().manual_seed(11)
+    dq, dv = 192, 128
+    q, k, v = rand_bf16((B, L, Hq, dq), g), rand_bf16((B, L, Hkv, dq), g), rand_bf16((B, L, Hkv, dv), g)
+    scale = 1.0 / math.sqrt(dq)
+    mask = band_mask(L, window)
+    ref = F.scaled_dot_product_attention(to_bhld(q), to_bhld(k), to_bhld(v), attn_mask=mask,
+                                         scale=scale, enable_gqa=True).permute(0, 2, 1, 3)
+    scores = torch.matmul(to_bhld(q), to_bhld(k).repeat_interleave(Hq // Hkv, 1).transpose(-1, -2))
+    scores = (scores * scale).masked_fill(~mask, float("-inf"))
+    ref_lse = torch.logsumexp(scores, dim=-1).permute(0, 2, 1)
+    for sink in (None, torch.full((Hq,), float("-inf"))):
+        o, lse, _ = oracle.prefill(q, k, v, sink, scale, window)
+        assert torch.allclose(o, ref, rtol=0, atol=1e-12)
+        assert torch.allclose(lse, ref_lse, rtol=0, atol=1e-12)
+
+
+def eager_sink_attention(q, k, v, sink, scale, window):
+    """The pages' eager formulation: scaled, masked scores; append the per-head sink as one
+    more column; softmax over S+1; drop the sink column; multiply by V."""
+    B, L, Hq, _ = q.shape
+    G = Hq // k.shape[2]
+    qq, kk, vv = to_bhld(q), to_bhld(k).repeat_interleave(G, 1), to_bhld(v).repeat_interleave(G, 1)
+    scores = torch.matmul(qq, kk.transpose(-1, -2)) * scale
+    scores = scores.masked_fill(~band_mask(L, window), float("-inf"))
+    s = sink.double().reshape(1, Hq, 1, 1).expand(B, Hq, L, 1)
+    cat = torch.cat([scores, s], dim=-1)
+    probs = torch.softmax(cat, dim=-1)[..., :-1]
+    out = torch.matmul(probs, vv).permute(0, 2, 1, 3)
+    lse = torch.logsumexp(cat, dim=-1).permute(0, 2, 1)
+    wsink = torch.softmax(cat, dim=-1)[..., -1].permute(0, 2, 1)
+    return out, lse, wsink
+
+
+@pytest.mark.parametrize("B,L,Hq,Hkv,window,scale", [
+    (1, 64, 8, 1, 128, 1 / math.sqrt(192)),
+    (2, 50, 4, 2, 0, 1 / math.sqrt(192)),
+    (1, 200, 4, 1, 128, 1 / math.sqrt(192)),
+    (1, 40, 2, 1, 7, 0.37),           # scale != 1 separates "sink in post-scale units"
+])
+def test_equals_eager_concat_softmax_drop(B, L, Hq, Hkv, window, scale):
+    g = torch.Generator().manual_seed(13)
+    dq, dv = 192, 128
+    q, k, v = rand_bf16((B, L, Hq, dq), g), rand_bf16((B, L, Hkv, dq), g), rand_bf16((B, L, Hkv, dv), g)
+    sink = torch.rand(Hq, generator=g) * 6.0
+    sink[0] = float("-inf")
+    o, lse, ws = oracle.prefill(q, k, v, sink, scale, window, want_wsink=True)
+    ro, rl, rw = eager_sink_attention(q, k, v, sink, scale, window)
+    assert torch.allclose(o, ro, rtol=0, atol=1e-12)
+    assert torch.allclose(lse, rl, rtol=0, atol=1e-12)
+    assert torch.allclose(ws, rw, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------------------------
+# invariants
+# ----------------------------------------------------------------------------------------------
+
+def test_weights_plus_sink_share_is_one():
+    """The kept weights sum to 1 - (sink share) (QA Q3.8: the sink's mass is dropped)."""
+    g = torch.Generator().manual_seed(17)
+    L, dq, dv = 128, 192, 128
+    q, k = rand_bf16((1, L, 4, dq), g), rand_bf16((1, L, 2, dq), g)
+    v = torch.eye(L, dv).reshape(1, L, 1, dv).repeat(1, 1, 2, 1).to(torch.bfloat16)
+    sink = torch.tensor([0.0, 3.0, 6.0, float("-inf")])
+    for window in (0, 128, 31):
+        o, lse, ws = oracle.prefill(q, k, v, sink, 1 / math.sqrt(dq), window, want_wsink=True)
+        total = o.sum(-1) + ws
+        assert torch.allclose(total, torch.ones_like(total), rtol=0, atol=1e-12)
+        assert (ws[..., 3] == 0).all()          # -inf sink takes no mass
+        assert (ws[..., :3] > 0).all()
+
+
+def test_shift_invariance():
+    """Adding c to every logit and to the sink leaves O unchanged and adds c to LSE."""
+    g = torch.Generator().manual_seed(19)
+    L, dq, dv, c = 40, 16, 128, 3.0
+    q, k, v = rand_bf16((1, L, 2, dq), g), rand_bf16((1, L, 1, dq), g), rand_bf16((1, L, 1, dv), g)
+    sink = torch.tensor([1.5, 5.0])
+    o, lse, _ = oracle.prefill(q, k, v, sink, 1.0, 0)
+    q2 = torch.cat([q, torch.ones(1, L, 2, 1, dtype=torch.bfloat16)], -1)
+    k2 = torch.cat([k, torch.full((1, L, 1, 1), c, dtype=torch.bfloat16)], -1)
+    o2, lse2, _ = oracle.prefill(q2, k2, v, sink + c, 1.0, 0)
+    assert torch.allclose(o2, o, rtol=0, atol=1e-12)
+    assert torch.allclose(lse2, lse + c, rtol=0, atol=1e-12)
+
+
+def test_swa_equals_ga_when_window_covers_sequence():
+    g = torch.Generator().manual_seed(23)
+    L = 100
+    q, k, v = rand_bf16((2, L, 4, 192), g), rand_bf16((2, L, 2, 192), g), rand_bf16((2, L, 2, 128), g)
+    sink = torch.rand(4, generator=g) * 6
+    a = oracle.prefill(q, k, v, sink, 0.07, 0)
+    for window in (L, L + 1, 4096):
+        b = oracle.prefill(q, k, v, sink, 0.07, window)
+        assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+    c = oracle.prefill(q, k, v, sink, 0.07, L - 1)
+    assert not torch.equal(a[0], c[0])
+
+
+def test_gqa_equals_mha_with_repeated_kv():
+    g = torch.Generator().manual_seed(29)
+    L, Hq, Hkv = 30, 8, 2
+    q, k, v = rand_bf16((1, L, Hq, 192), g), rand_bf16((1, L, Hkv, 192), g), rand_bf16((1, L, Hkv, 128), g)
+    sink = torch.rand(Hq, generator=g) * 6
+    a = oracle.prefill(q, k, v, sink, 0.07, 9)
+    G = Hq // Hkv
+    b = oracle.prefill(q, k.repeat_interleave(G, 2), v.repeat_interleave(G, 2), sink, 0.07, 9)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_row_sampling_matches_full():
+    g = torch.Generator().manual_seed(31)
+    q, k, v = rand_bf16((2, 50, 4, 192), g), rand_bf16((2, 50, 1, 192), g), rand_bf16((2, 50, 1, 128), g)
+    sink = torch.rand(4, generator=g) * 6
+    full = oracle.prefill(q, k, v, sink, 0.07, 16)
+    rows = [[1, 0], [0, 49], [1, 17]]
+    part = oracle.prefill(q, k, v, sink, 0.07, 16, rows=rows)
+    for n, (b, i) in enumerate(rows):
+        assert torch.equal(part[0][n], full[0][b, i]) and torch.equal(part[1][n], full[1][b, i])
+
+
+# ----------------------------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------------------------
+
+def concat_prefill_rows(k_cache_seq, v_cache_seq, q, k_new, v_new, sink, scale, window):
+    """Prefill of [cached tokens ++ new tokens]; returns the rows of the new tokens."""
+    n = k_cache_seq.shape[0]
+    T, Hq, dq = q.shape
+    Hkv = k_new.shape[1]
+    L = n + T
+    qq = torch.zeros(1, L, Hq, dq, dtype=torch.bfloat16)
+    qq[0, n:] = q
+    kk = torch.cat([k_cache_seq, k_new], 0)[None]
+    vv = torch.cat([v_cache_seq, v_new], 0)[None]
+    rows = [[0, n + t] for t in range(T)]
+    o, lse, _ = oracle.prefill(qq, kk, vv, sink, scale, window, rows=rows)
+    return o, lse
+
+
+@pytest.mark.parametrize("T,window", [(1, 0), (4, 0), (1, 128), (4, 128), (3, 7)])
+def test_decode_contig_equals_prefill_of_concatenation(T, window):
+    g = torch.Generator().manual_seed(37)
+    B, Hq, Hkv, maxc = 3, 4, 2, 300
+    q = rand_bf16((B, T, Hq, 192), g)
+    kn, vn = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    kc, vc = rand_bf16((B, maxc, Hkv, 192), g), rand_bf16((B, maxc, Hkv, 128), g)
+    ctx = torch.tensor([0, 129, 300], dtype=torch.int32)
+    sink = torch.rand(Hq, generator=g) * 6
+    o, lse, _ = oracle.decode(oracle.KV_CONTIG, q, kn, vn, kc, vc, sink, 0.07, window, ctx_len=ctx)
+    for b in range(B):
+        n = int(ctx[b])
+        ro, rl = concat_prefill_rows(kc[b, :n], vc[b, :n], q[b], kn[b], vn[b], sink, 0.07, window)
+        assert torch.equal(o[b], ro) and torch.equal(lse[b], rl)
+
+
+@pytest.mark.parametrize("T", [1, 2, 4])
+def test_decode_ring_equals_contig_tail(T):
+    """A 128-slot ring with head h holds the last ring_len tokens, oldest at slot h."""
+    g = torch.Generator().manual_seed(41)
+    B, Hq, Hkv, cap, W = 4, 8, 2, 128, 128
+    q = rand_bf16((B, T, Hq, 192), g)
+    kn, vn = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    ring_len = torch.tensor([128, 5, 128, 0], dtype=torch.int32)
+    ring_head = torch.tensor([77, 3, 0, 9], dtype=torch.int32)
+    hist = [rand_bf16((int(n), Hkv, 192), g) for n in ring_len]   # tokens oldest first
+    histv = [rand_bf16((int(n), Hkv, 128), g) for n in ring_len]
+    kc = torch.zeros(B, cap, Hkv, 192, dtype=torch.bfloat16)
+    vc = torch.zeros(B, cap, Hkv, 128, dtype=torch.bfloat16)
+    for b in range(B):
+        for c in range(int(ring_len[b])):
+            kc[b, (int(ring_head[b]) + c) % cap] = hist[b][c]
+            vc[b, (int(ring_head[b]) + c) % cap] = histv[b][c]
+    sink = torch.rand(Hq, generator=g) * 6
+    o, lse, _ = oracle.decode(oracle.KV_RING, q, kn, vn, kc, vc, sink, 0.07, W,
+                              ring_head=ring_head, ring_len=ring_len)
+    for b in range(B):
+        ro, rl = concat_prefill_rows(hist[b], histv[b], q[b], kn[b], vn[b], sink, 0.07, W)
+        assert torch.equal(o[b], ro) and torch.equal(lse[b], rl)
+
+
+def test_decode_paged_equals_contig():
+    g = torch.Generator().manual_seed(43)
+    B, T, Hq, Hkv, P = 3, 2, 4, 1, 16
+    ctx = torch.tensor([1, 40, 64], dtype=torch.int32)
+    maxc = 64
+    q = rand_bf16((B, T, Hq, 192), g)
+    kn, vn = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    kc, vc = rand_bf16((B, maxc, Hkv, 192), g), rand_bf16((B, maxc, Hkv, 128), g)
+    max_pages = maxc // P
+    perm = torch.randperm(B * max_pages, generator=g).to(torch.int32)
+    table = perm.reshape(B, max_pages)
+    kp = torch.zeros(B * max_pages, P, Hkv, 192, dtype=torch.bfloat16)
+    vp = torch.zeros(B * max_pages, P, Hkv, 128, dtype=torch.bfloat16)
+    for b in range(B):
+        for c in range(maxc):
+            kp[table[b, c // P], c % P] = kc[b, c]
+            vp[table[b, c // P], c % P] = vc[b, c]
+    sink = torch.rand(Hq, generator=g) * 6
+    a = oracle.decode(oracle.KV_CONTIG, q, kn, vn, kc, vc, sink, 0.07, 0, ctx_len=ctx)
+    b_ = oracle.decode(oracle.KV_PAGED, q, kn, vn, kp, vp, sink, 0.07, 0, ctx_len=ctx,
+                       page_table=table, page_size=P)
+    assert torch.equal(a[0], b_[0]) and torch.equal(a[1], b_[1])
+
+
+def test_decode_seq_sampling():
+    w = W.SWA_DECODE
+    d = W.decode_inputs(w, B=6)
+    full = oracle.decode(w.kind, d["q"], d["k_new"], d["v_new"], d["k_cache"], d["v_cache"],
+                         d["sink"], W.SCALE, w.window, ring_head=d["ring_head"], ring_len=d["ring_len"])
+    part = oracle.decode(w.kind, d["q"], d["k_new"], d["v_new"], d["k_cache"], d["v_cache"],
+                         d["sink"], W.SCALE, w.window, ring_head=d["ring_head"],
+                         ring_len=d["ring_len"], seqs=[4, 1])
+    assert torch.equal(part[0][0], full[0][4]) and torch.equal(part[0][1], full[0][1])
+
+
+# ----------------------------------------------------------------------------------------------
+# split-KV algebra and the cache commit
+# ----------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("cuts", [[0, 200], [0, 1, 200], [0, 64, 64, 128, 199, 200],
+                                  [0, 13, 50, 77, 140, 200]])
+def test_split_merge_equals_direct_and_counts_sink_once(cuts):
+    g = torch.Generator().manual_seed(47)
+    n = cuts[-1]
+    q = rand_bf16((1, n, 1, 192), g)
+    k, v = rand_bf16((1, n, 1, 192), g), rand_bf16((1, n, 1, 128), g)
+    sink = torch.tensor([4.5])
+    o, lse, _ = oracle.prefill(q, k, v, sink, 0.07, 0, rows=[[0, n - 1]])
+    parts = [oracle.partial(q[0, n - 1, 0], k[0, :, 0], v[0, :, 0], a, b, 0.07)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    mo, ml = oracle.merge([p[0].numpy() for p in parts], [p[1] for p in parts],
+                          [p[2] for p in parts], 4.5)
+    assert torch.allclose(mo, o[0, 0], rtol=0, atol=1e-12)
+    assert abs(ml - float(lse[0, 0])) < 1e-12
+    # counting the sink once per span would be wrong: check the merge is not that
+    wrong = math.log(math.exp(ml) + (len(parts) - 1) * math.exp(4.5))
+    assert len(parts) == 1 or abs(wrong - ml) > 1e-6
+
+
+def test_commit_ring_and_contig_semantics():
+    g = torch.Generator().manual_seed(53)
+    B, T, Hkv, cap = 3, 4, 2, 8
+    kn, vn = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    kc, vc = rand_bf16((B, cap, Hkv, 192), g), rand_bf16((B, cap, Hkv, 128), g)
+    head = torch.tensor([6, 0, 2], dtype=torch.int32)
+    ln = torch.tensor([8, 5, 7], dtype=torch.int32)
+    acc = torch.tensor([3, 4, 0], dtype=torch.int32)
+    k2, v2, h2, l2, _ = oracle.commit(oracle.KV_RING, kn, vn, acc, kc, vc, ring_head=head, ring_len=ln)
+    for b in range(B):
+        before = [kc[b, (int(head[b]) + c) % cap] for c in range(int(ln[b]))]
+        seq = before + [kn[b, u] for u in range(int(acc[b]))]
+        want = seq[-cap:]
+        assert int(l2[b]) == len(want)
+        got = [k2[b, (int(h2[b]) + c) % cap] for c in range(int(l2[b]))]
+        assert all(torch.equal(x, y) for x, y in zip(got, want))
+    ctx = torch.tensor([0, 3, 10], dtype=torch.int32)
+    kc3, vc3 = rand_bf16((B, 16, Hkv, 192), g), rand_bf16((B, 16, Hkv, 128), g)
+    k3, v3, _, _, c3 = oracle.commit(oracle.KV_CONTIG, kn, vn, acc, kc3, vc3, ctx_len=ctx)
+    for b in range(B):
+        assert int(c3[b]) == int(ctx[b]) + int(acc[b])
+        assert torch.equal(k3[b, :int(ctx[b])], kc3[b, :int(ctx[b])])
+        assert torch.equal(k3[b, int(ctx[b]):int(c3[b])], kn[b, :int(acc[b])])
+        assert torch.equal(v3[b, int(ctx[b]):int(c3[b])], vn[b, :int(acc[b])])
+        assert torch.equal(k3[b, int(c3[b]):], kc3[b, int(c3[b]):])
+
+
+def test_workload_generators_are_seeded():
+    a = W.prefill_inputs(W.SWA_PREFILL_SMALL, L=64)
+    b = W.prefill_inputs(W.SWA_PREFILL_SMALL, L=64)
+    assert all(torch.equal(a[x], b[x]) for x in a)
+    s = W.prefill_inputs(W.GA_PREFILL, L=8)["sink"]
+    assert torch.isinf(s[7::8]).all() and torch.isfinite(s[0::8]).all()
+    assert float(s[torch.isfinite(s)].min()) >= 0 and float(s[torch.isfinite(s)].max()) <= 6
