@@ -1,0 +1,316 @@
+"""Sink-softmax GQA attention for NVIDIA B200: a thin ctypes binding over ``libsinkattn.so``.
+
+The functions carry the names of the C entry points declared in ``include/sinkattn.h`` and only
+marshal arguments: torch tensors supply device memory and the current CUDA stream, and every
+step of the computation runs in the library's CUDA kernels. There is no fallback: if the
+library is missing or cannot be loaded, every call raises.
+
+    o, lse = sinkattn_prefill_swa(q, k, v, sink, window=128)
+    o, lse = sinkattn_prefill_ga(q, k, v, sink)
+    o, lse = sinkattn_decode(KV_CONTIG, q, k_new, v_new, k_cache, v_cache, sink, ctx_len=...)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+
+import torch
+
+from . import workloads  # noqa: F401  (seeded inputs; no attention arithmetic)
+
+__all__ = [
+    "KV_RING", "KV_CONTIG", "KV_PAGED", "SinkAttnError", "lib", "library_path",
+    "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_decode",
+    "sinkattn_decode_workspace_size", "sinkattn_kv_commit", "sinkattn_take_device_error",
+    "sinkattn_status_string", "sinkattn_version", "EXPORTED_SYMBOLS",
+]
+
+KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
+DQ, DV = 192, 128
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libsinkattn.so")
+EXPORTED_SYMBOLS = [
+    "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_decode_workspace_size",
+    "sinkattn_decode", "sinkattn_kv_commit", "sinkattn_status_string", "sinkattn_version",
+    "sinkattn_take_device_error",
+]
+
+
+class SinkAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {sinkattn_status_string(status)} (status {status})")
+
+
+_P, _I32, _I64, _F32, _SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+
+
+class PrefillArgs(ctypes.Structure):
+    _fields_ = [("q", _P), ("k", _P), ("v", _P), ("sink", _P), ("o", _P), ("lse", _P),
+                ("B", _I32), ("L", _I32), ("Hq", _I32), ("Hkv", _I32), ("dq", _I32),
+                ("dv", _I32), ("scale", _F32),
+                ("q_sb", _I64), ("q_sl", _I64), ("q_sh", _I64),
+                ("k_sb", _I64), ("k_sl", _I64), ("k_sh", _I64),
+                ("v_sb", _I64), ("v_sl", _I64), ("v_sh", _I64),
+                ("o_sb", _I64), ("o_sl", _I64), ("o_sh", _I64)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("kind", _I32), ("B", _I32), ("T", _I32), ("Hq", _I32), ("Hkv", _I32),
+                ("dq", _I32), ("dv", _I32), ("window", _I32), ("scale", _F32), ("sink", _P),
+                ("q", _P), ("q_sb", _I64), ("q_st", _I64), ("q_sh", _I64),
+                ("k_new", _P), ("kn_sb", _I64), ("kn_st", _I64), ("kn_sh", _I64),
+                ("v_new", _P), ("vn_sb", _I64), ("vn_st", _I64), ("vn_sh", _I64),
+                ("k_cache", _P), ("kc_sb", _I64), ("kc_ss", _I64), ("kc_sh", _I64),
+                ("v_cache", _P), ("vc_sb", _I64), ("vc_ss", _I64), ("vc_sh", _I64),
+                ("ring_head", _P), ("ring_len", _P), ("ring_cap", _I32),
+                ("ctx_len", _P), ("max_ctx", _I32),
+                ("page_table", _P), ("page_size", _I32), ("max_pages", _I32),
+                ("num_pages", _I32),
+                ("o", _P), ("o_sb", _I64), ("o_st", _I64), ("o_sh", _I64), ("lse", _P)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library. Raises if it has not been built or cannot be loaded."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise RuntimeError(
+                    f"{library_path} is missing: build it with "
+                    "`python -m global_attention_sink_softmax_b200.build` (needs nvcc)")
+            L = ctypes.CDLL(library_path)
+            L.sinkattn_prefill_swa.argtypes = [ctypes.POINTER(PrefillArgs), _I32, _P]
+            L.sinkattn_prefill_swa.restype = ctypes.c_int
+            L.sinkattn_prefill_ga.argtypes = [ctypes.POINTER(PrefillArgs), _P]
+            L.sinkattn_prefill_ga.restype = ctypes.c_int
+            L.sinkattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]
+            L.sinkattn_decode_workspace_size.restype = _SZ
+            L.sinkattn_decode.argtypes = [ctypes.POINTER(DecodeArgs), _P, _SZ, _P]
+            L.sinkattn_decode.restype = ctypes.c_int
+            L.sinkattn_kv_commit.argtypes = [ctypes.POINTER(DecodeArgs), _P, _P]
+            L.sinkattn_kv_commit.restype = ctypes.c_int
+            L.sinkattn_status_string.argtypes = [ctypes.c_int]
+            L.sinkattn_status_string.restype = ctypes.c_char_p
+            L.sinkattn_version.argtypes = []
+            L.sinkattn_version.restype = ctypes.c_int
+            L.sinkattn_take_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+            L.sinkattn_take_device_error.restype = ctypes.c_int
+            _lib = L
+    return _lib
+
+
+def sinkattn_status_string(status: int) -> str:
+    return lib().sinkattn_status_string(int(status)).decode()
+
+
+def sinkattn_version() -> int:
+    return int(lib().sinkattn_version())
+
+
+# ----------------------------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------------------------
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if isinstance(stream, torch.cuda.Stream) else int(stream))
+
+
+def _check_bf16(name, t, ndim=4):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != ndim or t.stride(-1) != 1:
+        raise ValueError(f"{name} must be {ndim}-D with a contiguous last dim")
+
+
+def _check_vec(name, t, dtype):
+    if t is None:
+        return
+    if t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} tensor")
+
+
+def _raise(status, where):
+    if status != 0:
+        raise SinkAttnError(status, where)
+
+
+# ----------------------------------------------------------------------------------------------
+# prefill
+# ----------------------------------------------------------------------------------------------
+
+def _prefill_args(q, k, v, sink, o, lse, scale):
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _check_bf16(n, t)
+    _check_vec("sink", sink, torch.float32)
+    _check_vec("lse", lse, torch.float32)
+    B, L, Hq, dq = q.shape
+    a = PrefillArgs()
+    a.q, a.k, a.v, a.sink, a.o, a.lse = (_ptr(q), _ptr(k), _ptr(v), _ptr(sink), _ptr(o),
+                                         _ptr(lse))
+    a.B, a.L, a.Hq, a.Hkv, a.dq, a.dv = B, L, Hq, k.shape[2], dq, v.shape[3]
+    a.scale = scale
+    a.q_sb, a.q_sl, a.q_sh = q.stride(0), q.stride(1), q.stride(2)
+    a.k_sb, a.k_sl, a.k_sh = k.stride(0), k.stride(1), k.stride(2)
+    a.v_sb, a.v_sl, a.v_sh = v.stride(0), v.stride(1), v.stride(2)
+    a.o_sb, a.o_sl, a.o_sh = o.stride(0), o.stride(1), o.stride(2)
+    return a
+
+
+def _prefill(fn, q, k, v, sink, window, o, lse, scale, stream, want_lse):
+    B, L, Hq, dq = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dq)
+    if o is None:
+        o = torch.empty(B, L, Hq, v.shape[3], dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device)
+    a = _prefill_args(q, k, v, sink, o, lse, scale)
+    L_ = lib()
+    if fn == "swa":
+        st = L_.sinkattn_prefill_swa(ctypes.byref(a), int(window), _stream(stream))
+    else:
+        st = L_.sinkattn_prefill_ga(ctypes.byref(a), _stream(stream))
+    _raise(st, f"sinkattn_prefill_{fn}")
+    return o, lse
+
+
+def sinkattn_prefill_swa(q, k, v, sink=None, window=128, *, o=None, lse=None, scale=None,
+                         stream=None, want_lse=True):
+    """Sliding-window sink attention over whole sequences.
+
+    q [B,L,Hq,192], k [B,L,Hkv,192], v [B,L,Hkv,128] bf16 CUDA tensors (token-major, any
+    strides with a contiguous last dim); sink fp32 [Hq] or None. Returns (o [B,L,Hq,128] bf16,
+    lse [B,Hq,L] fp32 or None)."""
+    return _prefill("swa", q, k, v, sink, window, o, lse, scale, stream, want_lse)
+
+
+def sinkattn_prefill_ga(q, k, v, sink=None, *, o=None, lse=None, scale=None, stream=None,
+                        want_lse=True):
+    """Global (full causal) sink attention over whole sequences; arguments as for SWA."""
+    return _prefill("ga", q, k, v, sink, 0, o, lse, scale, stream, want_lse)
+
+
+# ----------------------------------------------------------------------------------------------
+# decode
+# ----------------------------------------------------------------------------------------------
+
+def _decode_args(kind, q, k_new, v_new, k_cache, v_cache, sink, window, scale, ring_head,
+                 ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse):
+    for n, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                 ("v_cache", v_cache)):
+        _check_bf16(n, t)
+    if o is not None:
+        _check_bf16("o", o)
+    _check_vec("sink", sink, torch.float32)
+    _check_vec("lse", lse, torch.float32)
+    for n, t in (("ring_head", ring_head), ("ring_len", ring_len), ("ctx_len", ctx_len)):
+        _check_vec(n, t, torch.int32)
+    if page_table is not None and (page_table.dtype != torch.int32 or not page_table.is_cuda
+                                   or not page_table.is_contiguous() or page_table.dim() != 2):
+        raise ValueError("page_table must be a contiguous 2-D CUDA int32 tensor")
+    B, T, Hq, dq = q.shape
+    a = DecodeArgs()
+    a.kind, a.B, a.T, a.Hq, a.Hkv, a.dq, a.dv = kind, B, T, Hq, k_new.shape[2], dq, v_new.shape[3]
+    a.window, a.scale, a.sink = int(window), scale, _ptr(sink)
+    a.q, a.q_sb, a.q_st, a.q_sh = _ptr(q), q.stride(0), q.stride(1), q.stride(2)
+    a.k_new, a.kn_sb, a.kn_st, a.kn_sh = _ptr(k_new), k_new.stride(0), k_new.stride(1), k_new.stride(2)
+    a.v_new, a.vn_sb, a.vn_st, a.vn_sh = _ptr(v_new), v_new.stride(0), v_new.stride(1), v_new.stride(2)
+    a.k_cache, a.kc_sb, a.kc_ss, a.kc_sh = (_ptr(k_cache), k_cache.stride(0), k_cache.stride(1),
+                                            k_cache.stride(2))
+    a.v_cache, a.vc_sb, a.vc_ss, a.vc_sh = (_ptr(v_cache), v_cache.stride(0), v_cache.stride(1),
+                                            v_cache.stride(2))
+    a.ring_head, a.ring_len = _ptr(ring_head), _ptr(ring_len)
+    a.ring_cap = k_cache.shape[1] if kind == KV_RING else 0
+    a.ctx_len = _ptr(ctx_len)
+    if max_ctx is None:
+        if kind == KV_CONTIG:
+            max_ctx = k_cache.shape[1]
+        elif kind == KV_PAGED:
+            max_ctx = page_table.shape[1] * k_cache.shape[1]
+        else:
+            max_ctx = 0
+    a.max_ctx = int(max_ctx)
+    a.page_table = _ptr(page_table)
+    a.page_size = k_cache.shape[1] if kind == KV_PAGED else int(page_size or 0)
+    a.max_pages = page_table.shape[1] if page_table is not None else 0
+    a.num_pages = (k_cache.shape[0] if num_pages is None else int(num_pages)) if kind == KV_PAGED else 0
+    if o is not None:
+        a.o, a.o_sb, a.o_st, a.o_sh = _ptr(o), o.stride(0), o.stride(1), o.stride(2)
+    a.lse = _ptr(lse)
+    return a
+
+
+def sinkattn_decode_workspace_size(kind, q, k_new, v_new, k_cache, v_cache, *, window=0,
+                                   ring_head=None, ring_len=None, ctx_len=None, max_ctx=None,
+                                   page_table=None, page_size=None, num_pages=None) -> int:
+    a = _decode_args(kind, q, k_new, v_new, k_cache, v_cache, None, window, 1.0, ring_head,
+                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, None, None)
+    return int(lib().sinkattn_decode_workspace_size(ctypes.byref(a)))
+
+
+def sinkattn_decode(kind, q, k_new, v_new, k_cache, v_cache, sink=None, *, window=0,
+                    ring_head=None, ring_len=None, ctx_len=None, max_ctx=None, page_table=None,
+                    page_size=None, num_pages=None, o=None, lse=None, workspace=None,
+                    scale=None, stream=None, want_lse=True):
+    """Decode / speculative verify of T (1..4) new tokens per sequence against a KV cache.
+
+    kind: KV_RING (k_cache [B,cap,Hkv,192] with ring_head/ring_len int32 [B]), KV_CONTIG
+    (k_cache [B,max_ctx,Hkv,192] with ctx_len [B]) or KV_PAGED (k_cache [pages,page,Hkv,192]
+    with page_table [B,max_pages] and ctx_len [B]). The new tokens' K/V are not in the cache.
+    Returns (o [B,T,Hq,128] bf16, lse [B,T,Hq] fp32 or None)."""
+    B, T, Hq, dq = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dq)
+    if o is None:
+        o = torch.empty(B, T, Hq, v_new.shape[3], dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, T, Hq, dtype=torch.float32, device=q.device)
+    a = _decode_args(kind, q, k_new, v_new, k_cache, v_cache, sink, window, scale, ring_head,
+                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse)
+    L_ = lib()
+    need = int(L_.sinkattn_decode_workspace_size(ctypes.byref(a)))
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if need > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if need > 0 else 0
+    st = L_.sinkattn_decode(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream))
+    _raise(st, "sinkattn_decode")
+    return o, lse
+
+
+def sinkattn_kv_commit(kind, k_new, v_new, n_accept, k_cache, v_cache, *, ring_head=None,
+                       ring_len=None, ctx_len=None, max_ctx=None, page_table=None,
+                       num_pages=None, stream=None):
+    """Append the first n_accept[b] of each sequence's T new tokens to its cache, in place."""
+    _check_vec("n_accept", n_accept, torch.int32)
+    B, T, Hkv, dq = k_new.shape
+    q_dummy = k_new  # only the cache-related fields are read
+    a = _decode_args(kind, q_dummy, k_new, v_new, k_cache, v_cache, None, 0, 1.0, ring_head,
+                     ring_len, ctx_len, max_ctx, page_table, None, num_pages, None, None)
+    st = lib().sinkattn_kv_commit(ctypes.byref(a), _ptr(n_accept), _stream(stream))
+    _raise(st, "sinkattn_kv_commit")
+
+
+def sinkattn_take_device_error() -> int:
+    """Reads and clears the kernels' wait-timeout flag (synchronises the device)."""
+    flag = ctypes.c_uint32(0)
+    _raise(lib().sinkattn_take_device_error(ctypes.byref(flag)), "sinkattn_take_device_error")
+    return int(flag.value)

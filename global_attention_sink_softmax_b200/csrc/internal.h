@@ -1,0 +1,73 @@
+// Internal host-side interface between the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sinkattn {
+
+// ---- prefill -------------------------------------------------------------------------------
+struct PrefillParams {
+    int B, L, Hq, Hkv, G;
+    int window;           // > 0 sliding window, 0 full causal
+    int n_qtiles;         // ceil(L / 128)
+    float scale_log2;     // scale * log2(e)
+    const float *sink;    // [Hq] or nullptr
+    void *o;              // bf16
+    int64_t o_sb, o_sl, o_sh;
+    float *lse;           // [B, Hq, L] or nullptr
+};
+
+// Q map: dims {192, Hq, L, B}; K map: {192, Hkv, L, B}; V map: {128, Hkv, L, B}; 128-byte
+// swizzle, 64-element inner box.
+cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                                const CUtensorMap &tmV, const PrefillParams &p,
+                                cudaStream_t stream);
+
+// ---- decode --------------------------------------------------------------------------------
+struct DecodeParams {
+    int kind, B, T, Hq, Hkv, G, R, MT;   // R = T * G rows per unit, MT = ceil(R / 16)
+    int window;
+    int splits, chunk;                  // key spans per (b, kv head) and keys per span
+    float scale_log2;
+    const float *sink;
+    const uint16_t *q, *k_new, *v_new, *k_cache, *v_cache;
+    int64_t q_sb, q_st, q_sh;
+    int64_t kn_sb, kn_st, kn_sh, vn_sb, vn_st, vn_sh;
+    int64_t kc_sb, kc_ss, kc_sh, vc_sb, vc_ss, vc_sh;
+    const int32_t *ring_head, *ring_len;
+    int ring_cap;
+    const int32_t *ctx_len;
+    int max_ctx;
+    const int32_t *page_table;
+    int page_size, max_pages, num_pages;
+    uint16_t *o;
+    int64_t o_sb, o_st, o_sh;
+    float *lse;
+    float *ws_o;    // [B, Hkv, splits, R, 128] (splits > 1)
+    float *ws_ml;   // [B, Hkv, splits, R, 2]
+};
+
+cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream);
+
+struct CommitParams {
+    int kind, B, T, Hkv;
+    const uint16_t *k_new, *v_new;
+    int64_t kn_sb, kn_st, kn_sh, vn_sb, vn_st, vn_sh;
+    uint16_t *k_cache, *v_cache;
+    int64_t kc_sb, kc_ss, kc_sh, vc_sb, vc_ss, vc_sh;
+    int32_t *ring_head, *ring_len;
+    int ring_cap;
+    int32_t *ctx_len;
+    int max_ctx;
+    const int32_t *page_table;
+    int page_size, max_pages, num_pages;
+    const int32_t *n_accept;
+};
+
+cudaError_t launch_commit(const CommitParams &p, cudaStream_t stream);
+
+cudaError_t read_and_clear_device_error(uint32_t *flag);
+
+} // namespace sinkattn

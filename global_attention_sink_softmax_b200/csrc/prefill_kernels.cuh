@@ -1,0 +1,416 @@
+// Sink-softmax attention prefill on tcgen05 tensor cores (sm_100a).
+//
+// What it computes ("MiMo-V2-Flash 架构 QA" Q3.7/Q3.8; "MiMo-V2-Flash 模型架构深度拆解" CH10.1,
+// CH10.3): for each query row i of head h, over the keys j its mask keeps (j <= i, and
+// j > i - W for a sliding window W),
+//     O_i = sum_j exp(a_ij - m_i) v_j / (exp(sink_h - m_i) + sum_j exp(a_ij - m_i)),
+//     a_ij = scale <q_i, k_j>, m_i = max(sink_h, max_j a_ij), LSE_i = m_i + ln(denominator).
+//
+// Band kernel. One CTA = 128 query rows of one head against the 128-key tiles of its band:
+// tiles j_lo .. j_hi where the band is [i - W + 1, i] (SWA, at most 2 tiles for W = 128:
+// "MiMo-V2-Flash 架构 QA" Q3.6) or [0, i] (GA; tiles above the diagonal are never visited).
+//
+// Roles (224 threads):
+//   warps 0-3  softmax + epilogue: thread t owns query row t (TMEM lane t). It reads its row of
+//              S from TMEM, runs the online softmax seeded with the sink (m0 = sink, l0 = 1),
+//              writes P (bf16) into shared memory in the UMMA 128B-swizzled K-major layout,
+//              rescales its O row in TMEM when needed, and at the end normalises O and writes
+//              O (bf16) and LSE.
+//   warp 4     TMA producer for Q (once) and K tiles (2-stage ring).
+//   warp 5     TMA producer for V tiles (1 stage).
+//   warp 6     TMEM allocator and the single UMMA issuer: S = Q K^T (M128 N128 K16 x 12) into
+//              a double-buffered S in TMEM, O += P V (M128 N128 K16 x 8) into O in TMEM.
+// The issue order S_0, {S_{j+1}, PV_j} lets the tensor cores compute S_{j+1} while the softmax
+// warps work on S_j.
+//
+// Lazy rescaling: the running max used for the exponent is only raised when a tile's row max
+// exceeds it by more than 8 (log2 units); P values stay <= 2^8 and the final O / l and LSE are
+// exact for whatever reference max was used.
+#pragma once
+#include "common.cuh"
+#include "internal.h"
+
+namespace sinkattn {
+
+namespace pf {
+constexpr int BM = 128;                  // query rows per CTA
+constexpr int BN = 128;                  // keys per tile
+constexpr int ROW_BYTES = 128;           // one 64-element bf16 chunk row (the swizzle width)
+constexpr int Q_REGION = BM * ROW_BYTES; // 16 KB: 128 rows x 64 dims
+constexpr int Q_BYTES = 3 * Q_REGION;    // 192 dims
+constexpr int K_REGION = BN * ROW_BYTES;
+constexpr int K_BYTES = 3 * K_REGION;
+constexpr int V_BYTES = 2 * K_REGION;    // 128 dims
+constexpr int P_BYTES = 2 * BM * ROW_BYTES;
+constexpr int K_STAGES = 2;
+constexpr int OFF_Q = 0;
+constexpr int OFF_K = OFF_Q + Q_BYTES;
+constexpr int OFF_V = OFF_K + K_STAGES * K_BYTES;
+constexpr int OFF_P = OFF_V + V_BYTES;
+constexpr int OFF_BAR = OFF_P + P_BYTES;
+constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024; // barriers + 1 KB for aligning the base
+constexpr int THREADS = 224;
+constexpr int WARP_KLOAD = 4, WARP_VLOAD = 5, WARP_MMA = 6;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256;
+constexpr float TAU = 8.0f;
+
+enum Bar {
+    B_Q = 0,
+    B_KFULL = 1,   // + stage
+    B_KEMPTY = 3,  // + stage
+    B_VFULL = 5,
+    B_VEMPTY = 6,
+    B_SFULL = 7,   // + buffer
+    B_PFULL = 9,
+    B_PVDONE = 10,
+    B_DRAIN = 11,
+    NUM_BARS = 12
+};
+} // namespace pf
+
+// tcgen05.ld of 4 x 32 columns, then one wait; the wait names the registers so no use of them
+// can be scheduled before it.
+SA_DEV void tmem_ld128(uint32_t taddr, uint32_t (&r)[128])
+{
+    uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+    uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+    uint32_t(&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+    uint32_t(&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+    tmem_ld32(taddr + 0, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_ld32(taddr + 64, c);
+    tmem_ld32(taddr + 96, d);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 128; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
+}
+
+SA_DEV void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32])
+{
+    tmem_ld32(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
+}
+
+// A wait whose result is the same in every lane of the warp (required before warp-collective
+// tcgen05.ld/st).
+SA_DEV bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    bool ok = mbar_wait(bar, parity, abort, 1u);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__global__ void __launch_bounds__(pf::THREADS, 1)
+    prefill_band_kernel(const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV, const PrefillParams p)
+{
+    using namespace pf;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
+    volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    // ---- which tile: (query tile, batch, head), head fastest so the CTAs of one KV group run
+    // together and share K/V through L2; for GA the longest (last) query tiles go first.
+    const int per_tile = p.B * p.Hq;
+    const int t_idx = blockIdx.x / per_tile;
+    const int qt = (p.window > 0) ? t_idx : (p.n_qtiles - 1 - t_idx);
+    const int rem = blockIdx.x - t_idx * per_tile;
+    const int b = rem / p.Hq;
+    const int h = rem - b * p.Hq;
+    const int g = h / p.G;
+    const int r0 = qt * BM;
+    const int r_last = min(r0 + BM, p.L) - 1;
+    const int k_lo = (p.window > 0) ? max(0, r0 - p.window + 1) : 0;
+    const int j_lo = k_lo / BN;
+    const int j_hi = r_last / BN;
+    const int n_tiles = j_hi - j_lo + 1;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars[B_Q], 1);
+        mbar_init(&bars[B_KFULL + 0], 1);
+        mbar_init(&bars[B_KFULL + 1], 1);
+        mbar_init(&bars[B_KEMPTY + 0], 1);
+        mbar_init(&bars[B_KEMPTY + 1], 1);
+        mbar_init(&bars[B_VFULL], 1);
+        mbar_init(&bars[B_VEMPTY], 1);
+        mbar_init(&bars[B_SFULL + 0], 1);
+        mbar_init(&bars[B_SFULL + 1], 1);
+        mbar_init(&bars[B_PFULL], 128);
+        mbar_init(&bars[B_PVDONE], 1);
+        mbar_init(&bars[B_DRAIN], 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == WARP_MMA) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == WARP_KLOAD) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            mbar_arrive_expect_tx(&bars[B_Q], Q_BYTES);
+            for (int c = 0; c < 3; ++c)
+                tma_load_4d(smem + OFF_Q + c * Q_REGION, &tmQ, &bars[B_Q], c * 64, h, r0, b);
+            int issued = 0;
+            for (int idx = 0; idx < n_tiles; ++idx) {
+                const int s = idx & 1;
+                if (idx >= 2 && !mbar_wait(&bars[B_KEMPTY + s], ((idx >> 1) - 1) & 1, abort, 1u))
+                    break;
+                const int j = j_lo + idx;
+                mbar_arrive_expect_tx(&bars[B_KFULL + s], K_BYTES);
+                for (int c = 0; c < 3; ++c)
+                    tma_load_4d(smem + OFF_K + s * K_BYTES + c * K_REGION, &tmK,
+                                &bars[B_KFULL + s], c * 64, g, j * BN, b);
+                issued = idx + 1;
+            }
+            // make sure no copy of ours is still landing in shared memory when the CTA ends
+            for (int idx = max(0, issued - 2); idx < issued; ++idx)
+                mbar_wait_drain(&bars[B_KFULL + (idx & 1)], (idx >> 1) & 1);
+            mbar_wait_drain(&bars[B_Q], 0);
+        }
+        __syncwarp();
+    } else if (warp == WARP_VLOAD) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tmV);
+            int issued = 0;
+            for (int idx = 0; idx < n_tiles; ++idx) {
+                if (idx >= 1 && !mbar_wait(&bars[B_VEMPTY], (idx - 1) & 1, abort, 1u))
+                    break;
+                const int j = j_lo + idx;
+                mbar_arrive_expect_tx(&bars[B_VFULL], V_BYTES);
+                for (int c = 0; c < 2; ++c)
+                    tma_load_4d(smem + OFF_V + c * K_REGION, &tmV, &bars[B_VFULL], c * 64, g,
+                                j * BN, b);
+                issued = idx + 1;
+            }
+            if (issued > 0)
+                mbar_wait_drain(&bars[B_VFULL], (issued - 1) & 1);
+        }
+        __syncwarp();
+    } else if (warp == WARP_MMA) {
+        if (lane == 0) {
+            const uint32_t idesc_s = umma_idesc_bf16(BM, BN, 0);
+            const uint32_t idesc_o = umma_idesc_bf16(BM, 128, 1);
+            const uint32_t sQ = smem_u32(smem + OFF_Q);
+            const uint32_t sK = smem_u32(smem + OFF_K);
+            const uint32_t sV = smem_u32(smem + OFF_V);
+            const uint32_t sP = smem_u32(smem + OFF_P);
+            bool ok = mbar_wait(&bars[B_Q], 0, abort, 1u);
+            // S_idx = Q K_idx^T into S buffer idx & 1
+            auto issue_s = [&](int idx) -> bool {
+                const int s = idx & 1;
+                if (!mbar_wait(&bars[B_KFULL + s], (idx >> 1) & 1, abort, 1u))
+                    return false;
+                tc_fence_after();
+                const uint32_t d = tmem + (s ? TMEM_S1 : TMEM_S0);
+#pragma unroll
+                for (int kk = 0; kk < 12; ++kk) {
+                    const uint32_t off = (kk >> 2) * Q_REGION + (kk & 3) * 32;
+                    umma_ss(d, smem_desc_sw128(sQ + off, 16, 1024),
+                            smem_desc_sw128(sK + s * K_BYTES + off, 16, 1024), idesc_s, kk > 0);
+                }
+                umma_commit(&bars[B_SFULL + s]);
+                umma_commit(&bars[B_KEMPTY + s]);
+                return true;
+            };
+            if (ok)
+                ok = issue_s(0);
+            for (int idx = 0; ok && idx < n_tiles; ++idx) {
+                if (idx + 1 < n_tiles && !issue_s(idx + 1))
+                    break;
+                if (!mbar_wait(&bars[B_PFULL], idx & 1, abort, 1u))
+                    break;
+                if (!mbar_wait(&bars[B_VFULL], idx & 1, abort, 1u))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    // A = P (128 rows x 16 keys, K-major); B = V (16 keys x 128 dims, dims
+                    // contiguous: MN-major, dims 64..127 one 16 KB region further on)
+                    umma_ss(tmem + TMEM_O,
+                            smem_desc_sw128(sP + (kk >> 2) * Q_REGION + (kk & 3) * 32, 16, 1024),
+                            smem_desc_sw128(sV + kk * 16 * ROW_BYTES, K_REGION, 1024), idesc_o,
+                            (idx > 0 || kk > 0) ? 1u : 0u);
+                }
+                umma_commit(&bars[B_PVDONE]);
+                umma_commit(&bars[B_VEMPTY]);
+            }
+            // every MMA of ours has finished before TMEM is released
+            umma_commit(&bars[B_DRAIN]);
+            mbar_wait_drain(&bars[B_DRAIN], 0);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- softmax warps: thread = query row ----------------
+        const int row = threadIdx.x;          // 0..127
+        const int rp = r0 + row;              // position of this query row
+        const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+        const float sink_l2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
+        float m_run = sink_l2;                         // m_0 = sink
+        float l_run = (sink_l2 > -INFINITY) ? 1.f : 0.f; // l_0 = exp(sink - m_0)
+        uint8_t *prow = smem + OFF_P + row * ROW_BYTES;
+        bool ok = true;
+        for (int idx = 0; idx < n_tiles; ++idx) {
+            const int s = idx & 1;
+            const int kbase = (j_lo + idx) * BN;
+            ok = warp_wait(&bars[B_SFULL + s], (idx >> 1) & 1, abort);
+            if (!ok)
+                break;
+            tc_fence_after();
+            uint32_t raw[128];
+            tmem_ld128(tmem + lane_addr + (s ? TMEM_S1 : TMEM_S0), raw);
+            float x[128];
+            // mask only on tiles that cross the diagonal or the window's lower edge
+            const bool need_mask = (kbase + BN - 1 > r0) ||
+                                   (p.window > 0 && kbase < r0 + BM - p.window);
+            float mx = -INFINITY;
+            if (need_mask) {
+                const int hi = rp - kbase;                                   // keep c <= hi
+                const int lo = (p.window > 0) ? rp - p.window + 1 - kbase : -BN; // keep c >= lo
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    const float v = __uint_as_float(raw[c]) * p.scale_log2;
+                    x[c] = (c <= hi && c >= lo) ? v : -INFINITY;
+                    mx = fmaxf(mx, x[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 128; ++c) {
+                    x[c] = __uint_as_float(raw[c]) * p.scale_log2;
+                    mx = fmaxf(mx, x[c]);
+                }
+            }
+            const bool rescale = mx > m_run + TAU;
+            float alpha = 1.f;
+            if (rescale) {
+                alpha = fast_exp2(m_run - mx); // 0 when m_run is -inf
+                l_run *= alpha;
+                m_run = mx;
+            }
+            if (idx > 0) {
+                // PV of the previous tile is done: P buffer free, O up to date
+                ok = warp_wait(&bars[B_PVDONE], (idx - 1) & 1, abort);
+                if (!ok)
+                    break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * 32, o);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(tmem + lane_addr + TMEM_O + c * 32, o);
+                    }
+                    tmem_st_wait();
+                }
+            }
+            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+            float sum = 0.f;
+#pragma unroll
+            for (int c8 = 0; c8 < 16; ++c8) {
+                float e[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    e[u] = fast_exp2(x[c8 * 8 + u] - m_use);
+                    sum += e[u];
+                }
+                uint4 pk;
+                pk.x = pack_bf16x2(e[0], e[1]);
+                pk.y = pack_bf16x2(e[2], e[3]);
+                pk.z = pack_bf16x2(e[4], e[5]);
+                pk.w = pack_bf16x2(e[6], e[7]);
+                const int region = c8 >> 3, chunk = (c8 & 7) ^ (row & 7);
+                *reinterpret_cast<uint4 *>(prow + region * Q_REGION + chunk * 16) = pk;
+            }
+            l_run += sum;
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bars[B_PFULL]);
+        }
+        if (ok && n_tiles > 0)
+            ok = warp_wait(&bars[B_PVDONE], (n_tiles - 1) & 1, abort);
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = 1.f / l_run;
+            const bool valid = rp < p.L;
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (int64_t)b * p.o_sb +
+                                  (int64_t)rp * p.o_sl + (int64_t)h * p.o_sh;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * 32, o);
+                if (valid) {
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(__uint_as_float(o[v4 * 8 + 0]) * inv_l,
+                                           __uint_as_float(o[v4 * 8 + 1]) * inv_l);
+                        pk.y = pack_bf16x2(__uint_as_float(o[v4 * 8 + 2]) * inv_l,
+                                           __uint_as_float(o[v4 * 8 + 3]) * inv_l);
+                        pk.z = pack_bf16x2(__uint_as_float(o[v4 * 8 + 4]) * inv_l,
+                                           __uint_as_float(o[v4 * 8 + 5]) * inv_l);
+                        pk.w = pack_bf16x2(__uint_as_float(o[v4 * 8 + 6]) * inv_l,
+                                           __uint_as_float(o[v4 * 8 + 7]) * inv_l);
+                        *reinterpret_cast<uint4 *>(orow + c * 32 + v4 * 8) = pk;
+                    }
+                }
+            }
+            if (valid && p.lse)
+                p.lse[((int64_t)b * p.Hq + h) * p.L + rp] = (m_run + fast_log2(l_run)) * kLn2;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == WARP_MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                                const CUtensorMap &tmV, const PrefillParams &p,
+                                cudaStream_t stream)
+{
+    static int configured_devices = 0; // bit per device: shared-memory opt-in done
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 32 && !(configured_devices & (1 << dev))) {
+        e = cudaFuncSetAttribute(prefill_band_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 pf::SMEM_BYTES);
+        if (e != cudaSuccess)
+            return e;
+        configured_devices |= (1 << dev);
+    }
+    const int64_t blocks = (int64_t)p.n_qtiles * p.B * p.Hq;
+    if (blocks <= 0)
+        return cudaSuccess;
+    if (blocks > 0x7fffffff)
+        return cudaErrorInvalidConfiguration;
+    prefill_band_kernel<<<(unsigned)blocks, pf::THREADS, pf::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+    return cudaGetLastError();
+}
+
+} // namespace sinkattn

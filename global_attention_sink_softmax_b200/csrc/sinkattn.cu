@@ -1,0 +1,406 @@
+// C ABI of the sink-attention library: argument validation, TMA descriptor set-up, split-KV
+// sizing and kernel launches. Everything is enqueued on the caller's stream; the library
+// allocates no device memory. The kernels live in prefill_kernels.cuh / decode_kernels.cuh;
+// the whole library is this one translation unit.
+#include <math.h>
+#include <mutex>
+
+#include "sinkattn.h"
+
+#include "common.cuh"
+#include "decode_kernels.cuh"
+#include "internal.h"
+#include "prefill_kernels.cuh"
+
+namespace {
+
+using namespace sinkattn;
+
+constexpr int kDQ = 192, kDV = 128;
+constexpr int kNumSMs = 148;      // B200; only used to size the split-KV grid
+constexpr int kMinSpanKeys = 512; // below this a key span is not split further
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// element strides of bf16 tensors: positive and a whole number of 16-byte units
+bool stride_ok(int64_t s) { return s > 0 && (s % 8) == 0; }
+
+// 4-D bf16 map over [B, tokens, heads, d] given as dims {d, heads, tokens, B}; box
+// {64, box_heads, box_tokens, 1}, 128-byte swizzle, zero fill outside the tensor.
+int make_map(CUtensorMap *map, const void *base, int d, int heads, int tokens, int B,
+             int64_t s_head, int64_t s_tok, int64_t s_b, int box_heads, int box_tokens)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return SINKATTN_ERR_CUDA;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)tokens,
+                                (cuuint64_t)B};
+    const cuuint64_t strides[3] = {(cuuint64_t)s_head * 2, (cuuint64_t)s_tok * 2,
+                                   (cuuint64_t)s_b * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)box_heads, (cuuint32_t)box_tokens, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? SINKATTN_OK : SINKATTN_ERR_INVALID_ARG;
+}
+
+int validate_prefill(const sinkattn_prefill_args *a)
+{
+    if (!a)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->L < 0 || a->Hq <= 0 || a->Hkv <= 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->dq != kDQ || a->dv != kDV || a->Hq % a->Hkv != 0)
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (!isfinite(a->scale))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->B == 0 || a->L == 0)
+        return SINKATTN_OK;
+    if (!a->q || !a->k || !a->v || !a->o)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (!aligned16(a->q) || !aligned16(a->k) || !aligned16(a->v) || !aligned16(a->o))
+        return SINKATTN_ERR_ALIGNMENT;
+    const int64_t s[12] = {a->q_sb, a->q_sl, a->q_sh, a->k_sb, a->k_sl, a->k_sh,
+                           a->v_sb, a->v_sl, a->v_sh, a->o_sb, a->o_sl, a->o_sh};
+    for (int i = 0; i < 12; ++i) {
+        if (s[i] <= 0)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (!stride_ok(s[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    return SINKATTN_OK;
+}
+
+int run_prefill(const sinkattn_prefill_args *a, int window, void *stream)
+{
+    int st = validate_prefill(a);
+    if (st != SINKATTN_OK || a->B == 0 || a->L == 0)
+        return st;
+    CUtensorMap tq, tk, tv;
+    if ((st = make_map(&tq, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, 1, 128)))
+        return st;
+    if ((st = make_map(&tk, a->k, kDQ, a->Hkv, a->L, a->B, a->k_sh, a->k_sl, a->k_sb, 1, 128)))
+        return st;
+    if ((st = make_map(&tv, a->v, kDV, a->Hkv, a->L, a->B, a->v_sh, a->v_sl, a->v_sb, 1, 128)))
+        return st;
+    PrefillParams p;
+    p.B = a->B;
+    p.L = a->L;
+    p.Hq = a->Hq;
+    p.Hkv = a->Hkv;
+    p.G = a->Hq / a->Hkv;
+    p.window = window;
+    p.n_qtiles = (a->L + 127) / 128;
+    p.scale_log2 = a->scale * kLog2e;
+    p.sink = a->sink;
+    p.o = a->o;
+    p.o_sb = a->o_sb;
+    p.o_sl = a->o_sl;
+    p.o_sh = a->o_sh;
+    p.lse = a->lse;
+    const cudaError_t e = launch_prefill_band(tq, tk, tv, p, (cudaStream_t)stream);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+// ---- decode sizing ----------------------------------------------------------------------------
+struct Split {
+    int splits, chunk;
+};
+
+// Longest key sequence a (b, kv head) unit can have: used cached tokens + the T new ones.
+int64_t max_unit_keys(const sinkattn_decode_args *a)
+{
+    int64_t cached = (a->kind == SINKATTN_KV_RING) ? a->ring_cap : a->max_ctx;
+    if (a->window > 0)
+        cached = cached < a->window - 1 ? cached : a->window - 1;
+    return cached + a->T;
+}
+
+Split plan_split(const sinkattn_decode_args *a)
+{
+    const int64_t n = max_unit_keys(a);
+    const int64_t units = (int64_t)a->B * a->Hkv;
+    int64_t splits = (kNumSMs * 8 + units - 1) / units;
+    const int64_t by_len = (n + kMinSpanKeys - 1) / kMinSpanKeys;
+    if (splits > by_len)
+        splits = by_len;
+    if (splits < 1)
+        splits = 1;
+    int64_t chunk = (n + splits - 1) / splits;
+    chunk = (chunk + 63) / 64 * 64;
+    splits = (n + chunk - 1) / chunk;
+    return Split{(int)splits, (int)chunk};
+}
+
+size_t workspace_bytes(const sinkattn_decode_args *a, const Split &s)
+{
+    if (s.splits <= 1)
+        return 0;
+    const size_t rows = (size_t)a->B * a->Hkv * s.splits * (size_t)(a->T * (a->Hq / a->Hkv));
+    return rows * (kDV + 2) * sizeof(float);
+}
+
+int validate_decode(const sinkattn_decode_args *a)
+{
+    if (!a)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind != SINKATTN_KV_RING && a->kind != SINKATTN_KV_CONTIG && a->kind != SINKATTN_KV_PAGED)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->T < 0 || a->Hq <= 0 || a->Hkv <= 0 || a->window < 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->dq != kDQ || a->dv != kDV || a->Hq % a->Hkv != 0 || a->T > 4)
+        return SINKATTN_ERR_UNSUPPORTED;
+    const int G = a->Hq / a->Hkv;
+    if (G > 16 || a->T * G > 64)
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (!isfinite(a->scale))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind == SINKATTN_KV_RING) {
+        if (a->ring_cap <= 0 || !a->ring_head || !a->ring_len)
+            return SINKATTN_ERR_INVALID_ARG;
+    } else {
+        if (a->max_ctx < 0 || !a->ctx_len)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (a->kind == SINKATTN_KV_PAGED) {
+            if (a->page_size <= 0 || a->max_pages <= 0 || a->num_pages <= 0 || !a->page_table)
+                return SINKATTN_ERR_INVALID_ARG;
+            if ((int64_t)a->max_ctx > (int64_t)a->max_pages * a->page_size)
+                return SINKATTN_ERR_INVALID_ARG;
+        }
+    }
+    if (a->B == 0 || a->T == 0)
+        return SINKATTN_OK;
+    if (!a->q || !a->k_new || !a->v_new || !a->o || !a->k_cache || !a->v_cache)
+        return SINKATTN_ERR_INVALID_ARG;
+    const void *ptrs[6] = {a->q, a->k_new, a->v_new, a->k_cache, a->v_cache, a->o};
+    for (int i = 0; i < 6; ++i)
+        if (!aligned16(ptrs[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    const int64_t s[15] = {a->q_sb,  a->q_st,  a->q_sh,  a->kn_sb, a->kn_st,
+                           a->kn_sh, a->vn_sb, a->vn_st, a->vn_sh, a->kc_sb,
+                           a->kc_ss, a->kc_sh, a->vc_sb, a->vc_ss, a->vc_sh};
+    for (int i = 0; i < 15; ++i) {
+        if (s[i] <= 0)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (!stride_ok(s[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    const int64_t so[3] = {a->o_sb, a->o_st, a->o_sh};
+    for (int i = 0; i < 3; ++i) {
+        if (so[i] <= 0)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (!stride_ok(so[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    return SINKATTN_OK;
+}
+
+void fill_decode_params(DecodeParams &p, const sinkattn_decode_args *a, const Split &s, void *ws)
+{
+    p.kind = a->kind;
+    p.B = a->B;
+    p.T = a->T;
+    p.Hq = a->Hq;
+    p.Hkv = a->Hkv;
+    p.G = a->Hq / a->Hkv;
+    p.R = a->T * p.G;
+    p.MT = (p.R + 15) / 16;
+    p.window = a->window;
+    p.splits = s.splits;
+    p.chunk = s.chunk;
+    p.scale_log2 = a->scale * kLog2e;
+    p.sink = a->sink;
+    p.q = static_cast<const uint16_t *>(a->q);
+    p.k_new = static_cast<const uint16_t *>(a->k_new);
+    p.v_new = static_cast<const uint16_t *>(a->v_new);
+    p.k_cache = static_cast<const uint16_t *>(a->k_cache);
+    p.v_cache = static_cast<const uint16_t *>(a->v_cache);
+    p.q_sb = a->q_sb;
+    p.q_st = a->q_st;
+    p.q_sh = a->q_sh;
+    p.kn_sb = a->kn_sb;
+    p.kn_st = a->kn_st;
+    p.kn_sh = a->kn_sh;
+    p.vn_sb = a->vn_sb;
+    p.vn_st = a->vn_st;
+    p.vn_sh = a->vn_sh;
+    p.kc_sb = a->kc_sb;
+    p.kc_ss = a->kc_ss;
+    p.kc_sh = a->kc_sh;
+    p.vc_sb = a->vc_sb;
+    p.vc_ss = a->vc_ss;
+    p.vc_sh = a->vc_sh;
+    p.ring_head = a->ring_head;
+    p.ring_len = a->ring_len;
+    p.ring_cap = a->ring_cap;
+    p.ctx_len = a->ctx_len;
+    p.max_ctx = a->max_ctx;
+    p.page_table = a->page_table;
+    p.page_size = a->page_size;
+    p.max_pages = a->max_pages;
+    p.num_pages = a->num_pages;
+    p.o = static_cast<uint16_t *>(a->o);
+    p.o_sb = a->o_sb;
+    p.o_st = a->o_st;
+    p.o_sh = a->o_sh;
+    p.lse = a->lse;
+    const size_t rows = (size_t)a->B * a->Hkv * s.splits * (size_t)p.R;
+    p.ws_o = static_cast<float *>(ws);
+    p.ws_ml = ws ? static_cast<float *>(ws) + rows * kDV : nullptr;
+}
+
+} // namespace
+
+extern "C" {
+
+const char *sinkattn_status_string(int status)
+{
+    switch (status) {
+    case SINKATTN_OK: return "ok";
+    case SINKATTN_ERR_INVALID_ARG: return "invalid argument";
+    case SINKATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SINKATTN_ERR_ALIGNMENT: return "pointer or stride not 16-byte aligned";
+    case SINKATTN_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case SINKATTN_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+    }
+}
+
+int sinkattn_version(void) { return SINKATTN_VERSION; }
+
+int sinkattn_prefill_swa(const sinkattn_prefill_args *args, int32_t window, void *stream)
+{
+    if (window < 1)
+        return SINKATTN_ERR_INVALID_ARG;
+    return run_prefill(args, window, stream);
+}
+
+int sinkattn_prefill_ga(const sinkattn_prefill_args *args, void *stream)
+{
+    return run_prefill(args, 0, stream);
+}
+
+size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args)
+{
+    if (validate_decode(args) != SINKATTN_OK || args->B == 0 || args->T == 0)
+        return 0;
+    return workspace_bytes(args, plan_split(args));
+}
+
+int sinkattn_decode(const sinkattn_decode_args *args, void *workspace, size_t ws_bytes,
+                    void *stream)
+{
+    int st = validate_decode(args);
+    if (st != SINKATTN_OK || args->B == 0 || args->T == 0)
+        return st;
+    const Split s = plan_split(args);
+    const size_t need = workspace_bytes(args, s);
+    if (need > 0) {
+        if (!workspace || ws_bytes < need)
+            return SINKATTN_ERR_WORKSPACE_TOO_SMALL;
+        if (!aligned16(workspace))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    DecodeParams p;
+    fill_decode_params(p, args, s, need > 0 ? workspace : nullptr);
+    const cudaError_t e = launch_decode(p, (cudaStream_t)stream);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, void *stream)
+{
+    if (!a || (a->kind != SINKATTN_KV_RING && a->kind != SINKATTN_KV_CONTIG &&
+               a->kind != SINKATTN_KV_PAGED))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->T < 0 || a->Hkv <= 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->dq != kDQ || a->dv != kDV)
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->T == 0)
+        return SINKATTN_OK;
+    if (!n_accept || !a->k_new || !a->v_new || !a->k_cache || !a->v_cache)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind == SINKATTN_KV_RING && (a->ring_cap <= 0 || !a->ring_head || !a->ring_len))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind != SINKATTN_KV_RING && (a->max_ctx < 0 || !a->ctx_len))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind == SINKATTN_KV_PAGED &&
+        (a->page_size <= 0 || a->max_pages <= 0 || a->num_pages <= 0 || !a->page_table))
+        return SINKATTN_ERR_INVALID_ARG;
+    const void *ptrs[4] = {a->k_new, a->v_new, a->k_cache, a->v_cache};
+    for (int i = 0; i < 4; ++i)
+        if (!aligned16(ptrs[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    const int64_t s[12] = {a->kn_sb, a->kn_st, a->kn_sh, a->vn_sb, a->vn_st, a->vn_sh,
+                           a->kc_sb, a->kc_ss, a->kc_sh, a->vc_sb, a->vc_ss, a->vc_sh};
+    for (int i = 0; i < 12; ++i) {
+        if (s[i] <= 0)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (!stride_ok(s[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    CommitParams p;
+    p.kind = a->kind;
+    p.B = a->B;
+    p.T = a->T;
+    p.Hkv = a->Hkv;
+    p.k_new = static_cast<const uint16_t *>(a->k_new);
+    p.v_new = static_cast<const uint16_t *>(a->v_new);
+    p.kn_sb = a->kn_sb;
+    p.kn_st = a->kn_st;
+    p.kn_sh = a->kn_sh;
+    p.vn_sb = a->vn_sb;
+    p.vn_st = a->vn_st;
+    p.vn_sh = a->vn_sh;
+    p.k_cache = static_cast<uint16_t *>(const_cast<void *>(a->k_cache));
+    p.v_cache = static_cast<uint16_t *>(const_cast<void *>(a->v_cache));
+    p.kc_sb = a->kc_sb;
+    p.kc_ss = a->kc_ss;
+    p.kc_sh = a->kc_sh;
+    p.vc_sb = a->vc_sb;
+    p.vc_ss = a->vc_ss;
+    p.vc_sh = a->vc_sh;
+    p.ring_head = const_cast<int32_t *>(a->ring_head);
+    p.ring_len = const_cast<int32_t *>(a->ring_len);
+    p.ring_cap = a->ring_cap;
+    p.ctx_len = const_cast<int32_t *>(a->ctx_len);
+    p.max_ctx = a->max_ctx;
+    p.page_table = a->page_table;
+    p.page_size = a->page_size;
+    p.max_pages = a->max_pages;
+    p.num_pages = a->num_pages;
+    p.n_accept = n_accept;
+    const cudaError_t e = launch_commit(p, (cudaStream_t)stream);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+int sinkattn_take_device_error(uint32_t *flag_out)
+{
+    if (!flag_out)
+        return SINKATTN_ERR_INVALID_ARG;
+    const cudaError_t e = read_and_clear_device_error(flag_out);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+} // extern "C"

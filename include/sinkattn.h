@@ -1,0 +1,205 @@
+/*
+ * sinkattn.h — causal grouped-query softmax attention with a per-head sink, for NVIDIA B200
+ * (sm_100a). Plain C ABI: pointers, sizes and element strides; no C++ or framework types.
+ *
+ * What is computed. For query position i of head h (KV head g = h / (Hq / Hkv)) and the set
+ * J(i) of keys it may see:
+ *
+ *     a_ij = scale * <q_i, k_j>
+ *     m_i  = max(sink_h, max_{j in J(i)} a_ij)
+ *     D_i  = exp(sink_h - m_i) + sum_{j in J(i)} exp(a_ij - m_i)
+ *     O_i  = sum_{j in J(i)} exp(a_ij - m_i) v_j / D_i
+ *     LSE_i = m_i + ln D_i
+ *
+ * The sink adds exp(sink_h - m_i) to the denominator and contributes no value. Sources:
+ * "MiMo-V2-Flash 架构 QA" Q3.7 (the max includes the sink) and Q3.8 (the formula and its
+ * concat -> softmax -> drop equivalent); "MiMo-V2-Flash 模型架构深度拆解" CH3.2 (a_ij = q k^T
+ * / sqrt(d)), CH10.1 (one fp32 sink per query head, appended after scaling and masking),
+ * CH10.3 (scaling head_dim^-0.5; GA causal mask, SWA "only the latest 128 tokens");
+ * "MiMo-V2-Flash Technical Report" paper notes §4.1, §4.3 (128 keys in the W = 128 window).
+ *
+ * Visible keys J(i): global attention (GA) keeps j <= i; sliding-window attention (SWA) with
+ * window W keeps i - W < j <= i (exactly W keys once i >= W - 1, the query included).
+ *
+ * Conventions shared by every entry point.
+ *   - Element types: q, k, v, o and the caches are bf16; sink and lse are fp32.
+ *   - Layouts are token-major, [batch, token, head, dim], the dim contiguous; the other
+ *     three dims are given as element strides (int64). Base pointers and every non-unit
+ *     stride in bytes must be multiples of 16.
+ *   - Head dims: dq = 192 and dv = 128 (the kernels are specialised for them).
+ *     GQA group G = Hq / Hkv must be an integer in 1..16 (prefill) or 1..16 (decode).
+ *   - sink: fp32 [Hq] in post-scale logit units (not multiplied by scale). NULL means no sink
+ *     for any head; an entry of -inf means plain softmax for that head. NaN or +inf entries
+ *     give unspecified results (not checked).
+ *   - lse: natural log of the full denominator, sink included, so O = sum exp(a - LSE) v.
+ *     May be NULL.
+ *   - Ownership: the caller allocates and owns every buffer, host- and device-side. The
+ *     library allocates nothing and keeps no per-call state; decode scratch is a caller
+ *     workspace. All device pointers must be device memory of the current device.
+ *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream). Work is enqueued on
+ *     it; nothing synchronises the host. Returns after the launch.
+ *   - Errors: every entry point returns a sinkattn_status. Arguments are validated on the host
+ *     before anything is enqueued; an invalid call enqueues nothing. SINKATTN_ERR_CUDA reports
+ *     a launch failure (cudaGetLastError); faults during execution surface at the caller's next
+ *     synchronisation. A kernel that ever waits longer than about a second on an internal
+ *     barrier gives up, records it in a device flag and returns; sinkattn_take_device_error()
+ *     reads and clears that flag.
+ *   - Empty work (B == 0, L == 0, T == 0) is valid and enqueues nothing.
+ */
+#ifndef SINKATTN_H
+#define SINKATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SINKATTN_VERSION 1
+
+typedef enum sinkattn_status {
+    SINKATTN_OK = 0,
+    SINKATTN_ERR_INVALID_ARG = 1,          /* NULL pointer, negative size, bad stride */
+    SINKATTN_ERR_UNSUPPORTED = 2,          /* head dims != 192/128, G out of range, T > 4 ... */
+    SINKATTN_ERR_ALIGNMENT = 3,            /* pointer or stride not 16-byte aligned */
+    SINKATTN_ERR_WORKSPACE_TOO_SMALL = 4,  /* decode workspace below the size query */
+    SINKATTN_ERR_CUDA = 5                  /* a CUDA runtime call failed */
+} sinkattn_status;
+
+/* KV-cache layouts accepted by decode and commit. */
+typedef enum sinkattn_kv_kind {
+    SINKATTN_KV_RING = 0,    /* per-sequence ring of ring_cap slots (SWA) */
+    SINKATTN_KV_CONTIG = 1,  /* per-sequence contiguous cache of max_ctx rows (GA) */
+    SINKATTN_KV_PAGED = 2    /* page pool + per-sequence page table (GA) */
+} sinkattn_kv_kind;
+
+/* ---------------------------------------------------------------------------------------------
+ * Prefill: every position of every sequence attends to its own sequence.
+ *
+ *   q   [B, L, Hq,  192]  strides q_sb, q_sl, q_sh   (read)
+ *   k   [B, L, Hkv, 192]  strides k_sb, k_sl, k_sh   (read)
+ *   v   [B, L, Hkv, 128]  strides v_sb, v_sl, v_sh   (read)
+ *   o   [B, L, Hq,  128]  strides o_sb, o_sl, o_sh   (written; bf16, round-to-nearest-even)
+ *   lse [B, Hq, L] fp32, contiguous (written; may be NULL)
+ * ------------------------------------------------------------------------------------------- */
+typedef struct sinkattn_prefill_args {
+    const void *q;
+    const void *k;
+    const void *v;
+    const float *sink;
+    void *o;
+    float *lse;
+    int32_t B, L, Hq, Hkv, dq, dv;
+    float scale;
+    int64_t q_sb, q_sl, q_sh;
+    int64_t k_sb, k_sl, k_sh;
+    int64_t v_sb, v_sl, v_sh;
+    int64_t o_sb, o_sl, o_sh;
+} sinkattn_prefill_args;
+
+/* Sliding-window prefill (SWA), window >= 1 keys (the pages' model uses 128). Keys outside the
+ * window are never loaded: a W = 128 row touches at most two 128-key chunks ("MiMo-V2-Flash 架构
+ * QA" Q3.6). */
+int sinkattn_prefill_swa(const sinkattn_prefill_args *args, int32_t window, void *stream);
+
+/* Global (full causal) prefill (GA). Key tiles above the diagonal are skipped. */
+int sinkattn_prefill_ga(const sinkattn_prefill_args *args, void *stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Decode / speculative verify: T (1..4) new query tokens per sequence attend to that sequence's
+ * cached tokens plus new tokens 0..t. The new tokens' K/V are passed separately and are NOT yet
+ * in the cache (sinkattn_kv_commit appends the accepted ones afterwards).
+ *
+ * Positions: cached token c (0 = oldest of n_b) sits at c - n_b, new token u at u; new query t
+ * sees keys at positions p <= t, and, when window > 0, p > t - window. For T = 1 and a full
+ * ring this equals "write the new token into the ring, then attend over all its slots".
+ *
+ *   q     [B, T, Hq, 192]   strides q_sb, q_st, q_sh
+ *   k_new [B, T, Hkv, 192], v_new [B, T, Hkv, 128]  strides kn_*, vn_*
+ *   RING:   k_cache [B, ring_cap, Hkv, 192], v_cache [B, ring_cap, Hkv, 128];
+ *           ring_head[B] = slot of the oldest cached token, ring_len[B] = tokens held
+ *           (0..ring_cap); cached token c is in slot (ring_head + c) mod ring_cap.
+ *   CONTIG: k_cache [B, max_ctx, Hkv, 192] ...; ctx_len[B] (0..max_ctx) tokens held.
+ *   PAGED:  k_cache [num_pages, page_size, Hkv, 192] ...; cached token c of sequence b is row
+ *           c mod page_size of page page_table[b * max_pages + c / page_size]; ctx_len[B]
+ *           (0..max_ctx, max_ctx <= max_pages * page_size). Page ids outside [0, num_pages)
+ *           make that page's keys invisible (no out-of-bounds read).
+ *   ring_head, ring_len, ctx_len, page_table: int32 device arrays. max_ctx is a host-side
+ *   upper bound on ctx_len (entries above it are clamped to it).
+ *   o [B, T, Hq, 128] strides o_sb, o_st, o_sh;  lse [B, T, Hq] fp32 contiguous (may be NULL).
+ *   cache strides: kc_sb = stride between sequences (RING, CONTIG) or pages (PAGED),
+ *                  kc_ss = stride between slots / tokens / page rows, kc_sh = between heads.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct sinkattn_decode_args {
+    int32_t kind; /* sinkattn_kv_kind */
+    int32_t B, T, Hq, Hkv, dq, dv;
+    int32_t window; /* > 0: sliding window of `window` keys; 0: full causal (GA) */
+    float scale;
+    const float *sink;
+    const void *q;
+    int64_t q_sb, q_st, q_sh;
+    const void *k_new;
+    int64_t kn_sb, kn_st, kn_sh;
+    const void *v_new;
+    int64_t vn_sb, vn_st, vn_sh;
+    const void *k_cache;
+    int64_t kc_sb, kc_ss, kc_sh;
+    const void *v_cache;
+    int64_t vc_sb, vc_ss, vc_sh;
+    const int32_t *ring_head;
+    const int32_t *ring_len;
+    int32_t ring_cap;
+    const int32_t *ctx_len;
+    int32_t max_ctx;
+    const int32_t *page_table;
+    int32_t page_size, max_pages, num_pages;
+    void *o;
+    int64_t o_sb, o_st, o_sh;
+    float *lse;
+} sinkattn_decode_args;
+
+/* Bytes of device workspace sinkattn_decode needs for these arguments (split-KV partials:
+ * per split, an unnormalised fp32 O row and its running max and sum). 0 when no split is
+ * needed. Returns 0 for invalid arguments too; sinkattn_decode reports those. */
+size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args);
+
+/* Split-KV decode: each (sequence, KV head, key span) block computes sink-free partials; the
+ * merge counts the sink exactly once: m = max(sink, max_p m_p), D = exp(sink - m) +
+ * sum_p l_p exp(m_p - m), O = sum_p O_p exp(m_p - m) / D, LSE = m + ln D (derived from
+ * "MiMo-V2-Flash 架构 QA" Q3.8). `workspace` is caller-owned device memory of at least
+ * sinkattn_decode_workspace_size(args) bytes, 16-byte aligned (may be NULL when that is 0);
+ * its contents on entry do not matter. */
+int sinkattn_decode(const sinkattn_decode_args *args, void *workspace, size_t workspace_bytes,
+                    void *stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * Commit accepted tokens to the cache (the attention module's "KV cache update" step,
+ * "MiMo-V2-Flash 模型架构深度拆解" CH10.3). For each sequence b the first n_accept[b] (0..T)
+ * of its T new tokens are appended oldest first:
+ *   RING:   token goes to slot (ring_head + ring_len) mod ring_cap; ring_len grows to at most
+ *           ring_cap, after which each new token replaces the oldest and ring_head advances.
+ *   CONTIG: row ctx_len[b] + u (tokens beyond max_ctx are dropped); ctx_len grows.
+ *   PAGED:  position ctx_len[b] + u through the page table (positions beyond
+ *           max_pages * page_size are dropped); ctx_len grows.
+ * Uses the cache, metadata and *_new fields of `args` (q, o, lse, sink are ignored). Updates
+ * k_cache, v_cache, ring_head / ring_len or ctx_len in place, in stream order.
+ * ------------------------------------------------------------------------------------------- */
+int sinkattn_kv_commit(const sinkattn_decode_args *args, const int32_t *n_accept, void *stream);
+
+/* Human-readable name of a status code (static storage). */
+const char *sinkattn_status_string(int status);
+
+/* SINKATTN_VERSION of the built library. */
+int sinkattn_version(void);
+
+/* Reads and clears the device flag that kernels set when an internal wait gives up (bit 0:
+ * prefill, bit 1: decode). Synchronises the current device. Returns SINKATTN_OK and writes the
+ * flag to *flag_out, or SINKATTN_ERR_CUDA. */
+int sinkattn_take_device_error(uint32_t *flag_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SINKATTN_H */

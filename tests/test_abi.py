@@ -1,0 +1,182 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the header declares,
+its structs have the layout the Python binding assumes, and invalid arguments are rejected on
+the host before any CUDA call."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+import torch
+
+import global_attention_sink_softmax_b200 as sa
+from global_attention_sink_softmax_b200 import build as sa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sinkattn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    sa_build.build()
+    return sa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sinkattn_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree_on_entry_points():
+    assert declared_functions() == sorted(sa.EXPORTED_SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", sa.library_path], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT (sinkattn_\w+)", out))
+    missing = set(declared_functions()) - exported
+    assert not missing, missing
+    for name in declared_functions():
+        assert hasattr(L, name)
+
+
+def test_version_and_status_strings(L):
+    assert sa.sinkattn_version() == 1
+    assert sa.sinkattn_status_string(0) == "ok"
+    for s in range(1, 6):
+        assert sa.sinkattn_status_string(s) not in ("ok", "unknown status")
+    assert sa.sinkattn_status_string(99) == "unknown status"
+
+
+C_LAYOUT = r"""
+#include <stddef.h>
+#include <stdio.h>
+#include "sinkattn.h"
+#define F(S, f) printf(#S "." #f " %zu\n", offsetof(S, f));
+int main(void) {
+  printf("sinkattn_prefill_args %zu\n", sizeof(sinkattn_prefill_args));
+  printf("sinkattn_decode_args %zu\n", sizeof(sinkattn_decode_args));
+  %FIELDS%
+  return 0;
+}
+"""
+
+
+def test_struct_layout_matches_header(tmp_path):
+    lines = []
+    for cname, py in (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs)):
+        for f, _ in py._fields_:
+            lines.append(f"F({cname}, {f})")
+    src = C_LAYOUT.replace("%FIELDS%", "\n  ".join(lines))
+    c = tmp_path / "layout.c"
+    exe = tmp_path / "layout"
+    c.write_text(src)
+    subprocess.check_call(["gcc", "-std=c11", "-I", os.path.join(ROOT, "include"), str(c), "-o", str(exe)])
+    got = dict(l.rsplit(" ", 1) for l in subprocess.check_output([str(exe)], text=True).splitlines())
+    assert int(got["sinkattn_prefill_args"]) == ctypes.sizeof(sa.PrefillArgs)
+    assert int(got["sinkattn_decode_args"]) == ctypes.sizeof(sa.DecodeArgs)
+    for cname, py in (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs)):
+        for f, _ in py._fields_:
+            assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
+
+
+def _prefill_args(**kw):
+    a = sa.PrefillArgs()
+    a.q = a.k = a.v = a.o = 0x10000
+    a.B, a.L, a.Hq, a.Hkv, a.dq, a.dv = 1, 64, 8, 1, 192, 128
+    a.scale = 0.07
+    for f in ("q", "k", "v", "o"):
+        d = 192 if f in ("q", "k") else 128
+        h = 8 if f in ("q", "o") else 1
+        setattr(a, f + "_sh", d)
+        setattr(a, f + "_sl", d * h)
+        setattr(a, f + "_sb", d * h * 64)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(dq=128), 2), (dict(dv=192), 2), (dict(Hkv=3), 2), (dict(B=-1), 1), (dict(Hq=0), 1),
+    (dict(q=None), 1), (dict(q=0x10008), 3), (dict(k_sl=100), 3), (dict(o_sh=0), 1),
+    (dict(scale=float("inf")), 1),
+])
+def test_prefill_rejects_bad_arguments(L, kw, status):
+    a = _prefill_args(**kw)
+    assert L.sinkattn_prefill_ga(ctypes.byref(a), None) == status
+    assert L.sinkattn_prefill_swa(ctypes.byref(a), 128, None) == status
+
+
+def test_prefill_empty_is_ok_and_window_checked(L):
+    assert L.sinkattn_prefill_ga(ctypes.byref(_prefill_args(L=0)), None) == 0
+    assert L.sinkattn_prefill_ga(ctypes.byref(_prefill_args(B=0, q=None)), None) == 0
+    assert L.sinkattn_prefill_swa(ctypes.byref(_prefill_args()), 0, None) == 1
+    assert L.sinkattn_prefill_swa(ctypes.byref(_prefill_args()), -5, None) == 1
+    assert L.sinkattn_prefill_ga(None, None) == 1
+
+
+def _decode_args(**kw):
+    a = sa.DecodeArgs()
+    a.kind, a.B, a.T, a.Hq, a.Hkv, a.dq, a.dv, a.window = 1, 2, 1, 64, 4, 192, 128, 0
+    a.scale = 0.07
+    a.q = a.k_new = a.v_new = a.k_cache = a.v_cache = a.o = 0x20000
+    a.ctx_len = 0x30000
+    a.max_ctx = 4096
+    for pre, d in (("q", 192), ("kn", 192), ("vn", 128), ("kc", 192), ("vc", 128), ("o", 128)):
+        for i, s in enumerate(("sb", "st" if pre in ("q", "kn", "vn", "o") else "ss", "sh")):
+            setattr(a, f"{pre}_{s}", d * (4096 if i == 0 else (64 if i == 1 else 1)))
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kind=7), 1), (dict(T=5), 2), (dict(Hkv=2), 2), (dict(Hkv=3), 2), (dict(dq=64), 2),
+    (dict(ctx_len=None), 1), (dict(kind=0), 1), (dict(kind=2), 1), (dict(o=None), 1),
+    (dict(k_cache=0x20004), 3), (dict(kc_ss=10), 3), (dict(window=-1), 1),
+    (dict(kind=2, page_table=0x40000, page_size=128, max_pages=2, num_pages=4), 1),
+])
+def test_decode_rejects_bad_arguments(L, kw, status):
+    a = _decode_args(**kw)
+    assert L.sinkattn_decode(ctypes.byref(a), None, 0, None) == status
+    assert L.sinkattn_decode_workspace_size(ctypes.byref(a)) == 0
+
+
+def test_decode_workspace_sizing(L):
+    # GA decode at 262144 tokens of context, 8 x 4 units: split, workspace = partial rows
+    a = _decode_args(B=8, max_ctx=262144)
+    need = L.sinkattn_decode_workspace_size(ctypes.byref(a))
+    assert need > 0 and need % (130 * 4 * 16) == 0
+    assert L.sinkattn_decode(ctypes.byref(a), None, 0, None) == 4
+    assert L.sinkattn_decode(ctypes.byref(a), ctypes.c_void_p(0x50000), need - 1, None) == 4
+    assert L.sinkattn_decode(ctypes.byref(a), ctypes.c_void_p(0x50008), need, None) == 3
+    # a 128-slot ring never needs a split
+    r = _decode_args(kind=0, ring_head=0x30000, ring_len=0x30100, ring_cap=128, window=128, Hkv=8)
+    assert L.sinkattn_decode_workspace_size(ctypes.byref(r)) == 0
+    # empty work
+    assert L.sinkattn_decode(ctypes.byref(_decode_args(B=0)), None, 0, None) == 0
+    assert L.sinkattn_decode(ctypes.byref(_decode_args(T=0)), None, 0, None) == 0
+
+
+def test_commit_rejects_bad_arguments(L):
+    a = _decode_args()
+    assert L.sinkattn_kv_commit(ctypes.byref(a), None, None) == 1
+    assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(dv=64)), ctypes.c_void_p(0x60000), None) == 2
+    assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(kind=0)), ctypes.c_void_p(0x60000), None) == 1
+    assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(B=0)), None, None) == 0
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(sa, "library_path", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(sa, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        sa.lib()
+
+
+def test_binding_checks_tensor_types():
+    q = torch.zeros(1, 4, 8, 192)
+    with pytest.raises(TypeError):
+        sa.sinkattn_prefill_ga(q, q, q, o=torch.zeros(1, 4, 8, 128))
