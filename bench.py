@@ -433,6 +433,9 @@ def main():
     ap.add_argument("--only", default=None,
                     help="run one workload only: swa_prefill, ga_prefill, ga_decode, swa_decode, hybrid")
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--small", action="store_true",
+                    help="profiling case: prefill workloads at B=1 (SWA L=16384, GA L=8192), "
+                         "decode at B=2")
     args = ap.parse_args()
     world, rank, local = init_dist(args)
     args.gpus = max(args.gpus, world)
@@ -453,8 +456,16 @@ def main():
     peaks, peak_src = load_peaks()
     flush = None
 
+    swa_w, ga_w, gad_w, swad_w = W.SWA_PREFILL, W.GA_PREFILL, W.GA_DECODE, W.SWA_DECODE
+    if args.small:
+        import dataclasses
+        swa_w = dataclasses.replace(swa_w, B=1, L=16384, name=swa_w.name + "_small_B1_L16384")
+        ga_w = dataclasses.replace(ga_w, L=8192, name=ga_w.name + "_small_L8192")
+        gad_w = dataclasses.replace(gad_w, B=2, name=gad_w.name + "_small_B2")
+        swad_w = dataclasses.replace(swad_w, B=64, name=swad_w.name + "_small_B64")
+
     def head_runner():
-        return PrefillRunner(W.SWA_PREFILL, dev)
+        return PrefillRunner(swa_w, dev)
 
     only = args.only
     result = None
@@ -491,7 +502,7 @@ def main():
             d_cpu = {k: v.cpu() for k, v in r.d.items()}
             r.release()
             torch.cuda.empty_cache()
-            cpu_base = cpu_baseline_prefill(W.SWA_PREFILL, d_cpu)
+            cpu_base = cpu_baseline_prefill(swa_w, d_cpu)
             del d_cpu
         r.release()
         del r
@@ -500,12 +511,12 @@ def main():
     if not args.no_secondary:
         jobs = []
         if only in (None, "ga_prefill"):
-            jobs.append(("ga_prefill", lambda: PrefillRunner(W.GA_PREFILL, dev), None))
+            jobs.append(("ga_prefill", lambda: PrefillRunner(ga_w, dev), None))
         if only in (None, "ga_decode"):
-            jobs.append(("ga_decode", lambda: DecodeRunner(W.GA_DECODE, dev), None))
+            jobs.append(("ga_decode", lambda: DecodeRunner(gad_w, dev), None))
         if only in (None, "swa_decode"):
-            jobs.append(("swa_decode", lambda: DecodeRunner(W.SWA_DECODE, dev), "flush"))
-        if only in (None, "hybrid"):
+            jobs.append(("swa_decode", lambda: DecodeRunner(swad_w, dev), "flush"))
+        if only in (None, "hybrid") and not args.small:
             jobs.append(("hybrid", lambda: HybridRunner(dev), None))
         for name, make, fl in jobs:
             r = make()

@@ -237,6 +237,12 @@ SA_DEV uint32_t pack_bf16x2(float lo, float hi)
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// Sum of the two bf16 halves of a packed pair, as fp32 (bf16 -> fp32 is exact).
+SA_DEV float sum_bf16x2(uint32_t v)
+{
+    return __uint_as_float(v << 16) + __uint_as_float(v & 0xffff0000u);
+}
+
 // ---------------------------------------------------------------------------------------------
 // Warp-level tensor-core path (cp.async + ldmatrix + mma.sync), used by decode
 // ---------------------------------------------------------------------------------------------

@@ -31,7 +31,7 @@ constexpr int STAGE_V = KT * VROW;
 constexpr int STAGE = STAGE_K + STAGE_V + KT; // + one validity byte per key
 constexpr int SMEM = NSTAGE * STAGE;
 constexpr int THREADS = 128;
-constexpr int RED_STRIDE = 68;         // floats per lane in the cross-warp combine
+constexpr int RED_STRIDE = 70;         // floats per lane in the cross-warp combine
 } // namespace dec
 
 struct KeyRows {
@@ -152,7 +152,8 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
 #pragma unroll
     for (int i = 0; i < 16; ++i)
         o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f;
+    // per row: running max m, sum of bf16-rounded P (l*, normalises O) and of fp32 P (e*, LSE)
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.f, l_b = 0.f, e_a = 0.f, e_b = 0.f;
 
     // prologue: NSTAGE - 1 tiles in flight
 #pragma unroll
@@ -226,18 +227,25 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
         const float ua = (mna == -INFINITY) ? 0.f : mna, ub = (mnb == -INFINITY) ? 0.f : mnb;
         m_a = mna;
         m_b = mnb;
-        float sa = 0.f, sb = 0.f;
+        // P in bf16 pairs: [nt][0] row a, [nt][1] row b; the row sums add these same rounded
+        // values so the weights of numerator and denominator agree
+        uint32_t pp[NT][2];
+        float sa = 0.f, sb = 0.f, xa = 0.f, xb = 0.f;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-            sacc[nt][0] = fast_exp2(sacc[nt][0] - ua);
-            sacc[nt][1] = fast_exp2(sacc[nt][1] - ua);
-            sacc[nt][2] = fast_exp2(sacc[nt][2] - ub);
-            sacc[nt][3] = fast_exp2(sacc[nt][3] - ub);
-            sa += sacc[nt][0] + sacc[nt][1];
-            sb += sacc[nt][2] + sacc[nt][3];
+            const float p0 = fast_exp2(sacc[nt][0] - ua), p1 = fast_exp2(sacc[nt][1] - ua);
+            const float p2 = fast_exp2(sacc[nt][2] - ub), p3 = fast_exp2(sacc[nt][3] - ub);
+            xa += p0 + p1;
+            xb += p2 + p3;
+            pp[nt][0] = pack_bf16x2(p0, p1);
+            pp[nt][1] = pack_bf16x2(p2, p3);
+            sa += sum_bf16x2(pp[nt][0]);
+            sb += sum_bf16x2(pp[nt][1]);
         }
         l_a = l_a * alpha_a + sa;
         l_b = l_b * alpha_b + sb;
+        e_a = e_a * alpha_a + xa;
+        e_b = e_b * alpha_b + xb;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
             o[i][0] *= alpha_a;
@@ -250,10 +258,10 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
 #pragma unroll
         for (int kq = 0; kq < NT / 2; ++kq) {
             uint32_t a[4];
-            a[0] = pack_bf16x2(sacc[2 * kq][0], sacc[2 * kq][1]);
-            a[1] = pack_bf16x2(sacc[2 * kq][2], sacc[2 * kq][3]);
-            a[2] = pack_bf16x2(sacc[2 * kq + 1][0], sacc[2 * kq + 1][1]);
-            a[3] = pack_bf16x2(sacc[2 * kq + 1][2], sacc[2 * kq + 1][3]);
+            a[0] = pp[2 * kq][0];
+            a[1] = pp[2 * kq][1];
+            a[2] = pp[2 * kq + 1][0];
+            a[3] = pp[2 * kq + 1][1];
             const int key = key0 + kq * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
             for (int np = 0; np < 8; ++np) {
@@ -272,6 +280,10 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    e_a += __shfl_xor_sync(0xffffffffu, e_a, 1);
+    e_a += __shfl_xor_sync(0xffffffffu, e_a, 2);
+    e_b += __shfl_xor_sync(0xffffffffu, e_b, 1);
+    e_b += __shfl_xor_sync(0xffffffffu, e_b, 2);
 
     // ---- combine the KP key slices of each m-tile (same fragment layout in every warp)
     if (KP > 1) {
@@ -290,6 +302,8 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
             dst[65] = m_b;
             dst[66] = l_a;
             dst[67] = l_b;
+            dst[68] = e_a;
+            dst[69] = e_b;
         }
         __syncthreads();
         if (active && ks == 0) {
@@ -311,6 +325,8 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
                 }
                 l_a = l_a * a1 + src[66] * a2;
                 l_b = l_b * b1 + src[67] * b2;
+                e_a = e_a * a1 + src[68] * a2;
+                e_b = e_b * b1 + src[69] * b2;
                 m_a = mna;
                 m_b = mnb;
             }
@@ -329,13 +345,13 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
             if (r >= p.R)
                 continue;
             const int t = r / p.G, h = g * p.G + r % p.G;
-            const float m = half ? m_b : m_a, l = half ? l_b : l_a;
+            const float m = half ? m_b : m_a, l = half ? l_b : l_a, le = half ? e_b : e_a;
             const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
             const float mf = fmaxf(m, sk);
             const float cm = (m == -INFINITY) ? 0.f : fast_exp2(m - mf);
             const float cs = (sk == -INFINITY) ? 0.f : fast_exp2(sk - mf);
-            const float D = l * cm + cs;
-            const float scl = cm / D;
+            const float D = le * cm + cs;         // exact denominator: LSE
+            const float scl = cm / (l * cm + cs); // rounded-P denominator: O
             uint16_t *orow = p.o + (int64_t)b * p.o_sb + (int64_t)t * p.o_st + (int64_t)h * p.o_sh;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -362,10 +378,12 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
                 *reinterpret_cast<float2 *>(wo + i * 8 + c2) = v2;
             }
             if ((lane & 3) == 0) {
-                float2 ml;
+                float4 ml;
                 ml.x = half ? m_b : m_a;
                 ml.y = half ? l_b : l_a;
-                *reinterpret_cast<float2 *>(p.ws_ml + (unit * p.R + r) * 2) = ml;
+                ml.z = half ? e_b : e_a;
+                ml.w = 0.f;
+                *reinterpret_cast<float4 *>(p.ws_ml + (unit * p.R + r) * 4) = ml;
             }
         }
     }
@@ -394,12 +412,12 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     const int g = h / p.G;
     const int r = t * p.G + (h - g * p.G);
     const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
-    float m = sk, l = (sk == -INFINITY) ? 0.f : 1.f;
+    float m = sk, l = (sk == -INFINITY) ? 0.f : 1.f, le = l;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     const int64_t unit0 = ((int64_t)b * p.Hkv + g) * p.splits;
     for (int s = 0; s < p.splits; ++s) {
         const int64_t idx = (unit0 + s) * p.R + r;
-        const float2 ml = *reinterpret_cast<const float2 *>(p.ws_ml + idx * 2);
+        const float4 ml = *reinterpret_cast<const float4 *>(p.ws_ml + idx * 4);
         if (!(ml.y > 0.f))
             continue;
         const float mn = fmaxf(m, ml.x);
@@ -411,6 +429,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
         acc.z = acc.z * a + v.z * c;
         acc.w = acc.w * a + v.w * c;
         l = l * a + ml.y * c;
+        le = le * a + ml.z * c;
         m = mn;
     }
     const float inv = 1.f / l;
@@ -420,7 +439,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
     pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
     *reinterpret_cast<uint2 *>(orow + lane * 4) = pk;
     if (p.lse && lane == 0)
-        p.lse[((int64_t)b * p.T + t) * p.Hq + h] = (m + fast_log2(l)) * kLn2;
+        p.lse[((int64_t)b * p.T + t) * p.Hq + h] = (m + fast_log2(le)) * kLn2;
 }
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream)

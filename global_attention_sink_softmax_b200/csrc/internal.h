@@ -46,7 +46,7 @@ struct DecodeParams {
     int64_t o_sb, o_st, o_sh;
     float *lse;
     float *ws_o;    // [B, Hkv, splits, R, 128] (splits > 1)
-    float *ws_ml;   // [B, Hkv, splits, R, 2]
+    float *ws_ml;   // [B, Hkv, splits, R, 4]: max, sum of rounded P, sum of fp32 P, pad
 };
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream);

@@ -23,6 +23,9 @@
 // The issue order S_0, {S_{j+1}, PV_j} lets the tensor cores compute S_{j+1} while the softmax
 // warps work on S_j.
 //
+// Two row sums: O is normalised by the sum of the bf16-rounded P values (the ones the P.V MMA
+// multiplies), so numerator and denominator use identical weights; LSE uses the fp32 sum.
+//
 // Lazy rescaling: the running max used for the exponent is only raised when a tile's row max
 // exceeds it by more than 8 (log2 units); P values stay <= 2^8 and the final O / l and LSE are
 // exact for whatever reference max was used.
@@ -264,8 +267,13 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         const int rp = r0 + row;              // position of this query row
         const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
         const float sink_l2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
-        float m_run = sink_l2;                         // m_0 = sink
-        float l_run = (sink_l2 > -INFINITY) ? 1.f : 0.f; // l_0 = exp(sink - m_0)
+        const float c_l2 = p.scale_log2; // > 0, so max(s) * c = max(s * c)
+        // m_run: reference max (log2 units); l_exact: sum of fp32 P (gives LSE); l_round: sum
+        // of the bf16-rounded P the P.V MMA consumes (normalises O). Both start with the sink:
+        // m_0 = sink, l_0 = exp(sink - m_0) = 1.
+        float m_run = sink_l2;
+        float l_exact = (sink_l2 > -INFINITY) ? 1.f : 0.f;
+        float l_round = l_exact;
         uint8_t *prow = smem + OFF_P + row * ROW_BYTES;
         bool ok = true;
         for (int idx = 0; idx < n_tiles; ++idx) {
@@ -277,7 +285,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             tc_fence_after();
             uint32_t raw[128];
             tmem_ld128(tmem + lane_addr + (s ? TMEM_S1 : TMEM_S0), raw);
-            float x[128];
+            float x[128]; // raw scores q.k; masked keys -inf
             // mask only on tiles that cross the diagonal or the window's lower edge
             const bool need_mask = (kbase + BN - 1 > r0) ||
                                    (p.window > 0 && kbase < r0 + BM - p.window);
@@ -287,22 +295,23 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 const int lo = (p.window > 0) ? rp - p.window + 1 - kbase : -BN; // keep c >= lo
 #pragma unroll
                 for (int c = 0; c < 128; ++c) {
-                    const float v = __uint_as_float(raw[c]) * p.scale_log2;
-                    x[c] = (c <= hi && c >= lo) ? v : -INFINITY;
+                    x[c] = (c <= hi && c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;
                     mx = fmaxf(mx, x[c]);
                 }
             } else {
 #pragma unroll
                 for (int c = 0; c < 128; ++c) {
-                    x[c] = __uint_as_float(raw[c]) * p.scale_log2;
+                    x[c] = __uint_as_float(raw[c]);
                     mx = fmaxf(mx, x[c]);
                 }
             }
+            mx *= c_l2;
             const bool rescale = mx > m_run + TAU;
             float alpha = 1.f;
             if (rescale) {
                 alpha = fast_exp2(m_run - mx); // 0 when m_run is -inf
-                l_run *= alpha;
+                l_exact *= alpha;
+                l_round *= alpha;
                 m_run = mx;
             }
             if (idx > 0) {
@@ -324,25 +333,27 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                     tmem_st_wait();
                 }
             }
-            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-            float sum = 0.f;
+            const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+            float se = 0.f, sr = 0.f;
 #pragma unroll
             for (int c8 = 0; c8 < 16; ++c8) {
                 float e[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    e[u] = fast_exp2(x[c8 * 8 + u] - m_use);
-                    sum += e[u];
+                    e[u] = fast_exp2(fmaf(x[c8 * 8 + u], c_l2, neg_m));
+                    se += e[u];
                 }
                 uint4 pk;
                 pk.x = pack_bf16x2(e[0], e[1]);
                 pk.y = pack_bf16x2(e[2], e[3]);
                 pk.z = pack_bf16x2(e[4], e[5]);
                 pk.w = pack_bf16x2(e[6], e[7]);
+                sr += (sum_bf16x2(pk.x) + sum_bf16x2(pk.y)) + (sum_bf16x2(pk.z) + sum_bf16x2(pk.w));
                 const int region = c8 >> 3, chunk = (c8 & 7) ^ (row & 7);
                 *reinterpret_cast<uint4 *>(prow + region * Q_REGION + chunk * 16) = pk;
             }
-            l_run += sum;
+            l_exact += se;
+            l_round += sr;
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL]);
@@ -351,7 +362,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             ok = warp_wait(&bars[B_PVDONE], (n_tiles - 1) & 1, abort);
         if (ok) {
             tc_fence_after();
-            const float inv_l = 1.f / l_run;
+            const float inv_l = 1.f / l_round;
             const bool valid = rp < p.L;
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (int64_t)b * p.o_sb +
                                   (int64_t)rp * p.o_sl + (int64_t)h * p.o_sh;
@@ -376,7 +387,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 }
             }
             if (valid && p.lse)
-                p.lse[((int64_t)b * p.Hq + h) * p.L + rp] = (m_run + fast_log2(l_run)) * kLn2;
+                p.lse[((int64_t)b * p.Hq + h) * p.L + rp] = (m_run + fast_log2(l_exact)) * kLn2;
         }
     }
 

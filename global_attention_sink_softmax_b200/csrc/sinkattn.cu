@@ -73,7 +73,7 @@ int validate_prefill(const sinkattn_prefill_args *a)
         return SINKATTN_ERR_INVALID_ARG;
     if (a->dq != kDQ || a->dv != kDV || a->Hq % a->Hkv != 0)
         return SINKATTN_ERR_UNSUPPORTED;
-    if (!isfinite(a->scale))
+    if (!isfinite(a->scale) || !(a->scale > 0.f))
         return SINKATTN_ERR_INVALID_ARG;
     if (a->B == 0 || a->L == 0)
         return SINKATTN_OK;
@@ -158,7 +158,7 @@ size_t workspace_bytes(const sinkattn_decode_args *a, const Split &s)
     if (s.splits <= 1)
         return 0;
     const size_t rows = (size_t)a->B * a->Hkv * s.splits * (size_t)(a->T * (a->Hq / a->Hkv));
-    return rows * (kDV + 2) * sizeof(float);
+    return rows * (kDV + 4) * sizeof(float);
 }
 
 int validate_decode(const sinkattn_decode_args *a)
@@ -174,7 +174,7 @@ int validate_decode(const sinkattn_decode_args *a)
     const int G = a->Hq / a->Hkv;
     if (G > 16 || a->T * G > 64)
         return SINKATTN_ERR_UNSUPPORTED;
-    if (!isfinite(a->scale))
+    if (!isfinite(a->scale) || !(a->scale > 0.f))
         return SINKATTN_ERR_INVALID_ARG;
     if (a->kind == SINKATTN_KV_RING) {
         if (a->ring_cap <= 0 || !a->ring_head || !a->ring_len)

@@ -33,6 +33,7 @@
  *     give unspecified results (not checked).
  *   - lse: natural log of the full denominator, sink included, so O = sum exp(a - LSE) v.
  *     May be NULL.
+ *   - scale: finite and > 0 (1/sqrt(192) for the pages' model).
  *   - Ownership: the caller allocates and owns every buffer, host- and device-side. The
  *     library allocates nothing and keeps no per-call state; decode scratch is a caller
  *     workspace. All device pointers must be device memory of the current device.
@@ -160,7 +161,8 @@ typedef struct sinkattn_decode_args {
 } sinkattn_decode_args;
 
 /* Bytes of device workspace sinkattn_decode needs for these arguments (split-KV partials:
- * per split, an unnormalised fp32 O row and its running max and sum). 0 when no split is
+ * per split and query row, an unnormalised fp32 O row, its running max and two running sums,
+ * one over the bf16-rounded P that multiplied V and one over fp32 P). 0 when no split is
  * needed. Returns 0 for invalid arguments too; sinkattn_decode reports those. */
 size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args);
 

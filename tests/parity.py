@@ -11,8 +11,14 @@ def assert_close(o_gpu, o_ref, lse_gpu=None, lse_ref=None, what=""):
     og = o_gpu.detach().double().cpu()
     assert og.shape == o_ref.shape, (og.shape, o_ref.shape)
     assert torch.isfinite(og).all(), f"{what}: non-finite O"
-    err = (og - o_ref).abs().max().item() if og.numel() else 0.0
-    assert err <= O_TOL, f"{what}: max |O - oracle| = {err:.3e} > {O_TOL}"
+    diff = (og - o_ref).abs()
+    err = diff.max().item() if og.numel() else 0.0
+    if err > O_TOL:
+        i = int(diff.argmax())
+        idx = torch.unravel_index(torch.tensor(i), diff.shape)
+        raise AssertionError(f"{what}: max |O - oracle| = {err:.3e} > {O_TOL} at "
+                             f"{tuple(int(x) for x in idx)}: gpu {og.flatten()[i].item():.6f} "
+                             f"oracle {o_ref.flatten()[i].item():.6f}")
     lerr = 0.0
     if lse_ref is not None:
         lg = lse_gpu.detach().double().cpu()
