@@ -388,6 +388,9 @@ def run_reference(args, world, rank):
     if rank != 0:
         return None
     w = W.SWA_PREFILL
+    if args.ref_L:
+        import dataclasses
+        w = dataclasses.replace(w, L=args.ref_L, name=f"{w.name}_L{args.ref_L}")
     # inputs of the full workload, drawn on the CPU generator
     d_cpu = W.prefill_inputs(w, device="cpu")
     rows_per_step = args.ref_rows
@@ -433,6 +436,7 @@ def main():
     ap.add_argument("--only", default=None,
                     help="run one workload only: swa_prefill, ga_prefill, ga_decode, swa_decode, hybrid")
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--ref-L", type=int, default=0, help="reference arm: shorter sequences (tests)")
     ap.add_argument("--small", action="store_true",
                     help="profiling case: prefill workloads at B=1 (SWA L=16384, GA L=8192), "
                          "decode at B=2")
