@@ -161,6 +161,31 @@ size_t workspace_bytes(const sinkattn_decode_args *a, const Split &s)
     return rows * (kDV + 4) * sizeof(float);
 }
 
+// The sizes and layout kinds that fix the split plan and hence the workspace size.
+int validate_decode_shape(const sinkattn_decode_args *a)
+{
+    if (!a)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind != SINKATTN_KV_RING && a->kind != SINKATTN_KV_CONTIG && a->kind != SINKATTN_KV_PAGED)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->T < 0 || a->Hq <= 0 || a->Hkv <= 0 || a->window < 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->dq != kDQ || a->dv != kDV || a->Hq % a->Hkv != 0 || a->T > 4)
+        return SINKATTN_ERR_UNSUPPORTED;
+    const int G = a->Hq / a->Hkv;
+    if (G > 16 || a->T * G > 64)
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (a->kind == SINKATTN_KV_RING && a->ring_cap <= 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind != SINKATTN_KV_RING && a->max_ctx < 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->kind == SINKATTN_KV_PAGED &&
+        (a->page_size <= 0 || a->max_pages <= 0 ||
+         (int64_t)a->max_ctx > (int64_t)a->max_pages * a->page_size))
+        return SINKATTN_ERR_INVALID_ARG;
+    return SINKATTN_OK;
+}
+
 int validate_decode(const sinkattn_decode_args *a)
 {
     if (!a)
@@ -303,7 +328,7 @@ int sinkattn_prefill_ga(const sinkattn_prefill_args *args, void *stream)
 
 size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args)
 {
-    if (validate_decode(args) != SINKATTN_OK || args->B == 0 || args->T == 0)
+    if (validate_decode_shape(args) != SINKATTN_OK || args->B == 0 || args->T == 0)
         return 0;
     return workspace_bytes(args, plan_split(args));
 }

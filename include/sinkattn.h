@@ -163,7 +163,9 @@ typedef struct sinkattn_decode_args {
 /* Bytes of device workspace sinkattn_decode needs for these arguments (split-KV partials:
  * per split and query row, an unnormalised fp32 O row, its running max and two running sums,
  * one over the bf16-rounded P that multiplied V and one over fp32 P). 0 when no split is
- * needed. Returns 0 for invalid arguments too; sinkattn_decode reports those. */
+ * needed. Depends only on kind, B, T, Hq, Hkv, dq, dv, window, ring_cap / max_ctx and the page
+ * geometry; pointers and strides are not read. Returns 0 for invalid sizes too;
+ * sinkattn_decode reports those. */
 size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args);
 
 /* Split-KV decode: each (sequence, KV head, key span) block computes sink-free partials; the

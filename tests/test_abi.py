@@ -142,7 +142,16 @@ def _decode_args(**kw):
 def test_decode_rejects_bad_arguments(L, kw, status):
     a = _decode_args(**kw)
     assert L.sinkattn_decode(ctypes.byref(a), None, 0, None) == status
-    assert L.sinkattn_decode_workspace_size(ctypes.byref(a)) == 0
+
+
+def test_workspace_size_needs_shapes_only(L):
+    a = _decode_args(B=8, max_ctx=262144)
+    need = L.sinkattn_decode_workspace_size(ctypes.byref(a))
+    for f in ("q", "k_new", "v_new", "k_cache", "v_cache", "o", "ctx_len"):
+        b = _decode_args(B=8, max_ctx=262144, **{f: None})
+        assert L.sinkattn_decode_workspace_size(ctypes.byref(b)) == need
+    for kw in (dict(T=5), dict(Hkv=3), dict(dq=64), dict(kind=7), dict(window=-1)):
+        assert L.sinkattn_decode_workspace_size(ctypes.byref(_decode_args(B=8, **kw))) == 0
 
 
 def test_decode_workspace_sizing(L):
