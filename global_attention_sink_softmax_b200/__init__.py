@@ -25,6 +25,7 @@ __all__ = [
     "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_decode",
     "sinkattn_decode_workspace_size", "sinkattn_kv_commit", "sinkattn_take_device_error",
     "sinkattn_status_string", "sinkattn_version", "EXPORTED_SYMBOLS",
+    "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES",
 ]
 
 KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
@@ -34,8 +35,10 @@ library_path = os.path.join(_PKG, "libsinkattn.so")
 EXPORTED_SYMBOLS = [
     "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_decode_workspace_size",
     "sinkattn_decode", "sinkattn_kv_commit", "sinkattn_status_string", "sinkattn_version",
-    "sinkattn_take_device_error",
+    "sinkattn_take_device_error", "sinkattn_decode_noalloc",
 ]
+# Size of the library's own split-KV workspace used by sinkattn_decode_noalloc.
+NOALLOC_WORKSPACE_BYTES = 16 << 20
 
 
 class SinkAttnError(RuntimeError):
@@ -95,6 +98,8 @@ def lib() -> ctypes.CDLL:
             L.sinkattn_decode_workspace_size.restype = _SZ
             L.sinkattn_decode.argtypes = [ctypes.POINTER(DecodeArgs), _P, _SZ, _P]
             L.sinkattn_decode.restype = ctypes.c_int
+            L.sinkattn_decode_noalloc.argtypes = [ctypes.POINTER(DecodeArgs), _P]
+            L.sinkattn_decode_noalloc.restype = ctypes.c_int
             L.sinkattn_kv_commit.argtypes = [ctypes.POINTER(DecodeArgs), _P, _P]
             L.sinkattn_kv_commit.restype = ctypes.c_int
             L.sinkattn_status_string.argtypes = [ctypes.c_int]
@@ -293,6 +298,27 @@ def sinkattn_decode(kind, q, k_new, v_new, k_cache, v_cache, sink=None, *, windo
     ws_bytes = workspace.numel() * workspace.element_size() if need > 0 else 0
     st = L_.sinkattn_decode(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream))
     _raise(st, "sinkattn_decode")
+    return o, lse
+
+
+def sinkattn_decode_noalloc(kind, q, k_new, v_new, k_cache, v_cache, sink=None, *, window=0,
+                            ring_head=None, ring_len=None, ctx_len=None, max_ctx=None,
+                            page_table=None, page_size=None, num_pages=None, o=None, lse=None,
+                            scale=None, stream=None):
+    """Decode without a workspace, for callers that cannot allocate device memory (a plugin host
+    that passes only input/output buffers, a serving loop with all memory reserved up front).
+    The library keeps the split-KV partials in its own fixed 16 MiB device array; larger
+    problems are rejected (use sinkattn_decode with a workspace). Calls that overlap on the GPU
+    race on that array. `o` and `lse` must be given (nothing is allocated here)."""
+    B, T, Hq, dq = q.shape
+    if o is None or lse is None:
+        raise ValueError("sinkattn_decode_noalloc allocates nothing: pass o and lse")
+    if scale is None:
+        scale = 1.0 / math.sqrt(dq)
+    a = _decode_args(kind, q, k_new, v_new, k_cache, v_cache, sink, window, scale, ring_head,
+                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse)
+    _raise(lib().sinkattn_decode_noalloc(ctypes.byref(a), _stream(stream)),
+           "sinkattn_decode_noalloc")
     return o, lse
 
 

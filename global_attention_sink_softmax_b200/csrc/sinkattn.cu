@@ -295,6 +295,43 @@ void fill_decode_params(DecodeParams &p, const sinkattn_decode_args *a, const Sp
     p.ws_ml = ws ? static_cast<float *>(ws) + rows * kDV : nullptr;
 }
 
+// ---- decode without a caller workspace ------------------------------------------------------
+// Some callers hand this library only their input and output buffers and have no device
+// allocator to lend it: a plugin host whose interface passes fixed buffers, or a serving loop
+// whose device memory is all reserved up front, where a cudaMalloc on the decode path would
+// block the device or fail under memory pressure. sinkattn_decode_noalloc serves them with a
+// split-KV workspace that is a fixed array in the library's own device memory.
+constexpr size_t kNoAllocWorkspaceBytes = SINKATTN_NOALLOC_WORKSPACE_BYTES;
+static __device__ __align__(256) float g_noalloc_workspace[kNoAllocWorkspaceBytes / sizeof(float)];
+
+constexpr int kMaxCachedDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxCachedDevices] = {};
+
+// Device address of g_noalloc_workspace on the current device. Host code cannot use the
+// array's name as a device pointer, so the address is looked up with cudaGetSymbolAddress the
+// first time a device needs it (with that device current) and kept per device.
+cudaError_t noalloc_workspace_ptr(void **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (dev >= 0 && dev < kMaxCachedDevices && g_noalloc_ptr[dev]) {
+        *out = g_noalloc_ptr[dev];
+        return cudaSuccess;
+    }
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_workspace);
+    if (e != cudaSuccess)
+        return e;
+    if (dev >= 0 && dev < kMaxCachedDevices)
+        g_noalloc_ptr[dev] = p;
+    *out = p;
+    return cudaSuccess;
+}
+
 } // namespace
 
 extern "C" {
@@ -349,6 +386,26 @@ int sinkattn_decode(const sinkattn_decode_args *args, void *workspace, size_t ws
     }
     DecodeParams p;
     fill_decode_params(p, args, s, need > 0 ? workspace : nullptr);
+    const cudaError_t e = launch_decode(p, (cudaStream_t)stream);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+int sinkattn_decode_noalloc(const sinkattn_decode_args *args, void *stream)
+{
+    int st = validate_decode(args);
+    if (st != SINKATTN_OK || args->B == 0 || args->T == 0)
+        return st;
+    const Split s = plan_split(args);
+    const size_t need = workspace_bytes(args, s);
+    if (need > kNoAllocWorkspaceBytes)
+        return SINKATTN_ERR_WORKSPACE_TOO_SMALL;
+    void *ws = nullptr;
+    if (need > 0 && noalloc_workspace_ptr(&ws) != cudaSuccess)
+        return SINKATTN_ERR_CUDA;
+    // Every partial the merge reads is written first by the split kernel of the same call, so
+    // whatever an earlier call left in the array needs no clearing.
+    DecodeParams p;
+    fill_decode_params(p, args, s, need > 0 ? ws : nullptr);
     const cudaError_t e = launch_decode(p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }

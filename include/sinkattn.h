@@ -177,6 +177,31 @@ size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args);
 int sinkattn_decode(const sinkattn_decode_args *args, void *workspace, size_t workspace_bytes,
                     void *stream);
 
+/* Largest split-KV workspace sinkattn_decode_noalloc can provide: 16 MiB. */
+#define SINKATTN_NOALLOC_WORKSPACE_BYTES (16u << 20)
+
+/* Decode that allocates nothing and takes no workspace. The pages have no counterpart: this is
+ * a service of the library, not part of the method.
+ *
+ * For callers that cannot allocate device memory and have no workspace to lend: a plugin host
+ * that passes the library only its input and output buffers, or a serving loop whose device
+ * memory is reserved up front, where a cudaMalloc on the decode path would block the device or
+ * fail under memory pressure. It computes exactly what sinkattn_decode computes, with the
+ * split-KV partials kept in a fixed array in the library's own device memory
+ * (SINKATTN_NOALLOC_WORKSPACE_BYTES; every GPU that loads the library holds it until the process
+ * exits).
+ *   - Arguments, outputs and errors as for sinkattn_decode. Calls whose
+ *     sinkattn_decode_workspace_size exceeds SINKATTN_NOALLOC_WORKSPACE_BYTES are rejected with
+ *     SINKATTN_ERR_WORKSPACE_TOO_SMALL before anything is enqueued (e.g. B * Hkv * T * G * spans
+ *     * 528 bytes above 16 MiB); use sinkattn_decode with a caller workspace for those.
+ *   - The first call on a device that needs the array looks up its device address
+ *     (cudaGetSymbolAddress) with that device current and remembers it; make that first call
+ *     before any stream capture.
+ *   - Each device has its own copy of the array; all calls on that device share it, and it
+ *     keeps the last call's contents (nothing in it needs to start at zero). Calls that overlap
+ *     on the GPU, for example on two streams of one device, race on it: serialise them. */
+int sinkattn_decode_noalloc(const sinkattn_decode_args *args, void *stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Commit accepted tokens to the cache (the attention module's "KV cache update" step,
  * "MiMo-V2-Flash 模型架构深度拆解" CH10.3). For each sequence b the first n_accept[b] (0..T)
