@@ -155,6 +155,18 @@ SA_DEV void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t 
                  : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::f16. A (M x K, K-major) sits in tensor memory:
+// row i in lane i, two consecutive bf16 K elements per 32-bit column.
+SA_DEV void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                    uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05.mma issued so far by this thread has completed.
 SA_DEV void umma_commit(uint64_t *bar)
 {
@@ -210,8 +222,78 @@ SA_DEV void tmem_st32(uint32_t taddr, const uint32_t (&r)[32])
                  : "memory");
 }
 
+// 32 lanes x 16 consecutive 32-bit columns.
+SA_DEV void tmem_ld16(uint32_t taddr, uint32_t (&r)[16])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                   "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+}
+
 SA_DEV void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 8 consecutive 32-bit columns from registers.
+SA_DEV void tmem_st8(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3,
+                     uint32_t r4, uint32_t r5, uint32_t r6, uint32_t r7)
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(
+                     taddr),
+                 "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(r4), "r"(r5), "r"(r6), "r"(r7)
+                 : "memory");
+}
+
+// tcgen05.ld of 16 columns followed by the wait; the registers are tied to the wait so no use
+// of them is scheduled before it.
+SA_DEV void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16])
+{
+    tmem_ld16(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 16; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
+}
 SA_DEV void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// tcgen05.ld of 4 x 32 columns, then one wait; the wait names the registers so no use of them
+// can be scheduled before it.
+SA_DEV void tmem_ld128(uint32_t taddr, uint32_t (&r)[128])
+{
+    uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
+    uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
+    uint32_t(&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
+    uint32_t(&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
+    tmem_ld32(taddr + 0, a);
+    tmem_ld32(taddr + 32, b);
+    tmem_ld32(taddr + 64, c);
+    tmem_ld32(taddr + 96, d);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 128; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
+}
+
+SA_DEV void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32])
+{
+    tmem_ld32(taddr, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 32; i += 8)
+        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
+}
+
+// A wait whose result is the same in every lane of the warp (required before warp-collective
+// tcgen05.ld/st).
+SA_DEV bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
+{
+    bool ok = mbar_wait(bar, parity, abort, 1u);
+    return __all_sync(0xffffffffu, ok);
+}
 
 // ---------------------------------------------------------------------------------------------
 // scalar math

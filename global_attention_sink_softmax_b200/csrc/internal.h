@@ -25,6 +25,27 @@ cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                 const CUtensorMap &tmV, const PrefillParams &p,
                                 cudaStream_t stream);
 
+// SWA prefill, GQA-packed persistent kernel: item = (b, kv head, block of P = 128 / G positions)
+struct SwaParams {
+    int B, L, Hq, Hkv, G;
+    int P;                // positions per item
+    int W;                // window
+    int NS;               // key span per item (multiple of 16, <= 256)
+    int n_pblk, n_items;
+    float scale_log2;
+    const float *sink;
+    void *o;
+    int64_t o_sb, o_sl, o_sh;
+    float *lse;
+};
+
+// Q map box {64, G, P, 1}; K / V map box {64, 1, NS, 1}; grid = persistent CTAs.
+cudaError_t launch_prefill_swa_packed(const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                                      const CUtensorMap &tmV, const SwaParams &p, int grid,
+                                      cudaStream_t stream);
+// Largest dynamic shared memory the packed SWA kernel may use on this device.
+int swa_packed_smem_bytes(int ns);
+
 // ---- decode --------------------------------------------------------------------------------
 struct DecodeParams {
     int kind, B, T, Hq, Hkv, G, R, MT;   // R = T * G rows per unit, MT = ceil(R / 16)

@@ -72,43 +72,6 @@ enum Bar {
 };
 } // namespace pf
 
-// tcgen05.ld of 4 x 32 columns, then one wait; the wait names the registers so no use of them
-// can be scheduled before it.
-SA_DEV void tmem_ld128(uint32_t taddr, uint32_t (&r)[128])
-{
-    uint32_t(&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[0]);
-    uint32_t(&b)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[32]);
-    uint32_t(&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[64]);
-    uint32_t(&d)[32] = *reinterpret_cast<uint32_t(*)[32]>(&r[96]);
-    tmem_ld32(taddr + 0, a);
-    tmem_ld32(taddr + 32, b);
-    tmem_ld32(taddr + 64, c);
-    tmem_ld32(taddr + 96, d);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 128; i += 8)
-        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
-                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
-}
-
-SA_DEV void tmem_ld32_sync(uint32_t taddr, uint32_t (&r)[32])
-{
-    tmem_ld32(taddr, r);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 32; i += 8)
-        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
-                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
-}
-
-// A wait whose result is the same in every lane of the warp (required before warp-collective
-// tcgen05.ld/st).
-SA_DEV bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort)
-{
-    bool ok = mbar_wait(bar, parity, abort, 1u);
-    return __all_sync(0xffffffffu, ok);
-}
-
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_band_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
@@ -306,7 +269,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 }
             }
             mx *= c_l2;
-            const bool rescale = mx > m_run + TAU;
+            // The first tile sets the exact max (m = max(sink, row max)), so rows that see few
+            // keys get their dominant term exactly 1; later tiles raise it lazily.
+            const bool rescale = (idx == 0) ? (mx > m_run) : (mx > m_run + TAU);
             float alpha = 1.f;
             if (rescale) {
                 alpha = fast_exp2(m_run - mx); // 0 when m_run is -inf

@@ -11,6 +11,7 @@
 #include "decode_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
+#include "swa_kernels.cuh"
 
 namespace {
 
@@ -92,11 +93,98 @@ int validate_prefill(const sinkattn_prefill_args *a)
     return SINKATTN_OK;
 }
 
+// Per-device figures used to shape grids (cached; a device's properties do not change).
+struct DeviceInfo {
+    int sms = 0, smem_optin = 0;
+};
+
+int device_info(DeviceInfo *out)
+{
+    static std::mutex mu;
+    static DeviceInfo cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess)
+        return SINKATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= 0 && dev < 64 && cache[dev].sms > 0) {
+        *out = cache[dev];
+        return SINKATTN_OK;
+    }
+    DeviceInfo d;
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+        return SINKATTN_ERR_CUDA;
+    if (dev >= 0 && dev < 64)
+        cache[dev] = d;
+    *out = d;
+    return SINKATTN_OK;
+}
+
+// SWA prefill with the GQA group packed into the MMA rows: possible when G divides 128 and the
+// span of P + W - 1 keys (P = 128 / G positions) fits one MMA (<= 256) and shared memory.
+int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *stream, bool *done)
+{
+    *done = false;
+    const int G = a->Hq / a->Hkv;
+    if (128 % G != 0)
+        return SINKATTN_OK;
+    const int P = 128 / G;
+    const int64_t span = (int64_t)P + window - 1;
+    const int NS = (int)((span + 15) / 16 * 16);
+    if (span > 256)
+        return SINKATTN_OK;
+    DeviceInfo di;
+    int st = device_info(&di);
+    if (st != SINKATTN_OK)
+        return st;
+    if (swa_packed_smem_bytes(NS) > di.smem_optin)
+        return SINKATTN_OK;
+    CUtensorMap tq, tk, tv;
+    if ((st = make_map(&tq, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, G, P)))
+        return st;
+    if ((st = make_map(&tk, a->k, kDQ, a->Hkv, a->L, a->B, a->k_sh, a->k_sl, a->k_sb, 1, NS)))
+        return st;
+    if ((st = make_map(&tv, a->v, kDV, a->Hkv, a->L, a->B, a->v_sh, a->v_sl, a->v_sb, 1, NS)))
+        return st;
+    SwaParams p;
+    p.B = a->B;
+    p.L = a->L;
+    p.Hq = a->Hq;
+    p.Hkv = a->Hkv;
+    p.G = G;
+    p.P = P;
+    p.W = window;
+    p.NS = NS;
+    p.n_pblk = (a->L + P - 1) / P;
+    const int64_t items = (int64_t)a->B * a->Hkv * p.n_pblk;
+    if (items > 0x7fffffff)
+        return SINKATTN_ERR_UNSUPPORTED;
+    p.n_items = (int)items;
+    p.scale_log2 = a->scale * kLog2e;
+    p.sink = a->sink;
+    p.o = a->o;
+    p.o_sb = a->o_sb;
+    p.o_sl = a->o_sl;
+    p.o_sh = a->o_sh;
+    p.lse = a->lse;
+    const int grid = (int)(items < di.sms ? items : di.sms);
+    const cudaError_t e = launch_prefill_swa_packed(tq, tk, tv, p, grid, (cudaStream_t)stream);
+    *done = true;
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
 int run_prefill(const sinkattn_prefill_args *a, int window, void *stream)
 {
     int st = validate_prefill(a);
     if (st != SINKATTN_OK || a->B == 0 || a->L == 0)
         return st;
+    if (window > 0) {
+        bool done = false;
+        st = try_prefill_swa_packed(a, window, stream, &done);
+        if (st != SINKATTN_OK || done)
+            return st;
+    }
     CUtensorMap tq, tk, tv;
     if ((st = make_map(&tq, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, 1, 128)))
         return st;
