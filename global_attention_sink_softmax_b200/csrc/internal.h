@@ -39,12 +39,14 @@ struct SwaParams {
     float *lse;
 };
 
-// Q map box {64, G, P, 1}; K / V map box {64, 1, NS, 1}; grid = persistent CTAs.
+// Q map box {64, G, P, 1}; K / V map box {64, 1, NS, 1}; K / V chunk map box {64, 1, 16, 1};
+// grid = persistent CTAs. Specialised for NS = 144, P = 16 (G = 8, W <= 128).
 cudaError_t launch_prefill_swa_packed(const CUtensorMap &tmQ, const CUtensorMap &tmK,
-                                      const CUtensorMap &tmV, const SwaParams &p, int grid,
+                                      const CUtensorMap &tmV, const CUtensorMap &tmKc,
+                                      const CUtensorMap &tmVc, const SwaParams &p, int grid,
                                       cudaStream_t stream);
 // Largest dynamic shared memory the packed SWA kernel may use on this device.
-int swa_packed_smem_bytes(int ns);
+int swa_packed_smem_bytes(int ns, int P);
 
 // ---- decode --------------------------------------------------------------------------------
 struct DecodeParams {

@@ -252,22 +252,28 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             // mask only on tiles that cross the diagonal or the window's lower edge
             const bool need_mask = (kbase + BN - 1 > r0) ||
                                    (p.window > 0 && kbase < r0 + BM - p.window);
-            float mx = -INFINITY;
+            // eight independent running maxima: short dependency chains
+            float mx8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mx8[i] = -INFINITY;
             if (need_mask) {
                 const int hi = rp - kbase;                                   // keep c <= hi
                 const int lo = (p.window > 0) ? rp - p.window + 1 - kbase : -BN; // keep c >= lo
 #pragma unroll
                 for (int c = 0; c < 128; ++c) {
                     x[c] = (c <= hi && c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;
-                    mx = fmaxf(mx, x[c]);
+                    mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
                 }
             } else {
 #pragma unroll
                 for (int c = 0; c < 128; ++c) {
                     x[c] = __uint_as_float(raw[c]);
-                    mx = fmaxf(mx, x[c]);
+                    mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
                 }
             }
+            float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             mx *= c_l2;
             // The first tile sets the exact max (m = max(sink, row max)), so rows that see few
             // keys get their dominant term exactly 1; later tiles raise it lazily.
@@ -299,26 +305,31 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 }
             }
             const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-            float se = 0.f, sr = 0.f;
+            float pe[4] = {0.f, 0.f, 0.f, 0.f}, pr[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c8 = 0; c8 < 16; ++c8) {
                 float e[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
+                for (int u = 0; u < 8; ++u)
                     e[u] = fast_exp2(fmaf(x[c8 * 8 + u], c_l2, neg_m));
-                    se += e[u];
-                }
                 uint4 pk;
                 pk.x = pack_bf16x2(e[0], e[1]);
                 pk.y = pack_bf16x2(e[2], e[3]);
                 pk.z = pack_bf16x2(e[4], e[5]);
                 pk.w = pack_bf16x2(e[6], e[7]);
-                sr += (sum_bf16x2(pk.x) + sum_bf16x2(pk.y)) + (sum_bf16x2(pk.z) + sum_bf16x2(pk.w));
+                pe[0] += e[0] + e[1];
+                pe[1] += e[2] + e[3];
+                pe[2] += e[4] + e[5];
+                pe[3] += e[6] + e[7];
+                pr[0] += sum_bf16x2(pk.x);
+                pr[1] += sum_bf16x2(pk.y);
+                pr[2] += sum_bf16x2(pk.z);
+                pr[3] += sum_bf16x2(pk.w);
                 const int region = c8 >> 3, chunk = (c8 & 7) ^ (row & 7);
                 *reinterpret_cast<uint4 *>(prow + region * Q_REGION + chunk * 16) = pk;
             }
-            l_exact += se;
-            l_round += sr;
+            l_exact += (pe[0] + pe[1]) + (pe[2] + pe[3]);
+            l_round += (pr[0] + pr[1]) + (pr[2] + pr[3]);
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL]);

@@ -130,6 +130,8 @@ int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *str
     if (128 % G != 0)
         return SINKATTN_OK;
     const int P = 128 / G;
+    if (P % 16 != 0) // the K / V rings advance in 16-key chunks
+        return SINKATTN_OK;
     const int64_t span = (int64_t)P + window - 1;
     const int NS = (int)((span + 15) / 16 * 16);
     if (span > 256)
@@ -138,10 +140,14 @@ int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *str
     int st = device_info(&di);
     if (st != SINKATTN_OK)
         return st;
-    if (swa_packed_smem_bytes(NS) > di.smem_optin)
+    if (swa_packed_smem_bytes(NS, P) > di.smem_optin)
         return SINKATTN_OK;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tkc, tvc;
     if ((st = make_map(&tq, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, G, P)))
+        return st;
+    if ((st = make_map(&tkc, a->k, kDQ, a->Hkv, a->L, a->B, a->k_sh, a->k_sl, a->k_sb, 1, 16)))
+        return st;
+    if ((st = make_map(&tvc, a->v, kDV, a->Hkv, a->L, a->B, a->v_sh, a->v_sl, a->v_sb, 1, 16)))
         return st;
     if ((st = make_map(&tk, a->k, kDQ, a->Hkv, a->L, a->B, a->k_sh, a->k_sl, a->k_sb, 1, NS)))
         return st;
@@ -169,7 +175,8 @@ int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *str
     p.o_sh = a->o_sh;
     p.lse = a->lse;
     const int grid = (int)(items < di.sms ? items : di.sms);
-    const cudaError_t e = launch_prefill_swa_packed(tq, tk, tv, p, grid, (cudaStream_t)stream);
+    const cudaError_t e =
+        launch_prefill_swa_packed(tq, tk, tv, tkc, tvc, p, grid, (cudaStream_t)stream);
     *done = true;
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
