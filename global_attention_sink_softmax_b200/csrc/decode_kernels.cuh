@@ -24,13 +24,14 @@ namespace sinkattn {
 
 namespace dec {
 constexpr int KT = 64;                 // keys per shared-memory tile
-constexpr int NSTAGE = 4;
 constexpr int KROW = 384, VROW = 256;  // bytes per K row (192 dims) / V row (128 dims)
 constexpr int STAGE_K = KT * KROW;
 constexpr int STAGE_V = KT * VROW;
 constexpr int STAGE = STAGE_K + STAGE_V + KT; // + one validity byte per key
-constexpr int SMEM = NSTAGE * STAGE;
 constexpr int THREADS = 128;
+// cp.async ring depth and CTAs per SM: 4 stages (160 KB, 1 CTA / SM) or 2 stages (80 KB,
+// 2 CTAs / SM)
+__host__ __device__ constexpr int smem_bytes(int nstage) { return nstage * STAGE; }
 constexpr int RED_STRIDE = 70;         // floats per lane in the cross-warp combine
 } // namespace dec
 
@@ -104,7 +105,7 @@ SA_DEV void load_tile(const DecodeParams &p, uint8_t *stage, int vt, int ke, int
         stage[STAGE_K + STAGE_V + key] = r.valid ? 1 : 0;
 }
 
-template <int KP>
+template <int KP, int NSTAGE>
 SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
 {
     using namespace dec;
@@ -391,11 +392,12 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
 
 // KP = warps that split each tile's keys: 4 when the unit has one 16-row m-tile (T x G <= 16),
 // 2 for two m-tiles, 1 for three or four.
-template <int KP>
-__global__ void __launch_bounds__(dec::THREADS) decode_split_kernel(const DecodeParams p)
+template <int KP, int NSTAGE>
+__global__ void __launch_bounds__(dec::THREADS, NSTAGE == 2 ? 2 : 1)
+    decode_split_kernel(const DecodeParams p)
 {
     extern __shared__ __align__(128) uint8_t dsmem[];
-    decode_body<KP>(p, dsmem);
+    decode_body<KP, NSTAGE>(p, dsmem);
 }
 
 // Merge the spans of each query row, counting the sink once. One warp per (b, t, h) row; each
@@ -442,6 +444,22 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
         p.lse[((int64_t)b * p.T + t) * p.Hq + h] = (m + fast_log2(le)) * kLn2;
 }
 
+template <int NSTAGE>
+cudaError_t launch_decode_split(const DecodeParams &p, cudaStream_t stream)
+{
+    dim3 grid(p.splits, p.Hkv, p.B);
+    const int smem = dec::smem_bytes(NSTAGE);
+    if (p.MT == 1)
+        decode_split_kernel<4, NSTAGE><<<grid, dec::THREADS, smem, stream>>>(p);
+    else if (p.MT == 2)
+        decode_split_kernel<2, NSTAGE><<<grid, dec::THREADS, smem, stream>>>(p);
+    else
+        decode_split_kernel<1, NSTAGE><<<grid, dec::THREADS, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+int decode_stages(const DecodeParams &p);
+
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream)
 {
     static int configured_devices = 0;
@@ -450,24 +468,21 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream)
     if (e != cudaSuccess)
         return e;
     if (dev < 32 && !(configured_devices & (1 << dev))) {
-        const void *fns[3] = {(const void *)decode_split_kernel<4>,
-                              (const void *)decode_split_kernel<2>,
-                              (const void *)decode_split_kernel<1>};
-        for (int i = 0; i < 3; ++i) {
-            e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize, dec::SMEM);
+        const void *fns[6] = {(const void *)decode_split_kernel<4, 4>,
+                              (const void *)decode_split_kernel<2, 4>,
+                              (const void *)decode_split_kernel<1, 4>,
+                              (const void *)decode_split_kernel<4, 2>,
+                              (const void *)decode_split_kernel<2, 2>,
+                              (const void *)decode_split_kernel<1, 2>};
+        for (int i = 0; i < 6; ++i) {
+            e = cudaFuncSetAttribute(fns[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     dec::smem_bytes(i < 3 ? 4 : 2));
             if (e != cudaSuccess)
                 return e;
         }
         configured_devices |= (1 << dev);
     }
-    dim3 grid(p.splits, p.Hkv, p.B);
-    if (p.MT == 1)
-        decode_split_kernel<4><<<grid, dec::THREADS, dec::SMEM, stream>>>(p);
-    else if (p.MT == 2)
-        decode_split_kernel<2><<<grid, dec::THREADS, dec::SMEM, stream>>>(p);
-    else
-        decode_split_kernel<1><<<grid, dec::THREADS, dec::SMEM, stream>>>(p);
-    e = cudaGetLastError();
+    e = decode_stages(p) == 2 ? launch_decode_split<2>(p, stream) : launch_decode_split<4>(p, stream);
     if (e != cudaSuccess || p.splits == 1)
         return e;
     const int64_t rows = (int64_t)p.B * p.T * p.Hq;

@@ -429,6 +429,17 @@ cudaError_t noalloc_workspace_ptr(void **out)
 
 } // namespace
 
+namespace sinkattn {
+// Pipeline depth of the split-KV decode kernel: 2 stages let two CTAs share an SM, which
+// measured faster than one CTA with 4 stages for every decode workload (GA 262144-token
+// context, SWA ring, hybrid verify).
+int decode_stages(const DecodeParams &p)
+{
+    (void)p;
+    return 2;
+}
+} // namespace sinkattn
+
 extern "C" {
 
 const char *sinkattn_status_string(int status)
