@@ -98,6 +98,9 @@ class PrefillRunner:
         self.lse = torch.empty(w.B, w.Hq, w.L, dtype=torch.float32, device=dev)
         self.flops, self.bytes = prefill_counts(w)
         self.launches = 1
+        # the kernel the library dispatches this workload to
+        packed = w.window > 0 and w.Hq // w.Hkv == 8 and w.window <= 128
+        self.kernel = "prefill_swa_packed_kernel" if packed else "prefill_band_kernel"
         self.workload = w.name
         self.config = dict(B=w.B, L=w.L, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
                            window=w.window, kind="SWA" if w.window else "GA")
@@ -157,6 +160,7 @@ class DecodeRunner:
                                                  d["k_cache"], d["v_cache"], **self.kw)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.launches = 1 if need == 0 else 2
+        self.kernel = "decode_split_kernel" if w.kind == W.KV_CONTIG else None
         self.flops, self.bytes = decode_counts(w, d)
         self.workload = w.name
         self.config = dict(B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
@@ -315,6 +319,26 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def measured_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu table, or None when the kernel's
+    sources changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    entry = json.load(open(path)).get(kernel)
+    if not entry or entry.get("bytes_per_launch") is None:
+        return None
+    csrc = os.path.join(ROOT, "global_attention_sink_softmax_b200", "csrc")
+    files = {"prefill_swa_packed_kernel": ["common.cuh", "swa_kernels.cuh"],
+             "prefill_band_kernel": ["common.cuh", "prefill_kernels.cuh"],
+             "decode_split_kernel": ["common.cuh", "decode_kernels.cuh"]}[kernel]
+    m = hashlib.sha256()
+    for f in files:
+        m.update(open(os.path.join(csrc, f), "rb").read())
+    return entry["bytes_per_launch"] if m.hexdigest() == entry.get("source_sha256") else None
+
+
 def roofline(runner, ms_per_launch, peaks, source, bound=None):
     ai = runner.flops / max(1, runner.bytes)
     ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
@@ -325,9 +349,12 @@ def roofline(runner, ms_per_launch, peaks, source, bound=None):
     else:
         achieved = runner.bytes / (ms_per_launch * 1e-3) / 1e9
         peak, unit = peaks["hbm_gbs"], "GB/s"
+    kernel = getattr(runner, "kernel", None)
+    traffic = measured_traffic(kernel) if kernel else None
     return {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": unit,
-            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": source,
-            "algorithmic_flops": runner.flops, "algorithmic_bytes": runner.bytes}
+            "frac": round(achieved / peak, 4), "traffic": traffic, "kernel": kernel,
+            "peak_source": source, "algorithmic_flops": runner.flops,
+            "algorithmic_bytes": runner.bytes}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -353,13 +380,12 @@ def omp_threads():
     return int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
 
 
-def cpu_baseline_prefill(w, d_cpu, target_s=10.0):
-    """Times the oracle on growing row samples until about target_s of CPU work."""
-    n = 64
+def cpu_baseline_prefill(w, d_cpu, target_s=12.0):
+    """Times the oracle on a row sample sized for about target_s seconds of CPU work."""
+    n = 256
     flops, dt = oracle_prefill_sample(w, d_cpu, n)
-    while dt < target_s / 4 and n < 1 << 20:
-        n *= 4 if dt < target_s / 16 else 2
-        flops, dt = oracle_prefill_sample(w, d_cpu, n, seed=n)
+    n = max(n, min(1 << 22, int(n * target_s / max(dt, 1e-3))))
+    flops, dt = oracle_prefill_sample(w, d_cpu, n, seed=n)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": omp_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
             "sample": f"{n} random (batch, position) rows x all {w.Hq} heads of {w.name}"}
