@@ -160,7 +160,7 @@ class DecodeRunner:
                                                  d["k_cache"], d["v_cache"], **self.kw)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.launches = 1 if need == 0 else 2
-        self.kernel = "decode_split_kernel" if w.kind == W.KV_CONTIG else None
+        self.kernel = "decode_tma_kernel" if w.kind == W.KV_CONTIG else None
         self.flops, self.bytes = decode_counts(w, d)
         self.workload = w.name
         self.config = dict(B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
@@ -332,7 +332,9 @@ def measured_traffic(kernel):
     csrc = os.path.join(ROOT, "global_attention_sink_softmax_b200", "csrc")
     files = {"prefill_swa_packed_kernel": ["common.cuh", "swa_kernels.cuh"],
              "prefill_band_kernel": ["common.cuh", "prefill_kernels.cuh"],
-             "decode_split_kernel": ["common.cuh", "decode_kernels.cuh"]}[kernel]
+             "decode_split_kernel": ["common.cuh", "decode_kernels.cuh"],
+             "decode_tma_kernel": ["common.cuh", "decode_kernels.cuh",
+                                   "decode_tma_kernels.cuh"]}[kernel]
     m = hashlib.sha256()
     for f in files:
         m.update(open(os.path.join(csrc, f), "rb").read())

@@ -105,6 +105,66 @@ SA_DEV void load_tile(const DecodeParams &p, uint8_t *stage, int vt, int ke, int
         stage[STAGE_K + STAGE_V + key] = r.valid ? 1 : 0;
 }
 
+// Writes the result of one consumer warp's rows (lane/4 and lane/4 + 8 of its m-tile): with a
+// single span, the final O and LSE (the sink applied once: m_f = max(m, sink),
+// D = l e^(m - m_f) + e^(sink - m_f)); otherwise the span's partial (O, m, l_rounded, l_exact).
+SA_DEV void decode_write_output(const DecodeParams &p, int b, int g, int split, int ra, int rb,
+                                int lane, const float (&o)[16][4], float m_a, float m_b,
+                                float l_a, float l_b, float e_a, float e_b)
+{
+    const int c2 = 2 * (lane & 3);
+    if (p.splits == 1) {
+        // apply the sink once and finish: m_f = max(m, sink), D = l e^(m - m_f) + e^(sink - m_f)
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int r = half ? rb : ra;
+            if (r >= p.R)
+                continue;
+            const int t = r / p.G, h = g * p.G + r % p.G;
+            const float m = half ? m_b : m_a, l = half ? l_b : l_a, le = half ? e_b : e_a;
+            const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
+            const float mf = fmaxf(m, sk);
+            const float cm = (m == -INFINITY) ? 0.f : fast_exp2(m - mf);
+            const float cs = (sk == -INFINITY) ? 0.f : fast_exp2(sk - mf);
+            const float D = le * cm + cs;         // exact denominator: LSE
+            const float scl = cm / (l * cm + cs); // rounded-P denominator: O
+            uint16_t *orow = p.o + (int64_t)b * p.o_sb + (int64_t)t * p.o_st + (int64_t)h * p.o_sh;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float x0 = (half ? o[i][2] : o[i][0]) * scl;
+                const float x1 = (half ? o[i][3] : o[i][1]) * scl;
+                *reinterpret_cast<uint32_t *>(orow + i * 8 + c2) = pack_bf16x2(x0, x1);
+            }
+            if (p.lse && (lane & 3) == 0)
+                p.lse[((int64_t)b * p.T + t) * p.Hq + h] = (mf + fast_log2(D)) * kLn2;
+        }
+    } else {
+        const int64_t unit = ((int64_t)b * p.Hkv + g) * p.splits + split;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int r = half ? rb : ra;
+            if (r >= p.R)
+                continue;
+            float *wo = p.ws_o + (unit * p.R + r) * 128;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float2 v2;
+                v2.x = half ? o[i][2] : o[i][0];
+                v2.y = half ? o[i][3] : o[i][1];
+                *reinterpret_cast<float2 *>(wo + i * 8 + c2) = v2;
+            }
+            if ((lane & 3) == 0) {
+                float4 ml;
+                ml.x = half ? m_b : m_a;
+                ml.y = half ? l_b : l_a;
+                ml.z = half ? e_b : e_a;
+                ml.w = 0.f;
+                *reinterpret_cast<float4 *>(p.ws_ml + (unit * p.R + r) * 4) = ml;
+            }
+        }
+    }
+}
+
 template <int KP, int NSTAGE>
 SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
 {
@@ -336,58 +396,7 @@ SA_DEV void decode_body(const DecodeParams &p, uint8_t *smem)
     if (!active || ks != 0)
         return;
 
-    // ---- output
-    const int c2 = 2 * (lane & 3);
-    if (p.splits == 1) {
-        // apply the sink once and finish: m_f = max(m, sink), D = l e^(m - m_f) + e^(sink - m_f)
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int r = half ? rb : ra;
-            if (r >= p.R)
-                continue;
-            const int t = r / p.G, h = g * p.G + r % p.G;
-            const float m = half ? m_b : m_a, l = half ? l_b : l_a, le = half ? e_b : e_a;
-            const float sk = p.sink ? p.sink[h] * kLog2e : -INFINITY;
-            const float mf = fmaxf(m, sk);
-            const float cm = (m == -INFINITY) ? 0.f : fast_exp2(m - mf);
-            const float cs = (sk == -INFINITY) ? 0.f : fast_exp2(sk - mf);
-            const float D = le * cm + cs;         // exact denominator: LSE
-            const float scl = cm / (l * cm + cs); // rounded-P denominator: O
-            uint16_t *orow = p.o + (int64_t)b * p.o_sb + (int64_t)t * p.o_st + (int64_t)h * p.o_sh;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float x0 = (half ? o[i][2] : o[i][0]) * scl;
-                const float x1 = (half ? o[i][3] : o[i][1]) * scl;
-                *reinterpret_cast<uint32_t *>(orow + i * 8 + c2) = pack_bf16x2(x0, x1);
-            }
-            if (p.lse && (lane & 3) == 0)
-                p.lse[((int64_t)b * p.T + t) * p.Hq + h] = (mf + fast_log2(D)) * kLn2;
-        }
-    } else {
-        const int64_t unit = ((int64_t)b * p.Hkv + g) * p.splits + split;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            const int r = half ? rb : ra;
-            if (r >= p.R)
-                continue;
-            float *wo = p.ws_o + (unit * p.R + r) * 128;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float2 v2;
-                v2.x = half ? o[i][2] : o[i][0];
-                v2.y = half ? o[i][3] : o[i][1];
-                *reinterpret_cast<float2 *>(wo + i * 8 + c2) = v2;
-            }
-            if ((lane & 3) == 0) {
-                float4 ml;
-                ml.x = half ? m_b : m_a;
-                ml.y = half ? l_b : l_a;
-                ml.z = half ? e_b : e_a;
-                ml.w = 0.f;
-                *reinterpret_cast<float4 *>(p.ws_ml + (unit * p.R + r) * 4) = ml;
-            }
-        }
-    }
+    decode_write_output(p, b, g, split, ra, rb, lane, o, m_a, m_b, l_a, l_b, e_a, e_b);
 }
 
 // KP = warps that split each tile's keys: 4 when the unit has one 16-row m-tile (T x G <= 16),
@@ -444,6 +453,13 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const DecodeParams p)
         p.lse[((int64_t)b * p.T + t) * p.Hq + h] = (m + fast_log2(le)) * kLn2;
 }
 
+cudaError_t launch_decode_merge(const DecodeParams &p, cudaStream_t stream)
+{
+    const int64_t rows = (int64_t)p.B * p.T * p.Hq;
+    decode_merge_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
 template <int NSTAGE>
 cudaError_t launch_decode_split(const DecodeParams &p, cudaStream_t stream)
 {
@@ -485,9 +501,7 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream)
     e = decode_stages(p) == 2 ? launch_decode_split<2>(p, stream) : launch_decode_split<4>(p, stream);
     if (e != cudaSuccess || p.splits == 1)
         return e;
-    const int64_t rows = (int64_t)p.B * p.T * p.Hq;
-    decode_merge_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_decode_merge(p, stream);
 }
 
 // ---------------------------------------------------------------------------------------------

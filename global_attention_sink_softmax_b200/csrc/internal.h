@@ -73,6 +73,12 @@ struct DecodeParams {
 };
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream);
+// TMA-fed decode: cache maps {d, Hkv, rows, blocks} (rows = ring slots / positions / page rows,
+// blocks = sequences or pages) and new-token maps {d, Hkv, T, B}, box {64, 1, 64, 1}.
+cudaError_t launch_decode_tma(const CUtensorMap &kc, const CUtensorMap &vc, const CUtensorMap &kn,
+                              const CUtensorMap &vn, const DecodeParams &p, cudaStream_t stream);
+cudaError_t launch_decode_merge(const DecodeParams &p, cudaStream_t stream);
+int decode_stages(const DecodeParams &p);
 
 struct CommitParams {
     int kind, B, T, Hkv;

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "decode_kernels.cuh"
+#include "decode_tma_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
 #include "swa_kernels.cuh"
@@ -427,6 +428,42 @@ cudaError_t noalloc_workspace_ptr(void **out)
     return cudaSuccess;
 }
 
+// The TMA-fed decode kernel takes whole 64-key tiles: contiguous caches, and paged caches whose
+// pages hold a multiple of 64 tokens (without a window, so tiles stay page-aligned). Rings
+// (a 128-slot ring is two tiles plus a tile of new tokens per CTA) and other page sizes use the
+// cp.async kernel, which is faster there.
+bool decode_tma_ok(const sinkattn_decode_args *a, const DecodeParams &)
+{
+    if (a->kind == SINKATTN_KV_CONTIG)
+        return true;
+    if (a->kind == SINKATTN_KV_PAGED)
+        return a->window == 0 && a->page_size % 64 == 0;
+    return false;
+}
+
+int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *stream)
+{
+    cudaError_t e;
+    if (decode_tma_ok(a, p)) {
+        const int rows = a->kind == SINKATTN_KV_RING ? a->ring_cap
+                         : a->kind == SINKATTN_KV_CONTIG ? a->max_ctx
+                                                         : a->page_size;
+        const int blocks = a->kind == SINKATTN_KV_PAGED ? a->num_pages : a->B;
+        CUtensorMap kc, vc, kn, vn;
+        // a cache the tensor-map encoder rejects (e.g. an empty one) takes the cp.async kernel
+        if (rows > 0 &&
+            !make_map(&kc, a->k_cache, kDQ, a->Hkv, rows, blocks, a->kc_sh, a->kc_ss, a->kc_sb, 1, 64) &&
+            !make_map(&vc, a->v_cache, kDV, a->Hkv, rows, blocks, a->vc_sh, a->vc_ss, a->vc_sb, 1, 64) &&
+            !make_map(&kn, a->k_new, kDQ, a->Hkv, a->T, a->B, a->kn_sh, a->kn_st, a->kn_sb, 1, 64) &&
+            !make_map(&vn, a->v_new, kDV, a->Hkv, a->T, a->B, a->vn_sh, a->vn_st, a->vn_sb, 1, 64)) {
+            e = launch_decode_tma(kc, vc, kn, vn, p, (cudaStream_t)stream);
+            return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+        }
+    }
+    e = launch_decode(p, (cudaStream_t)stream);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
 } // namespace
 
 namespace sinkattn {
@@ -492,8 +529,7 @@ int sinkattn_decode(const sinkattn_decode_args *args, void *workspace, size_t ws
     }
     DecodeParams p;
     fill_decode_params(p, args, s, need > 0 ? workspace : nullptr);
-    const cudaError_t e = launch_decode(p, (cudaStream_t)stream);
-    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+    return run_decode(args, p, stream);
 }
 
 int sinkattn_decode_noalloc(const sinkattn_decode_args *args, void *stream)
@@ -512,8 +548,7 @@ int sinkattn_decode_noalloc(const sinkattn_decode_args *args, void *stream)
     // whatever an earlier call left in the array needs no clearing.
     DecodeParams p;
     fill_decode_params(p, args, s, need > 0 ? ws : nullptr);
-    const cudaError_t e = launch_decode(p, (cudaStream_t)stream);
-    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+    return run_decode(args, p, stream);
 }
 
 int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, void *stream)
