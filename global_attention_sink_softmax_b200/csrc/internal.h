@@ -77,6 +77,11 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream);
 // blocks = sequences or pages) and new-token maps {d, Hkv, T, B}, box {64, 1, 64, 1}.
 cudaError_t launch_decode_tma(const CUtensorMap &kc, const CUtensorMap &vc, const CUtensorMap &kn,
                               const CUtensorMap &vn, const DecodeParams &p, cudaStream_t stream);
+// tcgen05 decode for blocks of 17..64 query rows: q map {192, Hq, T, B} box {64, G, T, 1},
+// new-token maps with a 16-row box.
+cudaError_t launch_decode_umma(const CUtensorMap &q, const CUtensorMap &kc, const CUtensorMap &vc,
+                               const CUtensorMap &kn, const CUtensorMap &vn, const DecodeParams &p,
+                               cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeParams &p, cudaStream_t stream);
 int decode_stages(const DecodeParams &p);
 

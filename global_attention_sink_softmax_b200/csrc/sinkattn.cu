@@ -10,6 +10,7 @@
 #include "common.cuh"
 #include "decode_kernels.cuh"
 #include "decode_tma_kernels.cuh"
+#include "decode_umma_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
 #include "swa_kernels.cuh"
@@ -449,15 +450,25 @@ int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *strea
                          : a->kind == SINKATTN_KV_CONTIG ? a->max_ctx
                                                          : a->page_size;
         const int blocks = a->kind == SINKATTN_KV_PAGED ? a->num_pages : a->B;
-        CUtensorMap kc, vc, kn, vn;
-        // a cache the tensor-map encoder rejects (e.g. an empty one) takes the cp.async kernel
+        CUtensorMap kc, vc, kn, vn, q;
+        // blocks of more than 16 query rows go to the tcgen05 kernel, with the new tokens as a
+        // 16-row box; a cache the tensor-map encoder rejects (e.g. an empty one) takes the
+        // cp.async kernel
+        const int new_rows = p.R > 16 ? 16 : 64;
         if (rows > 0 &&
             !make_map(&kc, a->k_cache, kDQ, a->Hkv, rows, blocks, a->kc_sh, a->kc_ss, a->kc_sb, 1, 64) &&
             !make_map(&vc, a->v_cache, kDV, a->Hkv, rows, blocks, a->vc_sh, a->vc_ss, a->vc_sb, 1, 64) &&
-            !make_map(&kn, a->k_new, kDQ, a->Hkv, a->T, a->B, a->kn_sh, a->kn_st, a->kn_sb, 1, 64) &&
-            !make_map(&vn, a->v_new, kDV, a->Hkv, a->T, a->B, a->vn_sh, a->vn_st, a->vn_sb, 1, 64)) {
-            e = launch_decode_tma(kc, vc, kn, vn, p, (cudaStream_t)stream);
-            return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+            !make_map(&kn, a->k_new, kDQ, a->Hkv, a->T, a->B, a->kn_sh, a->kn_st, a->kn_sb, 1, new_rows) &&
+            !make_map(&vn, a->v_new, kDV, a->Hkv, a->T, a->B, a->vn_sh, a->vn_st, a->vn_sb, 1, new_rows)) {
+            if (p.R > 16) {
+                if (!make_map(&q, a->q, kDQ, a->Hq, a->T, a->B, a->q_sh, a->q_st, a->q_sb, p.G, a->T)) {
+                    e = launch_decode_umma(q, kc, vc, kn, vn, p, (cudaStream_t)stream);
+                    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+                }
+            } else {
+                e = launch_decode_tma(kc, vc, kn, vn, p, (cudaStream_t)stream);
+                return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+            }
         }
     }
     e = launch_decode(p, (cudaStream_t)stream);

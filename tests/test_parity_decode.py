@@ -128,6 +128,60 @@ def test_paged_decode(P, T):
     check(sa.KV_PAGED, d, 0, f"paged P{P} T{T}")
 
 
+@pytest.mark.parametrize("P", [128, 16])
+@pytest.mark.parametrize("T", [1, 2])
+def test_paged_decode_missing_pages(P, T):
+    """Page ids outside the pool hide that page's keys (the library's contract for a sparse
+    page table). Without a window every cached key is visible whatever its position, so the
+    answer is the oracle on a contiguous cache holding only the present pages' rows."""
+    g = torch.Generator().manual_seed(900 + P + T)
+    B, Hq, Hkv = 3, 64, 4
+    ctx = [5 * P + 7, 3 * P, 2 * P - 1]
+    max_pages = max((c + P - 1) // P for c in ctx)
+    npg = [(c + P - 1) // P for c in ctx]
+    total = sum(npg)
+    perm = torch.randperm(total, generator=g).to(torch.int32)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    off = 0
+    for b, n in enumerate(npg):
+        table[b, :n] = perm[off:off + n]
+        off += n
+    table[0, 1] = -1         # a hole in the middle
+    table[0, 4] = total + 3  # an id past the pool
+    table[1, 0] = -7         # the first page
+    table[2, 1] = total      # the last, partial page
+    kc, vc = rnd((total, P, Hkv, 192), g), rnd((total, P, Hkv, 128), g)
+    d = dict(q=rnd((B, T, Hq, 192), g), k_new=rnd((B, T, Hkv, 192), g),
+             v_new=rnd((B, T, Hkv, 128), g), k_cache=kc, v_cache=vc,
+             sink=make_sink(Hq, g, "mixed"), ctx_len=torch.tensor(ctx, dtype=torch.int32),
+             page_table=table, max_ctx=max_pages * P)
+    o, lse = gpu_decode(sa.KV_PAGED, d, 0)
+    assert sa.sinkattn_take_device_error() == 0
+    # the keys that stay: rows c < ctx of pages whose id is in the pool, in position order
+    rows_k, rows_v, kept = [], [], []
+    for b in range(B):
+        ks, vs = [], []
+        for c in range(ctx[b]):
+            pid = int(table[b, c // P])
+            if 0 <= pid < total:
+                ks.append(kc[pid, c % P])
+                vs.append(vc[pid, c % P])
+        kept.append(len(ks))
+        rows_k.append(ks)
+        rows_v.append(vs)
+    assert kept[0] == ctx[0] - 2 * P and kept[1] == ctx[1] - P and kept[2] == P
+    maxc = max(kept)
+    kcc = torch.zeros(B, maxc, Hkv, 192, dtype=torch.bfloat16)
+    vcc = torch.zeros(B, maxc, Hkv, 128, dtype=torch.bfloat16)
+    for b in range(B):
+        if kept[b]:
+            kcc[b, :kept[b]] = torch.stack(rows_k[b])
+            vcc[b, :kept[b]] = torch.stack(rows_v[b])
+    dc = dict(d, k_cache=kcc, v_cache=vcc, ctx_len=torch.tensor(kept, dtype=torch.int32))
+    ro, rl, _ = oracle_decode(sa.KV_CONTIG, dc, 0)
+    assert_close(o, ro, lse, rl, f"paged P{P} T{T} with missing pages")
+
+
 def test_full_size_swa_ring_decode():
     """B=256 sequences, 128-slot ring, 64 Q / 8 KV heads: every output."""
     w = W.SWA_DECODE
