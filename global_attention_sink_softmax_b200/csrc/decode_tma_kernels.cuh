@@ -40,17 +40,18 @@ struct DecodeTiles {
     bool has_new;    // plus one tile of new tokens
 };
 
-SA_DEV DecodeTiles decode_tiles(const DecodeParams &p, int b, int split)
+// Tiles of span `split` of sequence b, from its cached length (ring_len or ctx_len) and ring
+// head (0 for other caches).
+SA_DEV DecodeTiles decode_tiles(const DecodeParams &p, int split, int len, int head)
 {
     DecodeTiles d;
-    int n_cache = (p.kind == 0) ? p.ring_len[b] : p.ctx_len[b];
-    d.n_cache = max(0, min(n_cache, p.kind == 0 ? p.ring_cap : p.max_ctx));
+    d.n_cache = max(0, min(len, p.kind == 0 ? p.ring_cap : p.max_ctx));
     d.n_used = (p.window > 0) ? min(d.n_cache, p.window - 1) : d.n_cache;
     d.first_c = d.n_cache - d.n_used;
     d.n_total = d.n_used + p.T;
     d.kb = split * p.chunk;
     d.ke = min(d.kb + p.chunk, d.n_total);
-    d.ring_head = (p.kind == 0) ? ((p.ring_head[b] % p.ring_cap) + p.ring_cap) % p.ring_cap : 0;
+    d.ring_head = (p.kind == 0) ? ((head % p.ring_cap) + p.ring_cap) % p.ring_cap : 0;
     if (p.kind == 0) {
         d.cache_tiles = (d.kb < d.n_used) ? p.ring_cap / dt::KT : 0; // one span holds the ring
     } else {
@@ -59,6 +60,12 @@ SA_DEV DecodeTiles decode_tiles(const DecodeParams &p, int b, int split)
     }
     d.has_new = d.ke > d.n_used && d.kb < d.n_total;
     return d;
+}
+
+SA_DEV DecodeTiles decode_tiles(const DecodeParams &p, int b, int split)
+{
+    return p.kind == 0 ? decode_tiles(p, split, p.ring_len[b], p.ring_head[b])
+                       : decode_tiles(p, split, p.ctx_len[b], 0);
 }
 
 // Whether tile t's keys come from a page that exists (a page id outside the pool hides them).
@@ -79,8 +86,8 @@ SA_DEV void decode_key(const DecodeParams &p, const DecodeTiles &d, int t, int i
 {
     if (t < d.cache_tiles) {
         if (p.kind == 0) {
-            const int slot = t * dt::KT + i;
-            const int c = (slot - d.ring_head + p.ring_cap) % p.ring_cap;
+            const int slot = t * dt::KT + i; // slot and head both lie in [0, ring_cap)
+            const int c = slot >= d.ring_head ? slot - d.ring_head : slot - d.ring_head + p.ring_cap;
             valid = c >= d.first_c && c < d.n_cache;
             pos = c - d.n_cache;
         } else {

@@ -77,11 +77,12 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream);
 // blocks = sequences or pages) and new-token maps {d, Hkv, T, B}, box {64, 1, 64, 1}.
 cudaError_t launch_decode_tma(const CUtensorMap &kc, const CUtensorMap &vc, const CUtensorMap &kn,
                               const CUtensorMap &vn, const DecodeParams &p, cudaStream_t stream);
-// tcgen05 decode for blocks of 17..64 query rows: q map {192, Hq, T, B} box {64, G, T, 1},
-// new-token maps with a 16-row box.
+// tcgen05 decode (query blocks of 17..64 rows, and rings): q map {192, Hq, T, B} box
+// {64, G, T, 1}, new-token maps with a 16-row box. max_ctas > 0 caps the grid (the CTAs then
+// loop over the work items); 0 launches one CTA per item.
 cudaError_t launch_decode_umma(const CUtensorMap &q, const CUtensorMap &kc, const CUtensorMap &vc,
                                const CUtensorMap &kn, const CUtensorMap &vn, const DecodeParams &p,
-                               cudaStream_t stream);
+                               int max_ctas, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeParams &p, cudaStream_t stream);
 int decode_stages(const DecodeParams &p);
 

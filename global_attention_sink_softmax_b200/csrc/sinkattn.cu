@@ -429,10 +429,10 @@ cudaError_t noalloc_workspace_ptr(void **out)
     return cudaSuccess;
 }
 
-// The TMA-fed decode kernel takes whole 64-key tiles: contiguous caches, and paged caches whose
-// pages hold a multiple of 64 tokens (without a window, so tiles stay page-aligned). Rings
-// (a 128-slot ring is two tiles plus a tile of new tokens per CTA) and other page sizes use the
-// cp.async kernel, which is faster there.
+// The TMA-fed decode kernels take whole 64-key tiles: contiguous caches, and paged caches whose
+// pages hold a multiple of 64 tokens (without a window, so tiles stay page-aligned). Rings and
+// other page sizes use the cp.async kernel: on a 128-slot ring each (sequence, KV head) item is
+// only 80 KB, and there the cp.async kernel, two CTAs per SM, is the faster of the two.
 bool decode_tma_ok(const sinkattn_decode_args *a, const DecodeParams &)
 {
     if (a->kind == SINKATTN_KV_CONTIG)
@@ -450,23 +450,27 @@ int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *strea
                          : a->kind == SINKATTN_KV_CONTIG ? a->max_ctx
                                                          : a->page_size;
         const int blocks = a->kind == SINKATTN_KV_PAGED ? a->num_pages : a->B;
+        // tcgen05 kernel: blocks of more than 16 query rows; the mma.sync TMA kernel: up to 16
+        const bool umma = p.R > 16 || a->kind == SINKATTN_KV_RING;
+        const int new_rows = umma ? 16 : 64;
         CUtensorMap kc, vc, kn, vn, q;
-        // blocks of more than 16 query rows go to the tcgen05 kernel, with the new tokens as a
-        // 16-row box; a cache the tensor-map encoder rejects (e.g. an empty one) takes the
-        // cp.async kernel
-        const int new_rows = p.R > 16 ? 16 : 64;
+        // a cache the tensor-map encoder rejects (e.g. an empty one) takes the cp.async kernel
         if (rows > 0 &&
             !make_map(&kc, a->k_cache, kDQ, a->Hkv, rows, blocks, a->kc_sh, a->kc_ss, a->kc_sb, 1, 64) &&
             !make_map(&vc, a->v_cache, kDV, a->Hkv, rows, blocks, a->vc_sh, a->vc_ss, a->vc_sb, 1, 64) &&
             !make_map(&kn, a->k_new, kDQ, a->Hkv, a->T, a->B, a->kn_sh, a->kn_st, a->kn_sb, 1, new_rows) &&
             !make_map(&vn, a->v_new, kDV, a->Hkv, a->T, a->B, a->vn_sh, a->vn_st, a->vn_sb, 1, new_rows)) {
-            if (p.R > 16) {
-                if (!make_map(&q, a->q, kDQ, a->Hq, a->T, a->B, a->q_sh, a->q_st, a->q_sb, p.G, a->T)) {
-                    e = launch_decode_umma(q, kc, vc, kn, vn, p, (cudaStream_t)stream);
-                    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
-                }
-            } else {
+            if (!umma) {
                 e = launch_decode_tma(kc, vc, kn, vn, p, (cudaStream_t)stream);
+                return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+            }
+            DeviceInfo di;
+            const int st = device_info(&di);
+            if (st != SINKATTN_OK)
+                return st;
+            if (!make_map(&q, a->q, kDQ, a->Hq, a->T, a->B, a->q_sh, a->q_st, a->q_sb, p.G, a->T)) {
+                e = launch_decode_umma(q, kc, vc, kn, vn, p,
+                                       a->kind == SINKATTN_KV_RING ? di.sms : 0, (cudaStream_t)stream);
                 return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
             }
         }
