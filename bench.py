@@ -160,7 +160,12 @@ class DecodeRunner:
                                                  d["k_cache"], d["v_cache"], **self.kw)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.launches = 1 if need == 0 else 2
-        self.kernel = "decode_tma_kernel" if w.kind == W.KV_CONTIG else None
+        # the kernel the library dispatches this workload to
+        rows = w.T * (w.Hq // w.Hkv)
+        if w.kind == W.KV_RING or (w.kind == W.KV_PAGED and w.page_size % 64 != 0):
+            self.kernel = "decode_split_kernel"
+        else:
+            self.kernel = "decode_umma_kernel" if rows > 16 else "decode_tma_kernel"
         self.flops, self.bytes = decode_counts(w, d)
         self.workload = w.name
         self.config = dict(B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
@@ -197,6 +202,21 @@ class HybridRunner:
     def step(self):
         for r in self.layers:
             r.step()
+
+    def kind_runner(self, ring):
+        """The GA (ring=False) or SWA (ring=True) layers alone, for a per-kind breakdown."""
+        sel = [r for r in self.layers if (r.w.kind == W.KV_RING) == ring]
+
+        class Sub:
+            flops = sum(r.flops for r in sel)
+            bytes = sum(r.bytes for r in sel)
+            launches = sum(r.launches for r in sel)
+
+            @staticmethod
+            def step():
+                for r in sel:
+                    r.step()
+        return Sub
 
     def release(self):
         for r in self.layers:
@@ -334,7 +354,9 @@ def measured_traffic(kernel):
              "prefill_band_kernel": ["common.cuh", "prefill_kernels.cuh"],
              "decode_split_kernel": ["common.cuh", "decode_kernels.cuh"],
              "decode_tma_kernel": ["common.cuh", "decode_kernels.cuh",
-                                   "decode_tma_kernels.cuh"]}[kernel]
+                                   "decode_tma_kernels.cuh"],
+             "decode_umma_kernel": ["common.cuh", "decode_kernels.cuh",
+                                    "decode_tma_kernels.cuh", "decode_umma_kernels.cuh"]}[kernel]
     m = hashlib.sha256()
     for f in files:
         m.update(open(os.path.join(csrc, f), "rb").read())
@@ -467,7 +489,8 @@ def main():
     ap.add_argument("--ref-L", type=int, default=0, help="reference arm: shorter sequences (tests)")
     ap.add_argument("--small", action="store_true",
                     help="profiling case: prefill workloads at B=1 (SWA L=16384, GA L=8192), "
-                         "decode at B=2")
+                         "decode at B=2, SWA decode at B=64, hybrid verify as its first GA "
+                         "layer alone at B=8")
     args = ap.parse_args()
     world, rank, local = init_dist(args)
     args.gpus = max(args.gpus, world)
@@ -550,6 +573,11 @@ def main():
             jobs.append(("swa_decode", lambda: DecodeRunner(swad_w, dev), "flush"))
         if only in (None, "hybrid") and not args.small:
             jobs.append(("hybrid", lambda: HybridRunner(dev), None))
+        if only == "hybrid" and args.small:
+            import dataclasses
+            hyb0 = W.hybrid_layer_workload(0)
+            hyb0 = dataclasses.replace(hyb0, B=8, name=hyb0.name + "_small_B8")
+            jobs.append(("hybrid_ga_layer", lambda: DecodeRunner(hyb0, dev), None))
         for name, make, fl in jobs:
             r = make()
             flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if fl else None
@@ -566,6 +594,15 @@ def main():
             if name == "hybrid":
                 entry["note"] = ("layer list taken literally: 49 layer calls (9 GA, 40 SWA); "
                                  "GB/s over all layers' algorithmic bytes")
+                # the GA and the SWA layers timed on their own (the GA layers carry the target)
+                by_kind = {}
+                for kind, ring in (("ga_layers", False), ("swa_layers", True)):
+                    sub = r.kind_runner(ring)
+                    ms_k = measure(sub, steps, max(3, args.warmup), None, world) / steps
+                    by_kind[kind] = {"ms_per_step": round(ms_k, 4),
+                                     "gbs": round(sub.bytes / (ms_k * 1e-3) / 1e9, 2),
+                                     "roofline": roofline(sub, ms_k, peaks, peak_src, bound="hbm")}
+                entry["by_kind"] = by_kind
             secondary[name] = entry
             r.release()
             del r, flush

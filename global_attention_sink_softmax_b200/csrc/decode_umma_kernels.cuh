@@ -495,16 +495,21 @@ __global__ void __launch_bounds__(du::THREADS, 1)
             bool ok = true;
             int k = cg;
             for (int j = grp; j < x.nsteps; j += 2, ++k) {
+                // Cache tiles and the new tokens take the same path: the new tokens are keys
+                // 0..T-1 of an N = 16 step, which all fall in key part 0 (the other parts'
+                // columns hold stale values and are masked).
+                const bool cache = j < x.ct;
+                // a paged tile's page id, loaded before the wait so its latency hides there
+                const int pg = cache && p.kind == 2 ? (d.first_c + d.kb + j * KT) / p.page_size : 0;
+                const int pid = cache && p.kind == 2 && pg < p.max_pages
+                                    ? __ldg(p.page_table + (int64_t)x.b * p.max_pages + pg)
+                                    : -1;
                 ok = warp_wait(&bars[B_SFULL + grp], k & 1, abort);
                 if (!ok)
                     break;
                 tc_fence_after();
                 const uint32_t saddr = tmem + lane_addr + grp * 64;
-                // Cache tiles and the new tokens take the same path: the new tokens are keys
-                // 0..T-1 of an N = 16 step, which all fall in key part 0 (the other parts'
-                // columns hold stale values and are masked).
-                const bool cache = j < x.ct;
-                const bool tile_ok = !cache || decode_tile_ok(p, d, x.b, j);
+                const bool tile_ok = !cache || p.kind != 2 || (pid >= 0 && pid < p.num_pages);
                 if (cache) {
                     const KeySpan present = du_span(p, d, j, tile_ok, false, 0);
                     if (!present.covers(KT)) {

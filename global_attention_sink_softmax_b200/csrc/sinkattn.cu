@@ -238,6 +238,8 @@ Split plan_split(const sinkattn_decode_args *a)
 {
     const int64_t n = max_unit_keys(a);
     const int64_t units = (int64_t)a->B * a->Hkv;
+    // about 8 spans per SM (shorter spans even out ragged lengths but each CTA's start and
+    // epilogue cost more than that gains)
     int64_t splits = (kNumSMs * 8 + units - 1) / units;
     const int64_t by_len = (n + kMinSpanKeys - 1) / kMinSpanKeys;
     if (splits > by_len)
