@@ -162,7 +162,9 @@ class DecodeRunner:
         self.launches = 1 if need == 0 else 2
         # the kernel the library dispatches this workload to
         rows = w.T * (w.Hq // w.Hkv)
-        if w.kind == W.KV_RING or (w.kind == W.KV_PAGED and w.page_size % 64 != 0):
+        if w.kind == W.KV_RING:
+            self.kernel = "decode_ring_kernel"
+        elif w.kind == W.KV_PAGED and w.page_size % 64 != 0:
             self.kernel = "decode_split_kernel"
         else:
             self.kernel = "decode_umma_kernel" if rows > 16 else "decode_tma_kernel"
@@ -356,7 +358,9 @@ def measured_traffic(kernel):
              "decode_tma_kernel": ["common.cuh", "decode_kernels.cuh",
                                    "decode_tma_kernels.cuh"],
              "decode_umma_kernel": ["common.cuh", "decode_kernels.cuh",
-                                    "decode_tma_kernels.cuh", "decode_umma_kernels.cuh"]}[kernel]
+                                    "decode_tma_kernels.cuh", "decode_umma_kernels.cuh"],
+             "decode_ring_kernel": ["common.cuh", "decode_kernels.cuh",
+                                    "decode_ring_kernels.cuh"]}[kernel]
     m = hashlib.sha256()
     for f in files:
         m.update(open(os.path.join(csrc, f), "rb").read())

@@ -83,6 +83,11 @@ cudaError_t launch_decode_tma(const CUtensorMap &kc, const CUtensorMap &vc, cons
 cudaError_t launch_decode_umma(const CUtensorMap &q, const CUtensorMap &kc, const CUtensorMap &vc,
                                const CUtensorMap &kn, const CUtensorMap &vn, const DecodeParams &p,
                                int max_ctas, cudaStream_t stream);
+// Ring decode, one warp per (sequence, KV head, m16 row tile) item (one span): cache maps
+// {d, Hkv, ring_cap, B} and new-token maps {d, Hkv, T, B}, box {64, 1, 32, 1}.
+cudaError_t launch_decode_ring(const CUtensorMap &kc, const CUtensorMap &vc, const CUtensorMap &kn,
+                               const CUtensorMap &vn, const DecodeParams &p, int sms,
+                               cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeParams &p, cudaStream_t stream);
 int decode_stages(const DecodeParams &p);
 

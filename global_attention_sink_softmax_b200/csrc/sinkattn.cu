@@ -11,6 +11,7 @@
 #include "decode_kernels.cuh"
 #include "decode_tma_kernels.cuh"
 #include "decode_umma_kernels.cuh"
+#include "decode_ring_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
 #include "swa_kernels.cuh"
@@ -447,6 +448,21 @@ bool decode_tma_ok(const sinkattn_decode_args *a, const DecodeParams &)
 int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *stream)
 {
     cudaError_t e;
+    if (a->kind == SINKATTN_KV_RING && a->ring_cap % 32 == 0 && p.splits == 1) {
+        // a ring item (an m16 tile of a unit's rows) per warp, streamed in 32-key chunks
+        CUtensorMap kc, vc, kn, vn;
+        DeviceInfo di;
+        int st = device_info(&di);
+        if (st != SINKATTN_OK)
+            return st;
+        if (!make_map(&kc, a->k_cache, kDQ, a->Hkv, a->ring_cap, a->B, a->kc_sh, a->kc_ss, a->kc_sb, 1, 32) &&
+            !make_map(&vc, a->v_cache, kDV, a->Hkv, a->ring_cap, a->B, a->vc_sh, a->vc_ss, a->vc_sb, 1, 32) &&
+            !make_map(&kn, a->k_new, kDQ, a->Hkv, a->T, a->B, a->kn_sh, a->kn_st, a->kn_sb, 1, 32) &&
+            !make_map(&vn, a->v_new, kDV, a->Hkv, a->T, a->B, a->vn_sh, a->vn_st, a->vn_sb, 1, 32)) {
+            e = launch_decode_ring(kc, vc, kn, vn, p, di.sms, (cudaStream_t)stream);
+            return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+        }
+    }
     if (decode_tma_ok(a, p)) {
         const int rows = a->kind == SINKATTN_KV_RING ? a->ring_cap
                          : a->kind == SINKATTN_KV_CONTIG ? a->max_ctx
