@@ -40,9 +40,9 @@ struct DecodeTiles {
     bool has_new;    // plus one tile of new tokens
 };
 
-// Tiles of span `split` of sequence b, from its cached length (ring_len or ctx_len) and ring
-// head (0 for other caches).
-SA_DEV DecodeTiles decode_tiles(const DecodeParams &p, int split, int len, int head)
+// Tiles of span `split` of sequence b (kt keys each), from its cached length (ring_len or
+// ctx_len) and ring head (0 for other caches).
+SA_DEV DecodeTiles decode_tiles(const DecodeParams &p, int split, int len, int head, int kt = dt::KT)
 {
     DecodeTiles d;
     d.n_cache = max(0, min(len, p.kind == 0 ? p.ring_cap : p.max_ctx));
@@ -53,10 +53,10 @@ SA_DEV DecodeTiles decode_tiles(const DecodeParams &p, int split, int len, int h
     d.ke = min(d.kb + p.chunk, d.n_total);
     d.ring_head = (p.kind == 0) ? ((head % p.ring_cap) + p.ring_cap) % p.ring_cap : 0;
     if (p.kind == 0) {
-        d.cache_tiles = (d.kb < d.n_used) ? p.ring_cap / dt::KT : 0; // one span holds the ring
+        d.cache_tiles = (d.kb < d.n_used) ? p.ring_cap / kt : 0; // one span holds the ring
     } else {
         const int ce = min(d.ke, d.n_used);
-        d.cache_tiles = (ce > d.kb) ? (ce - d.kb + dt::KT - 1) / dt::KT : 0;
+        d.cache_tiles = (ce > d.kb) ? (ce - d.kb + kt - 1) / kt : 0;
     }
     d.has_new = d.ke > d.n_used && d.kb < d.n_total;
     return d;

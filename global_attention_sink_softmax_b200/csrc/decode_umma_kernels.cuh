@@ -2,36 +2,36 @@
 //
 // Same computation and split-KV partial / merge scheme as the mma.sync decode kernels (sink-free
 // span partials, the sink counted once when spans are merged: "MiMo-V2-Flash 架构 QA" Q3.8).
-// Both contractions are 128-row UMMAs with TMEM accumulators and A operands in TMEM:
-//   S = Q K^T   M 128, N 64 keys (16 for the new tokens), K 16 x 12  (A = Q in TMEM)
-//   O += P V    M 128, N 128 dims, K 16 keys per instruction        (A = P in TMEM, over S)
 // It serves query blocks of 17..64 rows (T new tokens x G heads of one KV group, as in a
 // 4-token draft verify on a 16-head group), where every KV byte feeds 64 FLOP: more than the
-// warp-level mma.sync path sustains at HBM speed.
+// warp-level mma.sync path sustains at HBM speed. Both contractions are 128-row UMMAs with TMEM
+// accumulators, over 128-key steps so each instruction carries as much work as it can:
+//   S = Q K^T   M 128, N 128 keys (16 for the new tokens), K 16 x 12   (A = Q in shared memory)
+//   O += P V    M 128, N 128 dims, K 16 keys x 8                       (A = P in TMEM, over S)
 //
 // Row layout. The R query rows are loaded F = 128 / RP times (RP = 32 or 64 >= R): TMEM lane L
-// holds query row r = L % RP and owns key part jp = L / RP of every 64-key tile (64 / F keys).
+// holds query row r = L % RP and owns key part jp = L / RP of every 128-key step (128 / F keys).
 // Each lane runs its own online softmax over its part (its P is zero on the other parts), so
 // the F lanes of a row are F partial softmaxes over disjoint keys, merged once at the end the
 // way split-KV partials are. All 128 lanes do softmax work and no lane waits for another.
 //
-// Two softmax warpgroups take alternate tiles (warpgroup g the steps j = g, g + 2, ...), each
-// with its own S buffer and O accumulator in TMEM; at the end of an item warpgroup 0 folds
-// warpgroup 1's O into its own (same lanes) and then merges the key parts in shared memory.
+// Pipelines. K and V stream through separate 2-stage rings: a K stage is free as soon as its S
+// MMA has read it, a V stage once P V has. S is double-buffered in TMEM, so S of the next step
+// runs on the tensor cores while the softmax warps work on this one. One thread issues the
+// MMAs from two queues (S and P V) and never lets a ready P V wait behind an S whose keys are
+// still loading.
 //
 // Work items are (span, KV head, sequence), span-major so the longest spans start first; a CTA
 // takes items blockIdx.x, + gridDim.x, ... (one CTA per item, unless the host caps the grid).
 //
-// Roles (352 threads):
-//   warps 0-7  softmax + epilogue (two warpgroups), thread = TMEM lane; warpgroup 0 also writes
-//              each item's Q rows into TMEM;
-//   warp 8     TMA producer of the 64-key cache tiles (5-stage ring, runs ahead across items);
-//   warp 9     TMEM allocator and the single UMMA issuer, which keeps an S queue and a P V
-//              queue and never lets a ready P V wait behind an S whose tile is still loading;
-//   warp 10    TMA producer of each item's new tokens (one 16-row box, rows past T arrive as
-//              zeros).
+// Roles (224 threads):
+//   warps 0-3  softmax + epilogue, thread = TMEM lane;
+//   warp 4     TMA producer of the cache tiles (K and V rings, run ahead across items);
+//   warp 5     TMEM allocator and the UMMA issuer;
+//   warp 6     TMA producer of each item's Q (once per key part) and new tokens (one 16-row box,
+//              rows past T arrive as zeros).
 //
-// Cache tiles: contiguous caches and pages of a multiple of 64 tokens in position order; a
+// Cache tiles: contiguous caches and pages of a multiple of 128 tokens in position order; a
 // ring's slots in physical order (each slot gets its position from the ring head). V rows of
 // keys a tile holds but the span must not see are zeroed in shared memory before P V reads
 // them, so a zero weight never meets whatever the cache held there.
@@ -44,41 +44,41 @@
 namespace sinkattn {
 
 namespace du {
-constexpr int KT = 64;                             // keys per cache tile
-constexpr int REGION = KT * 128;                   // 8 KB: 64 keys x 64 dims, 128B swizzle
-constexpr int STAGE = 5 * REGION;                  // K (3 regions) + V (2 regions): 40 KB
-constexpr int NSTAGE = 5;
+constexpr int KT = 128;                            // keys per cache step
+constexpr int REGION = KT * 128;                   // 16 KB: 128 rows x 64 dims, 128B swizzle
+constexpr int K_STAGE = 3 * REGION;                // 48 KB
+constexpr int V_STAGE = 2 * REGION;                // 32 KB
+constexpr int NK = 2, NV = 2;                      // ring depths
 constexpr int NEW_ROWS = 16;                       // new-token box (T <= 4 rows + zero fill)
 constexpr int NEW_REGION = NEW_ROWS * 128;         // 2 KB
 constexpr int MERGE_COLS = 32;                     // O columns merged per round
 constexpr int MERGE_STRIDE = MERGE_COLS + 4;       // floats per row of the merge buffer
-constexpr int OFF_NEWK = 0;                        // new K: 3 regions
-constexpr int OFF_NEWV = OFF_NEWK + 3 * NEW_REGION; // new V: 2 regions
-// Once every MMA of an item is done (and until the next item's new tokens load) the start of
-// shared memory holds the epilogue's merge data: row statistics [128] (float4), then the key
-// parts' O rows [F - 1][RP][MERGE_STRIDE] floats.
-constexpr int OFF_ML0 = 0;
-constexpr int OFF_OBUF = OFF_ML0 + 128 * 16;
-constexpr int OFF_ML1 = 16 * 1024;                 // warpgroup 1's row statistics [128]
-constexpr int OFF_STAGE = OFF_ML1 + 2 * 1024;      // 18 KB, 1 KB aligned
-constexpr int OFF_BAR = OFF_STAGE + NSTAGE * STAGE;
+constexpr int OFF_Q = 0;                           // 3 regions of 128 MMA rows
+// Once every MMA of an item is done the Q region holds the epilogue's merge data (row
+// statistics [128] float4, then the key parts' O rows [F - 1][RP][MERGE_STRIDE] floats); the
+// next item's Q waits for the merge.
+constexpr int OFF_ML = OFF_Q;
+constexpr int OFF_OBUF = OFF_Q + 128 * 16;
+constexpr int OFF_NEWK = 3 * REGION;               // 48 KB
+constexpr int OFF_NEWV = OFF_NEWK + 3 * NEW_REGION;
+constexpr int OFF_K = OFF_NEWV + 2 * NEW_REGION;   // 58 KB, 1 KB aligned
+constexpr int OFF_V = OFF_K + NK * K_STAGE;
+constexpr int OFF_BAR = OFF_V + NV * V_STAGE;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;   // barriers + 1 KB to align the base
-constexpr int THREADS = 352;
-constexpr int WARP_TILES = 8, WARP_MMA = 9, WARP_ITEM = 10;
+constexpr int THREADS = 224;
+constexpr int WARP_TILES = 4, WARP_MMA = 5, WARP_ITEM = 6;
 constexpr uint32_t TMEM_COLS = 512;
-// TMEM columns: S of warpgroup g at 64 g (P over it); O of warpgroup g at 128 + 128 g; Q (the
-// A operand of S = Q K^T, dims 2c and 2c + 1 in column c) at 384
-constexpr uint32_t TMEM_O = 128;
-constexpr uint32_t TMEM_Q = 384;
+constexpr uint32_t TMEM_O = 256;                   // S buffer b at column 128 b (P over it)
 constexpr float TAU = 8.0f;                        // lazy-rescale threshold (log2 units)
 
 enum Bar {
-    B_NEWFULL = 0,            // an item's new tokens have landed
-    B_QT = 1,                 // an item's Q is in TMEM (warpgroup 0)
-    B_MERGED = 2,             // warpgroup 0 has merged an item: new-token buffers and O_1 free
-    B_FULL = 3,               // + stage
-    B_EMPTY = B_FULL + NSTAGE,
-    B_SFULL = B_EMPTY + NSTAGE, // + warpgroup
+    B_QFULL = 0,              // an item's Q and new tokens have landed
+    B_MERGED = 1,             // the item is merged: Q region (scratch) and new tokens free
+    B_KFULL = 2,              // + K stage
+    B_KEMPTY = B_KFULL + NK,
+    B_VFULL = B_KEMPTY + NK,  // + V stage
+    B_VEMPTY = B_VFULL + NV,
+    B_SFULL = B_VEMPTY + NV,  // + S buffer
     B_PFULL = B_SFULL + 2,
     B_PVDONE = B_PFULL + 2,
     B_DRAIN = B_PVDONE + 2,
@@ -121,7 +121,7 @@ SA_DEV bool du_softmax(const float (&x)[NC], float c_l2, float &m, float &l_roun
     return rescale;
 }
 
-// The keys of step j (index 0..63 in a cache tile, 0..15 among the new tokens) as at most two
+// The keys of step j (index 0..127 in a cache tile, 0..15 among the new tokens) as at most two
 // intervals [a0, a1) u [b0, b1): those present in the span or, with `row`, those query row t may
 // see (cached keys precede every new token; the window may cut the oldest). A ring tile can
 // hold the span's keys in two pieces, where the ring wraps.
@@ -150,7 +150,7 @@ SA_DEV KeySpan du_span(const DecodeParams &p, const DecodeTiles &d, int j, bool 
             s.b0 = s.a0 - p.ring_cap;
             s.b1 = s.a1 - p.ring_cap;
         } else if (tile_ok) {
-            // span index v = kb + 64 j + i in [vlo, min(ke, n_used))
+            // span index v = kb + KT j + i in [vlo, min(ke, n_used))
             const int base = d.kb + j * du::KT;
             const int vlo = win ? max(d.kb, d.n_used + t - p.window + 1) : d.kb;
             s.a0 = vlo - base;
@@ -201,10 +201,23 @@ SA_DEV DuItem du_item(const DecodeParams &p, int it, const DuRaw &raw)
     x.split = it / units;
     x.b = (it % units) / p.Hkv;
     x.g = it % p.Hkv;
-    x.d = decode_tiles(p, x.split, raw.len, raw.head);
+    x.d = decode_tiles(p, x.split, raw.len, raw.head, du::KT);
     x.ct = x.d.cache_tiles;
     x.nsteps = x.ct + (x.d.has_new ? 1 : 0);
     return x;
+}
+
+// Page of the cache tile t of item (b, span d): the page id, or -1 for a page outside the pool
+// (its keys are hidden); contiguous caches and rings have no pages (0).
+SA_DEV int du_page(const DecodeParams &p, const DecodeTiles &d, int b, int t)
+{
+    if (p.kind != 2)
+        return 0;
+    const int pg = (d.first_c + d.kb + t * du::KT) / p.page_size;
+    if (pg >= p.max_pages)
+        return -1;
+    const int pid = p.page_table[(int64_t)b * p.max_pages + pg];
+    return (pid >= 0 && pid < p.num_pages) ? pid : -1;
 }
 
 template <int F>
@@ -217,24 +230,27 @@ __global__ void __launch_bounds__(du::THREADS, 1)
 {
     using namespace du;
     constexpr int RP = 128 / F;  // MMA rows per key part
-    constexpr int KPT = KT / F;  // keys of a cache tile per part
+    constexpr int KPT = KT / F;  // keys of a cache step per part
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + NUM_BARS);
     volatile int *abort = reinterpret_cast<volatile int *>(tmem_slot + 1);
-    volatile int *go_on = reinterpret_cast<volatile int *>(tmem_slot + 2); // [2], per item parity
+    volatile int *go_on = reinterpret_cast<volatile int *>(tmem_slot + 2);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = p.splits * p.Hkv * p.B;
 
     if (threadIdx.x == 0) {
-        mbar_init(&bars[B_NEWFULL], 1);
-        mbar_init(&bars[B_QT], 128);
+        mbar_init(&bars[B_QFULL], 1);
         mbar_init(&bars[B_MERGED], 128);
-        for (int i = 0; i < NSTAGE; ++i) {
-            mbar_init(&bars[B_FULL + i], 1);
-            mbar_init(&bars[B_EMPTY + i], 1);
+        for (int i = 0; i < NK; ++i) {
+            mbar_init(&bars[B_KFULL + i], 1);
+            mbar_init(&bars[B_KEMPTY + i], 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            mbar_init(&bars[B_VFULL + i], 1);
+            mbar_init(&bars[B_VEMPTY + i], 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bars[B_SFULL + i], 1);
@@ -243,7 +259,7 @@ __global__ void __launch_bounds__(du::THREADS, 1)
         }
         mbar_init(&bars[B_DRAIN], 1);
         *abort = 0;
-        go_on[0] = go_on[1] = 1;
+        *go_on = 1;
         fence_mbar_init();
     }
     if (warp == WARP_MMA) {
@@ -256,88 +272,103 @@ __global__ void __launch_bounds__(du::THREADS, 1)
     const uint32_t tmem = *tmem_slot;
 
     if (warp == WARP_TILES) {
-        // ---------------- cache tiles: one 3-stage ring across all items ----------------
+        // ---------------- cache tiles: K and V rings across all items ----------------
         if (lane == 0) {
             tma_prefetch_desc(&tmKc);
             tma_prefetch_desc(&tmVc);
-            int tt = 0; // tiles issued
+            int tt = 0;       // tiles issued
+            int k_issued = 0; // tiles whose K copy was issued (one more than tt if a V wait failed)
             bool ok = true;
             DuRaw raw = du_raw(p, blockIdx.x, n_items);
             for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
                 const DuItem x = du_item(p, it, raw);
                 raw = du_raw(p, it + gridDim.x, n_items);
                 for (int t = 0; t < x.ct; ++t, ++tt) {
-                    const int st = tt % NSTAGE;
-                    if (tt >= NSTAGE && !mbar_wait(&bars[B_EMPTY + st], ((tt / NSTAGE) - 1) & 1, abort, 2u)) {
-                        ok = false;
-                        break;
-                    }
-                    uint8_t *sk = smem + OFF_STAGE + st * STAGE;
-                    mbar_arrive_expect_tx(&bars[B_FULL + st], STAGE);
                     int row, blk = x.b;
                     if (p.kind == 0) { // ring: slots in physical order
                         row = t * KT;
                     } else {
                         row = x.d.first_c + x.d.kb + t * KT; // first cached token of the tile
                         if (p.kind == 2) {
-                            const int pg = row / p.page_size;
                             // a missing page is read at a block outside the pool (zeros); the
                             // softmax warps mask its keys
-                            blk = decode_tile_ok(p, x.d, x.b, t)
-                                      ? p.page_table[(int64_t)x.b * p.max_pages + pg]
-                                      : p.num_pages;
-                            row -= pg * p.page_size;
+                            const int pid = du_page(p, x.d, x.b, t);
+                            blk = pid >= 0 ? pid : p.num_pages;
+                            row -= (row / p.page_size) * p.page_size;
                         }
                     }
+                    const int ks = tt % NK, vs = tt % NV;
+                    if (tt >= NK && !mbar_wait(&bars[B_KEMPTY + ks], ((tt / NK) - 1) & 1, abort, 2u)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sk = smem + OFF_K + ks * K_STAGE;
+                    mbar_arrive_expect_tx(&bars[B_KFULL + ks], K_STAGE);
                     for (int c = 0; c < 3; ++c)
-                        tma_load_4d(sk + c * REGION, &tmKc, &bars[B_FULL + st], c * 64, x.g, row, blk);
+                        tma_load_4d(sk + c * REGION, &tmKc, &bars[B_KFULL + ks], c * 64, x.g, row, blk);
+                    k_issued = tt + 1;
+                    if (tt >= NV && !mbar_wait(&bars[B_VEMPTY + vs], ((tt / NV) - 1) & 1, abort, 2u)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sv = smem + OFF_V + vs * V_STAGE;
+                    mbar_arrive_expect_tx(&bars[B_VFULL + vs], V_STAGE);
                     for (int c = 0; c < 2; ++c)
-                        tma_load_4d(sk + (3 + c) * REGION, &tmVc, &bars[B_FULL + st], c * 64, x.g, row, blk);
+                        tma_load_4d(sv + c * REGION, &tmVc, &bars[B_VFULL + vs], c * 64, x.g, row, blk);
                 }
             }
             // no copy of ours may still be landing when the CTA leaves
-            for (int t = max(0, tt - NSTAGE); t < tt; ++t)
-                mbar_wait_drain(&bars[B_FULL + t % NSTAGE], (t / NSTAGE) & 1);
+            for (int t = max(0, k_issued - NK); t < k_issued; ++t)
+                mbar_wait_drain(&bars[B_KFULL + t % NK], (t / NK) & 1);
+            for (int t = max(0, tt - NV); t < tt; ++t)
+                mbar_wait_drain(&bars[B_VFULL + t % NV], (t / NV) & 1);
         }
         __syncwarp();
     } else if (warp == WARP_ITEM) {
-        // ---------------- the new tokens of each item ----------------
+        // ---------------- Q and the new tokens of each item ----------------
         if (lane == 0) {
-            int n = 0; // non-empty items
+            tma_prefetch_desc(&tmQ);
+            const uint32_t qbytes = (uint32_t)(F * 3 * p.R * 128);
+            int n = 0; // non-empty items loaded
             DuRaw raw = du_raw(p, blockIdx.x, n_items);
             for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
                 const DuItem x = du_item(p, it, raw);
                 raw = du_raw(p, it + gridDim.x, n_items);
                 if (x.nsteps == 0)
                     continue;
-                // the new-token buffers double as the previous item's merge scratch
+                // the Q region doubles as the previous item's merge scratch
                 if (n >= 1 && !mbar_wait(&bars[B_MERGED], (n - 1) & 1, abort, 2u))
                     break;
-                mbar_arrive_expect_tx(&bars[B_NEWFULL], x.d.has_new ? 5u * NEW_REGION : 0u);
+                mbar_arrive_expect_tx(&bars[B_QFULL], qbytes + (x.d.has_new ? 5u * NEW_REGION : 0u));
+                // rows (t, h) of the group: box {64 dims, G heads, T tokens}, row r = t G + h,
+                // once per key part at MMA row jp * RP
+                for (int jp = 0; jp < F; ++jp)
+                    for (int c = 0; c < 3; ++c)
+                        tma_load_4d(smem + OFF_Q + c * REGION + jp * RP * 128, &tmQ, &bars[B_QFULL],
+                                    c * 64, x.g * p.G, 0, x.b);
                 if (x.d.has_new) {
                     for (int c = 0; c < 3; ++c)
-                        tma_load_4d(smem + OFF_NEWK + c * NEW_REGION, &tmKn, &bars[B_NEWFULL], c * 64,
+                        tma_load_4d(smem + OFF_NEWK + c * NEW_REGION, &tmKn, &bars[B_QFULL], c * 64,
                                     x.g, 0, x.b);
                     for (int c = 0; c < 2; ++c)
-                        tma_load_4d(smem + OFF_NEWV + c * NEW_REGION, &tmVn, &bars[B_NEWFULL], c * 64,
+                        tma_load_4d(smem + OFF_NEWV + c * NEW_REGION, &tmVn, &bars[B_QFULL], c * 64,
                                     x.g, 0, x.b);
                 }
                 ++n;
             }
             if (n > 0)
-                mbar_wait_drain(&bars[B_NEWFULL], (n - 1) & 1);
+                mbar_wait_drain(&bars[B_QFULL], (n - 1) & 1);
         }
         __syncwarp();
     } else if (warp == WARP_MMA) {
         // ---------------- UMMA issuer ----------------
-        // Step j of an item belongs to warpgroup g = j & 1 and is its k-th step overall.
         if (lane == 0) {
             const uint32_t idesc_s = umma_idesc_bf16(128, KT, 0);
             const uint32_t idesc_n = umma_idesc_bf16(128, NEW_ROWS, 0);
             const uint32_t idesc_o = umma_idesc_bf16(128, 128, 1);
+            const uint64_t qd = smem_desc_sw128(smem_u32(smem + OFF_Q), 16, 1024);
             const uint32_t sKn = smem_u32(smem + OFF_NEWK);
-            int n = 0, tt = 0;     // items and cache tiles before this item
-            int cg0 = 0, cg1 = 0;  // steps of each warpgroup before this item
+            int n = 0, tt = 0, J = 0; // items, cache tiles and steps before this item
             bool ok = true;
             DuRaw raw = du_raw(p, blockIdx.x, n_items);
             for (int it = blockIdx.x; ok && it < n_items; it += gridDim.x) {
@@ -345,61 +376,63 @@ __global__ void __launch_bounds__(du::THREADS, 1)
                 raw = du_raw(p, it + gridDim.x, n_items);
                 if (x.nsteps == 0)
                     continue;
-                if (!mbar_wait(&bars[B_QT], n & 1, abort, 2u) ||
-                    !mbar_wait(&bars[B_NEWFULL], n & 1, abort, 2u))
+                if (!mbar_wait(&bars[B_QFULL], n & 1, abort, 2u))
                     break;
-                // One thread issues both queues in order (S_0, S_1, ...; PV_0, PV_1, ...) and
-                // never blocks one behind the other: a P V whose P is ready goes first (it frees
-                // a stage), an S goes as soon as its tile has landed and its warpgroup's S
-                // buffer has been read by the previous P V.
+                // Step j (global jg = J + j) uses S buffer jg & 1. S needs its keys landed and
+                // the buffer read by the P V two steps back; P V needs P and its V landed.
                 auto s_ready = [&](int j) -> bool {
-                    const int g = j & 1, k = (g ? cg1 : cg0) + (j >> 1);
-                    if (k >= 1 && !mbar_test(&bars[B_PVDONE + g], (k - 1) & 1))
+                    const int jg = J + j;
+                    if (jg >= 2 && !mbar_test(&bars[B_PVDONE + (jg & 1)], ((jg - 2) >> 1) & 1))
                         return false;
                     const int tg = tt + j;
-                    return j >= x.ct || mbar_test(&bars[B_FULL + tg % NSTAGE], (tg / NSTAGE) & 1);
+                    return j >= x.ct || mbar_test(&bars[B_KFULL + tg % NK], (tg / NK) & 1);
                 };
                 auto issue_s = [&](int j) {
-                    const int g = j & 1;
+                    const int jg = J + j;
                     uint32_t kb_addr = sKn, kreg = NEW_REGION, idesc = idesc_n;
                     if (j < x.ct) {
-                        kb_addr = smem_u32(smem + OFF_STAGE + ((tt + j) % NSTAGE) * STAGE);
+                        kb_addr = smem_u32(smem + OFF_K + ((tt + j) % NK) * K_STAGE);
                         kreg = REGION;
                         idesc = idesc_s;
                     }
-                    // B descriptors of the later k-steps: the start-address field (16-byte
-                    // units, shared memory < 256 KB) advanced by the step's byte offset
+                    // descriptors advanced by the k-step's byte offset (the start-address field
+                    // counts 16-byte units; shared memory < 256 KB)
                     const uint64_t kd = smem_desc_sw128(kb_addr, 16, 1024);
 #pragma unroll
-                    for (int kk = 0; kk < 12; ++kk)
-                        umma_ts(tmem + g * 64, tmem + TMEM_Q + kk * 8,
-                                kd + (((kk >> 2) * kreg + (kk & 3) * 32) >> 4), idesc, kk > 0 ? 1u : 0u);
-                    umma_commit(&bars[B_SFULL + g]);
+                    for (int kk = 0; kk < 12; ++kk) {
+                        const uint32_t koff = (kk & 3) * 32;
+                        umma_ss(tmem + (jg & 1) * 128, qd + (((kk >> 2) * REGION + koff) >> 4),
+                                kd + (((kk >> 2) * kreg + koff) >> 4), idesc, kk > 0);
+                    }
+                    umma_commit(&bars[B_SFULL + (jg & 1)]);
+                    if (j < x.ct)
+                        umma_commit(&bars[B_KEMPTY + (tt + j) % NK]); // K stage read
                 };
                 auto pv_ready = [&](int j) -> bool {
-                    const int g = j & 1, k = (g ? cg1 : cg0) + (j >> 1);
-                    return mbar_test(&bars[B_PFULL + g], k & 1);
+                    const int jg = J + j;
+                    if (!mbar_test(&bars[B_PFULL + (jg & 1)], (jg >> 1) & 1))
+                        return false;
+                    const int tg = tt + j;
+                    return j >= x.ct || mbar_test(&bars[B_VFULL + tg % NV], (tg / NV) & 1);
                 };
                 auto issue_pv = [&](int j) {
-                    const int g = j & 1;
-                    const uint32_t pt = tmem + g * 64;            // P: 16 keys per 8 columns
-                    const uint32_t od = tmem + TMEM_O + g * 128;  // this warpgroup's O
+                    const int jg = J + j;
+                    const uint32_t pt = tmem + (jg & 1) * 128; // P: 16 keys per 8 columns
                     if (j < x.ct) {
                         // B = V (16 keys x 128 dims, dims contiguous: MN-major; dims 64..127 one
                         // region further on)
-                        const int st = (tt + j) % NSTAGE;
-                        const uint64_t vd = smem_desc_sw128(
-                            smem_u32(smem + OFF_STAGE + st * STAGE + 3 * REGION), REGION, 1024);
+                        const int vs = (tt + j) % NV;
+                        const uint64_t vd = smem_desc_sw128(smem_u32(smem + OFF_V + vs * V_STAGE), REGION, 1024);
 #pragma unroll
                         for (int kk = 0; kk < KT / 16; ++kk)
-                            umma_ts(od, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_o,
-                                    (j >= 2 || kk > 0) ? 1u : 0u);
-                        umma_commit(&bars[B_PVDONE + g]);
-                        umma_commit(&bars[B_EMPTY + st]);
+                            umma_ts(tmem + TMEM_O, pt + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_o,
+                                    (j > 0 || kk > 0) ? 1u : 0u);
+                        umma_commit(&bars[B_PVDONE + (jg & 1)]);
+                        umma_commit(&bars[B_VEMPTY + vs]);
                     } else {
-                        umma_ts(od, pt, smem_desc_sw128(smem_u32(smem + OFF_NEWV), NEW_REGION, 1024),
-                                idesc_o, j >= 2 ? 1u : 0u);
-                        umma_commit(&bars[B_PVDONE + g]);
+                        umma_ts(tmem + TMEM_O, pt, smem_desc_sw128(smem_u32(smem + OFF_NEWV), NEW_REGION, 1024),
+                                idesc_o, j > 0 ? 1u : 0u);
+                        umma_commit(&bars[B_PVDONE + (jg & 1)]);
                     }
                 };
                 int ns = 0, np = 0; // S and P V issued
@@ -409,7 +442,7 @@ __global__ void __launch_bounds__(du::THREADS, 1)
                         tc_fence_after();
                         issue_pv(np++);
                         idle_since = 0;
-                    } else if (ns < x.nsteps && s_ready(ns)) {
+                    } else if (ns < x.nsteps && ns < np + 2 && s_ready(ns)) {
                         tc_fence_after();
                         issue_s(ns++);
                         idle_since = 0;
@@ -429,8 +462,7 @@ __global__ void __launch_bounds__(du::THREADS, 1)
                         }
                     }
                 }
-                cg0 += (x.nsteps + 1) >> 1;
-                cg1 += x.nsteps >> 1;
+                J += x.nsteps;
                 tt += x.ct;
                 ++n;
             }
@@ -440,20 +472,16 @@ __global__ void __launch_bounds__(du::THREADS, 1)
         }
         __syncwarp();
     } else {
-        // ---------- softmax warpgroups: thread = TMEM lane = (key part, query row) ----------
-        // Warpgroup grp takes the steps j = grp, grp + 2, ... of every item into its own O.
-        const int grp = warp >> 2;
-        const int L = (warp & 3) * 32 + lane;
+        // ---------- softmax warps: thread = TMEM lane = (key part, query row) ----------
+        const int L = threadIdx.x;
         const int jp = L / RP, r = L % RP; // jp is warp-uniform (RP >= 32)
         const bool row_ok = r < p.R;
         const int t = row_ok ? r / p.G : 0;
-        const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t o_addr = tmem + lane_addr + TMEM_O + grp * 128;
+        const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
         const float c_l2 = p.scale_log2;
-        float4 *ml0 = reinterpret_cast<float4 *>(smem + OFF_ML0);  // [128], after the MMAs
-        float4 *ml1 = reinterpret_cast<float4 *>(smem + OFF_ML1);  // [128]
-        float *obuf = reinterpret_cast<float *>(smem + OFF_OBUF);  // [F-1][RP][..], after the MMAs
-        int n = 0, tt = 0, cg = 0;
+        float4 *ml = reinterpret_cast<float4 *>(smem + OFF_ML);     // [128], after the MMAs
+        float *obuf = reinterpret_cast<float *>(smem + OFF_OBUF);   // [F-1][RP][..], after the MMAs
+        int n = 0, tt = 0, J = 0;
         DuRaw raw = du_raw(p, blockIdx.x, n_items);
         for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
             const DuItem x = du_item(p, it, raw);
@@ -461,76 +489,57 @@ __global__ void __launch_bounds__(du::THREADS, 1)
             const int64_t unit = ((int64_t)x.b * p.Hkv + x.g) * p.splits + x.split;
             if (x.nsteps == 0) {
                 // an empty span: its partial has no keys (the merge skips l = 0)
-                if (grp == 0 && L < p.R && p.splits > 1)
+                if (L < p.R && p.splits > 1)
                     *reinterpret_cast<float4 *>(p.ws_ml + (unit * p.R + L) * 4) =
                         make_float4(-INFINITY, 0.f, 0.f, 0.f);
                 continue;
             }
             const DecodeTiles &d = x.d;
             const int h = x.g * p.G + (row_ok ? r % p.G : 0);
-            if (grp == 0) {
-                // this lane's query row into TMEM (the A operand of S; rows past R are zero).
-                // The previous item's MMAs are all done: its merge came after them.
-                const uint4 *qrow = reinterpret_cast<const uint4 *>(
-                    p.q + (int64_t)x.b * p.q_sb + (int64_t)t * p.q_st + (int64_t)h * p.q_sh);
-#pragma unroll 1
-                for (int c = 0; c < 3; ++c) {
-                    uint32_t v[32];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const uint4 w = row_ok ? __ldg(qrow + c * 8 + u) : make_uint4(0u, 0u, 0u, 0u);
-                        v[4 * u] = w.x;
-                        v[4 * u + 1] = w.y;
-                        v[4 * u + 2] = w.z;
-                        v[4 * u + 3] = w.w;
-                    }
-                    tmem_st32(tmem + lane_addr + TMEM_Q + c * 32, v);
-                }
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&bars[B_QT]);
-            }
-            const float sink_h = (grp == 0 && p.sink) ? p.sink[h] : -INFINITY; // used at the end
+            const float sink_h = p.sink ? p.sink[h] : -INFINITY; // used at the end of the item
             float m = -INFINITY, l_round = 0.f, l_exact = 0.f;
             bool ok = true;
-            int k = cg;
-            for (int j = grp; j < x.nsteps; j += 2, ++k) {
+            for (int j = 0; j < x.nsteps; ++j) {
+                const int jg = J + j, sb = jg & 1;
                 // Cache tiles and the new tokens take the same path: the new tokens are keys
                 // 0..T-1 of an N = 16 step, which all fall in key part 0 (the other parts'
                 // columns hold stale values and are masked).
                 const bool cache = j < x.ct;
-                // a paged tile's page id, loaded before the wait so its latency hides there
-                const int pg = cache && p.kind == 2 ? (d.first_c + d.kb + j * KT) / p.page_size : 0;
-                const int pid = cache && p.kind == 2 && pg < p.max_pages
-                                    ? __ldg(p.page_table + (int64_t)x.b * p.max_pages + pg)
-                                    : -1;
-                ok = warp_wait(&bars[B_SFULL + grp], k & 1, abort);
+                // a paged tile's page, looked up before the wait so the load's latency hides
+                const int pid = cache ? du_page(p, d, x.b, j) : 0;
+                ok = warp_wait(&bars[B_SFULL + sb], (jg >> 1) & 1, abort);
                 if (!ok)
                     break;
                 tc_fence_after();
-                const uint32_t saddr = tmem + lane_addr + grp * 64;
-                const bool tile_ok = !cache || p.kind != 2 || (pid >= 0 && pid < p.num_pages);
+                const uint32_t saddr = tmem + lane_addr + sb * 128;
+                const bool tile_ok = pid >= 0;
                 if (cache) {
                     const KeySpan present = du_span(p, d, j, tile_ok, false, 0);
                     if (!present.covers(KT)) {
-                        // zero the V rows of keys outside the span: lane L takes key L % 64,
-                        // half L / 64
-                        if (!present.has(L & 63)) {
-                            uint4 *row = reinterpret_cast<uint4 *>(
-                                smem + OFF_STAGE + ((tt + j) % NSTAGE) * STAGE +
-                                (3 + (L >> 6)) * REGION + (L & 63) * 128);
+                        // zero the V rows of keys outside the span: lane L takes key L, both
+                        // halves, once the tile's V has landed
+                        const int tg = tt + j;
+                        ok = warp_wait(&bars[B_VFULL + tg % NV], (tg / NV) & 1, abort);
+                        if (!ok)
+                            break;
+                        if (!present.has(L)) {
+                            uint8_t *vrow = smem + OFF_V + (tg % NV) * V_STAGE + L * 128;
 #pragma unroll
-                            for (int u = 0; u < 8; ++u)
-                                row[u] = make_uint4(0u, 0u, 0u, 0u);
+                            for (int u = 0; u < 8; ++u) {
+                                *reinterpret_cast<uint4 *>(vrow + u * 16) = make_uint4(0u, 0u, 0u, 0u);
+                                *reinterpret_cast<uint4 *>(vrow + REGION + u * 16) = make_uint4(0u, 0u, 0u, 0u);
+                            }
                         }
                         fence_async_smem();
                     }
                 }
                 uint32_t raw_s[KPT];
-                if constexpr (KPT == 32) {
-                    tmem_ld32_sync(saddr + jp * KPT, raw_s);
+                if constexpr (KPT == 64) {
+                    tmem_ld32(saddr + jp * KPT, *reinterpret_cast<uint32_t(*)[32]>(&raw_s[0]));
+                    tmem_ld32(saddr + jp * KPT + 32, *reinterpret_cast<uint32_t(*)[32]>(&raw_s[32]));
+                    tmem_ld_wait();
                 } else {
-                    tmem_ld16_sync(saddr + jp * KPT, raw_s);
+                    tmem_ld32_sync(saddr + jp * KPT, *reinterpret_cast<uint32_t(*)[32]>(&raw_s[0]));
                 }
                 const KeySpan vis = row_ok ? du_span(p, d, j, tile_ok, true, t) : KeySpan{0, 0, 0, 0};
                 float xs[KPT];
@@ -555,76 +564,53 @@ __global__ void __launch_bounds__(du::THREADS, 1)
                 for (int q8 = 0; q8 < KT / 16; ++q8)
                     if (q8 / (KPT / 16) != jp)
                         tmem_st8(saddr + q8 * 8, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u);
-                // O holds this warpgroup's P V of the item up to its previous step: rescale it
-                // to the new reference max (its first step's P V overwrites O)
-                if (j >= 2 && __any_sync(0xffffffffu, rescale)) {
-                    ok = warp_wait(&bars[B_PVDONE + grp], (k - 1) & 1, abort);
+                // O holds P V up to step j - 1: rescale it to the new reference max (the first
+                // step's P V overwrites O)
+                if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+                    ok = warp_wait(&bars[B_PVDONE + ((jg - 1) & 1)], ((jg - 1) >> 1) & 1, abort);
                     if (!ok)
                         break;
                     tc_fence_after();
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
-                        tmem_ld32_sync(o_addr + c * 32, o);
+                        tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * 32, o);
 #pragma unroll
                         for (int e = 0; e < 32; ++e)
                             o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(o_addr + c * 32, o);
+                        tmem_st32(tmem + lane_addr + TMEM_O + c * 32, o);
                     }
                 }
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&bars[B_PFULL + grp]);
+                mbar_arrive(&bars[B_PFULL + sb]);
             }
-            if (ok && k > cg) {
-                const int kl = k - 1;
-                ok = warp_wait(&bars[B_PVDONE + grp], kl & 1, abort);
-            }
+            const int jl = J + x.nsteps - 1;
+            if (ok)
+                ok = warp_wait(&bars[B_PVDONE + (jl & 1)], (jl >> 1) & 1, abort);
             tc_fence_after();
-            cg = k;
+            J += x.nsteps;
             tt += x.ct;
 
-            // ---- warpgroup 1 hands its row statistics to warpgroup 0; one decision to go on
-            if (grp == 1) {
-                ml1[L] = make_float4(m, l_round, l_exact, ok ? 1.f : 0.f);
-                if (L == 0)
-                    go_on[n & 1] = !*abort;
-            }
-            named_bar_sync(2, 256);
-            const bool cont = go_on[n & 1] != 0;
-            if (grp == 1) {
-                ++n;
-                if (!cont)
-                    break;
-                continue;
-            }
-
-            // ---- warpgroup 0: combine the two warpgroups (same lanes), then the F key parts
-            const float4 s1 = ml1[L];
-            const bool has1 = x.nsteps >= 2;
-            ok = ok && s1.w != 0.f;
-            const float m01 = fmaxf(m, has1 ? s1.x : -INFINITY);
-            const float a0 = (m == -INFINITY) ? 0.f : fast_exp2(m - m01);
-            const float a1 = (!has1 || s1.x == -INFINITY) ? 0.f : fast_exp2(s1.x - m01);
-            const float lr01 = l_round * a0 + (has1 ? s1.y * a1 : 0.f);
-            const float le01 = l_exact * a0 + (has1 ? s1.z * a1 : 0.f);
-            ml0[L] = make_float4(m01, lr01, le01, 0.f);
+            // ---- merge the F key parts of each row (all MMAs of the item are done: the Q
+            // region is scratch); every softmax thread takes every barrier
+            ml[L] = make_float4(m, l_round, l_exact, 0.f);
+            if (L == 0)
+                *go_on = !*abort; // one decision for the four warps, read after the barriers
             named_bar_sync(1, 128);
             float mf = -INFINITY;
 #pragma unroll
             for (int jj = 0; jj < F; ++jj)
-                mf = fmaxf(mf, ml0[jj * RP + r].x);
+                mf = fmaxf(mf, ml[jj * RP + r].x);
             float lr = 0.f, le = 0.f;
 #pragma unroll
             for (int jj = 0; jj < F; ++jj) {
-                const float4 ml = ml0[jj * RP + r];
-                const float c = (ml.x == -INFINITY) ? 0.f : fast_exp2(ml.x - mf);
-                lr += ml.y * c;
-                le += ml.z * c;
+                const float4 v4 = ml[jj * RP + r];
+                const float c = (v4.x == -INFINITY) ? 0.f : fast_exp2(v4.x - mf);
+                lr += v4.y * c;
+                le += v4.z * c;
             }
-            // this lane's O = a0 O_0 + a1 O_1, brought to the row's reference max mf
-            const float sc = (m01 == -INFINITY) ? 0.f : fast_exp2(m01 - mf);
-            const float b0 = a0 * sc, b1 = a1 * sc;
+            const float a_self = (m == -INFINITY) ? 0.f : fast_exp2(m - mf);
             const bool writer = jp == 0 && row_ok;
             // final scaling (single span: the sink applied once) or the span's partial
             float scl = 1.f, lse = 0.f;
@@ -638,26 +624,27 @@ __global__ void __launch_bounds__(du::THREADS, 1)
             }
             uint16_t *orow = p.o + (int64_t)x.b * p.o_sb + (int64_t)t * p.o_st + (int64_t)h * p.o_sh;
             float *wrow = p.ws_o ? p.ws_o + (unit * p.R + r) * 128 : nullptr;
+            const bool cont = *go_on != 0;
             const bool write = writer && ok && cont;
 #pragma unroll 1
             for (int c = 0; c < 128 / MERGE_COLS; ++c) {
-                uint32_t o[MERGE_COLS], o1[MERGE_COLS];
-                tmem_ld32(tmem + lane_addr + TMEM_O + c * MERGE_COLS, o);
-                if (has1)
-                    tmem_ld32(tmem + lane_addr + TMEM_O + 128 + c * MERGE_COLS, o1);
-                tmem_ld_wait();
-                float v[MERGE_COLS];
-#pragma unroll
-                for (int e = 0; e < MERGE_COLS; ++e)
-                    v[e] = __uint_as_float(o[e]) * b0 + (has1 ? __uint_as_float(o1[e]) * b1 : 0.f);
+                uint32_t o[MERGE_COLS];
+                tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * MERGE_COLS, o);
                 if (jp > 0) {
                     float4 *dst = reinterpret_cast<float4 *>(obuf + ((jp - 1) * RP + r) * MERGE_STRIDE);
 #pragma unroll
                     for (int q = 0; q < MERGE_COLS / 4; ++q)
-                        dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+                        dst[q] = make_float4(__uint_as_float(o[4 * q]) * a_self,
+                                             __uint_as_float(o[4 * q + 1]) * a_self,
+                                             __uint_as_float(o[4 * q + 2]) * a_self,
+                                             __uint_as_float(o[4 * q + 3]) * a_self);
                 }
                 named_bar_sync(1, 128);
                 if (write) {
+                    float v[MERGE_COLS];
+#pragma unroll
+                    for (int e = 0; e < MERGE_COLS; ++e)
+                        v[e] = __uint_as_float(o[e]) * a_self;
 #pragma unroll
                     for (int jj = 1; jj < F; ++jj) {
                         const float4 *src = reinterpret_cast<const float4 *>(
@@ -691,8 +678,7 @@ __global__ void __launch_bounds__(du::THREADS, 1)
                 }
                 named_bar_sync(1, 128);
             }
-            // warpgroup 1's O is read and the merge scratch is dead: the next item may load
-            // its new tokens and overwrite O_1
+            // O and the merge scratch are free: the next item may load its Q and new tokens
             tc_fence_before();
             mbar_arrive(&bars[B_MERGED]);
             if (write) {

@@ -248,7 +248,7 @@ Split plan_split(const sinkattn_decode_args *a)
     if (splits < 1)
         splits = 1;
     int64_t chunk = (n + splits - 1) / splits;
-    chunk = (chunk + 63) / 64 * 64;
+    chunk = (chunk + 127) / 128 * 128; // whole tiles of every decode kernel (64 or 128 keys)
     splits = (n + chunk - 1) / chunk;
     return Split{(int)splits, (int)chunk};
 }
@@ -468,14 +468,17 @@ int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *strea
                          : a->kind == SINKATTN_KV_CONTIG ? a->max_ctx
                                                          : a->page_size;
         const int blocks = a->kind == SINKATTN_KV_PAGED ? a->num_pages : a->B;
-        // tcgen05 kernel: blocks of more than 16 query rows; the mma.sync TMA kernel: up to 16
-        const bool umma = p.R > 16 || a->kind == SINKATTN_KV_RING;
+        // tcgen05 kernel: blocks of more than 16 query rows over 128-key tiles (pages of a
+        // multiple of 128 tokens); the mma.sync TMA kernel: the rest, over 64-key tiles
+        const bool umma = (p.R > 16 && (a->kind != SINKATTN_KV_PAGED || a->page_size % 128 == 0)) ||
+                          a->kind == SINKATTN_KV_RING;
         const int new_rows = umma ? 16 : 64;
+        const int box = umma ? 128 : 64;
         CUtensorMap kc, vc, kn, vn, q;
         // a cache the tensor-map encoder rejects (e.g. an empty one) takes the cp.async kernel
         if (rows > 0 &&
-            !make_map(&kc, a->k_cache, kDQ, a->Hkv, rows, blocks, a->kc_sh, a->kc_ss, a->kc_sb, 1, 64) &&
-            !make_map(&vc, a->v_cache, kDV, a->Hkv, rows, blocks, a->vc_sh, a->vc_ss, a->vc_sb, 1, 64) &&
+            !make_map(&kc, a->k_cache, kDQ, a->Hkv, rows, blocks, a->kc_sh, a->kc_ss, a->kc_sb, 1, box) &&
+            !make_map(&vc, a->v_cache, kDV, a->Hkv, rows, blocks, a->vc_sh, a->vc_ss, a->vc_sb, 1, box) &&
             !make_map(&kn, a->k_new, kDQ, a->Hkv, a->T, a->B, a->kn_sh, a->kn_st, a->kn_sb, 1, new_rows) &&
             !make_map(&vn, a->v_new, kDV, a->Hkv, a->T, a->B, a->vn_sh, a->vn_st, a->vn_sb, 1, new_rows)) {
             if (!umma) {

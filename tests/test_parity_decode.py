@@ -106,7 +106,7 @@ def test_contig_decode_sink_none_and_window():
     check(sa.KV_CONTIG, d, 5, "contig with a 5 window")
 
 
-@pytest.mark.parametrize("P", [128, 16])
+@pytest.mark.parametrize("P", [128, 64, 16])
 @pytest.mark.parametrize("T", [1, 4])
 def test_paged_decode(P, T):
     g = torch.Generator().manual_seed(P + T)
