@@ -163,7 +163,7 @@ class DecodeRunner:
         # the kernel the library dispatches this workload to
         rows = w.T * (w.Hq // w.Hkv)
         if w.kind == W.KV_RING:
-            self.kernel = "decode_ring_kernel"
+            self.kernel = "decode_ring_kernel" if rows <= 16 else "decode_split_kernel"
         elif w.kind == W.KV_PAGED and w.page_size % 64 != 0:
             self.kernel = "decode_split_kernel"
         else:

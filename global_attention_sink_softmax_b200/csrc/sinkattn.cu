@@ -448,8 +448,9 @@ bool decode_tma_ok(const sinkattn_decode_args *a, const DecodeParams &)
 int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *stream)
 {
     cudaError_t e;
-    if (a->kind == SINKATTN_KV_RING && a->ring_cap % 32 == 0 && p.splits == 1) {
-        // a ring item (an m16 tile of a unit's rows) per warp, streamed in 32-key chunks
+    if (a->kind == SINKATTN_KV_RING && p.R <= 16 && a->ring_cap % 32 == 0 && p.splits == 1) {
+        // a ring item per warp, streamed in 32-key chunks (units of more than 16 rows, as in a
+        // 4-token verify, measured faster on the cp.async kernel, whose CTA serves all rows)
         CUtensorMap kc, vc, kn, vn;
         DeviceInfo di;
         int st = device_info(&di);
