@@ -80,6 +80,21 @@ def test_ring_decode(T, Hq, Hkv):
     check(sa.KV_RING, d, 128, f"ring T{T} {Hq}/{Hkv}")
 
 
+@pytest.mark.parametrize("cap,window", [(32, 128), (96, 64), (256, 128), (256, 0)])
+@pytest.mark.parametrize("T", [1, 3])
+def test_ring_decode_other_capacities(cap, window, T):
+    """Rings of other sizes (the one-warp-per-item ring kernel takes any multiple of 32 slots),
+    a window shorter than the ring, and a ring without a window."""
+    g = torch.Generator().manual_seed(cap + 7 * T + window)
+    B, Hq, Hkv = 5, 16, 2
+    d = dict(q=rnd((B, T, Hq, 192), g), k_new=rnd((B, T, Hkv, 192), g),
+             v_new=rnd((B, T, Hkv, 128), g), k_cache=rnd((B, cap, Hkv, 192), g),
+             v_cache=rnd((B, cap, Hkv, 128), g), sink=make_sink(Hq, g, "mixed"),
+             ring_head=torch.tensor([0, 1, cap - 1, cap // 2, 3], dtype=torch.int32),
+             ring_len=torch.tensor([cap, cap - 1, 1, 0, cap // 3], dtype=torch.int32))
+    check(sa.KV_RING, d, window, f"ring cap {cap} W{window} T{T}")
+
+
 @pytest.mark.parametrize("T", [1, 4])
 @pytest.mark.parametrize("ctx", [[0, 1, 63, 64], [65, 127, 128, 129], [1000, 5000, 3, 4093]])
 def test_contig_decode(T, ctx):
@@ -106,7 +121,7 @@ def test_contig_decode_sink_none_and_window():
     check(sa.KV_CONTIG, d, 5, "contig with a 5 window")
 
 
-@pytest.mark.parametrize("P", [128, 64, 16])
+@pytest.mark.parametrize("P", [256, 192, 128, 64, 16])
 @pytest.mark.parametrize("T", [1, 4])
 def test_paged_decode(P, T):
     g = torch.Generator().manual_seed(P + T)
