@@ -53,9 +53,12 @@ def visible_pairs_prefill(L: int, window: int) -> int:
 def prefill_counts(w, L=None, B=None):
     L = w.L if L is None else L
     B = w.B if B is None else B
-    pairs = B * w.Hq * visible_pairs_prefill(L, w.window)
+    P = w.prefix
+    # a chunk after P cached positions: rows P .. P+L-1 of the whole sequence's pairs
+    pairs = B * w.Hq * (visible_pairs_prefill(P + L, w.window) - visible_pairs_prefill(P, w.window))
     flops = pairs * FLOP_PER_PAIR
-    nbytes = (B * L * (w.Hq * w.dq + w.Hkv * (w.dq + w.dv) + w.Hq * w.dv) * 2 + B * w.Hq * L * 4)
+    nbytes = (B * L * (w.Hq * w.dq + w.Hq * w.dv) * 2 + B * (P + L) * w.Hkv * (w.dq + w.dv) * 2
+              + B * w.Hq * L * 4)
     return flops, nbytes
 
 
@@ -93,22 +96,29 @@ class PrefillRunner:
     def __init__(self, w, dev):
         import global_attention_sink_softmax_b200 as sa
         self.sa, self.w, self.dev = sa, w, dev
-        self.d = W.prefill_inputs(w, device=dev)
+        self.d = W.prefill_inputs(w, device=dev, L=w.prefix + w.L)
+        if w.prefix:
+            self.d["q"] = self.d["q"][:, w.prefix:]  # the chunk's queries (a strided view)
         self.o = torch.empty(w.B, w.L, w.Hq, w.dv, dtype=torch.bfloat16, device=dev)
         self.lse = torch.empty(w.B, w.Hq, w.L, dtype=torch.float32, device=dev)
         self.flops, self.bytes = prefill_counts(w)
         self.launches = 1
         # the kernel the library dispatches this workload to
-        packed = w.window > 0 and w.Hq // w.Hkv == 8 and w.window <= 128
+        packed = w.window > 0 and w.Hq // w.Hkv == 8 and w.window <= 128 and w.prefix == 0
         self.kernel = "prefill_swa_packed_kernel" if packed else "prefill_band_kernel"
         self.workload = w.name
         self.config = dict(B=w.B, L=w.L, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
                            window=w.window, kind="SWA" if w.window else "GA")
+        if w.prefix:
+            self.config["prefix"] = w.prefix
         self.in_bytes = sum(self.d[k].numel() * self.d[k].element_size() for k in self.d)
 
     def step(self):
         d, w = self.d, self.w
-        if w.window:
+        if w.prefix:
+            self.sa.sinkattn_prefill_chunk(d["q"], d["k"], d["v"], d["sink"], prefix=w.prefix,
+                                           window=w.window, o=self.o, lse=self.lse)
+        elif w.window:
             self.sa.sinkattn_prefill_swa(d["q"], d["k"], d["v"], d["sink"], w.window, o=self.o,
                                          lse=self.lse)
         else:
@@ -488,7 +498,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default=None,
-                    help="run one workload only: swa_prefill, ga_prefill, ga_decode, swa_decode, hybrid")
+                    help="run one workload only: swa_prefill, ga_prefill, ga_chunk_prefill, "
+                         "ga_decode, swa_decode, hybrid")
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--ref-L", type=int, default=0, help="reference arm: shorter sequences (tests)")
     ap.add_argument("--small", action="store_true",
@@ -516,12 +527,14 @@ def main():
     flush = None
 
     swa_w, ga_w, gad_w, swad_w = W.SWA_PREFILL, W.GA_PREFILL, W.GA_DECODE, W.SWA_DECODE
+    gac_w = W.GA_CHUNK
     if args.small:
         import dataclasses
         swa_w = dataclasses.replace(swa_w, B=1, L=16384, name=swa_w.name + "_small_B1_L16384")
         ga_w = dataclasses.replace(ga_w, L=8192, name=ga_w.name + "_small_L8192")
         gad_w = dataclasses.replace(gad_w, B=2, name=gad_w.name + "_small_B2")
         swad_w = dataclasses.replace(swad_w, B=64, name=swad_w.name + "_small_B64")
+        gac_w = dataclasses.replace(gac_w, L=4096, prefix=4096, name=gac_w.name + "_small_P4096_L4096")
 
     def head_runner():
         return PrefillRunner(swa_w, dev)
@@ -571,6 +584,8 @@ def main():
         jobs = []
         if only in (None, "ga_prefill"):
             jobs.append(("ga_prefill", lambda: PrefillRunner(ga_w, dev), None))
+        if only in (None, "ga_chunk_prefill"):
+            jobs.append(("ga_chunk_prefill", lambda: PrefillRunner(gac_w, dev), None))
         if only in (None, "ga_decode"):
             jobs.append(("ga_decode", lambda: DecodeRunner(gad_w, dev), None))
         if only in (None, "swa_decode"):

@@ -7,6 +7,7 @@ library is missing or cannot be loaded, every call raises.
 
     o, lse = sinkattn_prefill_swa(q, k, v, sink, window=128)
     o, lse = sinkattn_prefill_ga(q, k, v, sink)
+    o, lse = sinkattn_prefill_chunk(q_chunk, k_all, v_all, sink, prefix=P)
     o, lse = sinkattn_decode(KV_CONTIG, q, k_new, v_new, k_cache, v_cache, sink, ctx_len=...)
 """
 from __future__ import annotations
@@ -22,7 +23,7 @@ from . import workloads  # noqa: F401  (seeded inputs; no attention arithmetic)
 
 __all__ = [
     "KV_RING", "KV_CONTIG", "KV_PAGED", "SinkAttnError", "lib", "library_path",
-    "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_decode",
+    "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_prefill_chunk", "sinkattn_decode",
     "sinkattn_decode_workspace_size", "sinkattn_kv_commit", "sinkattn_take_device_error",
     "sinkattn_status_string", "sinkattn_version", "EXPORTED_SYMBOLS",
     "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES",
@@ -33,8 +34,8 @@ DQ, DV = 192, 128
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libsinkattn.so")
 EXPORTED_SYMBOLS = [
-    "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_decode_workspace_size",
-    "sinkattn_decode", "sinkattn_kv_commit", "sinkattn_status_string", "sinkattn_version",
+    "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_prefill_chunk",
+    "sinkattn_decode_workspace_size", "sinkattn_decode", "sinkattn_kv_commit", "sinkattn_status_string", "sinkattn_version",
     "sinkattn_take_device_error", "sinkattn_decode_noalloc",
 ]
 # Size of the library's own split-KV workspace used by sinkattn_decode_noalloc.
@@ -93,6 +94,8 @@ def lib() -> ctypes.CDLL:
             L.sinkattn_prefill_swa.argtypes = [ctypes.POINTER(PrefillArgs), _I32, _P]
             L.sinkattn_prefill_swa.restype = ctypes.c_int
             L.sinkattn_prefill_ga.argtypes = [ctypes.POINTER(PrefillArgs), _P]
+            L.sinkattn_prefill_chunk.restype = ctypes.c_int
+            L.sinkattn_prefill_chunk.argtypes = [ctypes.POINTER(PrefillArgs), _I32, _I32, _P]
             L.sinkattn_prefill_ga.restype = ctypes.c_int
             L.sinkattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]
             L.sinkattn_decode_workspace_size.restype = _SZ
@@ -179,7 +182,7 @@ def _prefill_args(q, k, v, sink, o, lse, scale):
     return a
 
 
-def _prefill(fn, q, k, v, sink, window, o, lse, scale, stream, want_lse):
+def _prefill(fn, q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix=0):
     B, L, Hq, dq = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(dq)
@@ -191,6 +194,8 @@ def _prefill(fn, q, k, v, sink, window, o, lse, scale, stream, want_lse):
     L_ = lib()
     if fn == "swa":
         st = L_.sinkattn_prefill_swa(ctypes.byref(a), int(window), _stream(stream))
+    elif fn == "chunk":
+        st = L_.sinkattn_prefill_chunk(ctypes.byref(a), int(prefix), int(window), _stream(stream))
     else:
         st = L_.sinkattn_prefill_ga(ctypes.byref(a), _stream(stream))
     _raise(st, f"sinkattn_prefill_{fn}")
@@ -211,6 +216,17 @@ def sinkattn_prefill_ga(q, k, v, sink=None, *, o=None, lse=None, scale=None, str
                         want_lse=True):
     """Global (full causal) sink attention over whole sequences; arguments as for SWA."""
     return _prefill("ga", q, k, v, sink, 0, o, lse, scale, stream, want_lse)
+
+
+def sinkattn_prefill_chunk(q, k, v, sink=None, *, prefix, window=0, o=None, lse=None, scale=None,
+                           stream=None, want_lse=True):
+    """Chunked prefill against cached keys: q [B,L,Hq,192] are the tokens at positions
+    prefix .. prefix+L-1; k [B,prefix+L,Hkv,192], v [B,prefix+L,Hkv,128] hold every position
+    (the cached prefix, then the chunk). window = 0 full causal, >= 1 sliding window. Returns
+    (o [B,L,Hq,128] bf16, lse [B,Hq,L] fp32 or None)."""
+    if k.shape[1] != prefix + q.shape[1] or v.shape[1] != prefix + q.shape[1]:
+        raise ValueError("k and v must hold prefix + L positions")
+    return _prefill("chunk", q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix)
 
 
 # ----------------------------------------------------------------------------------------------

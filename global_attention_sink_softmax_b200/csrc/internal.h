@@ -9,7 +9,8 @@ namespace sinkattn {
 
 // ---- prefill -------------------------------------------------------------------------------
 struct PrefillParams {
-    int B, L, Hq, Hkv, G;
+    int B, L, Hq, Hkv, G; // L query rows per sequence
+    int q_off;            // position of query row 0 (keys: q_off + L positions)
     int window;           // > 0 sliding window, 0 full causal
     int n_qtiles;         // ceil(L / 128)
     float scale_log2;     // scale * log2(e)
@@ -19,7 +20,7 @@ struct PrefillParams {
     float *lse;           // [B, Hq, L] or nullptr
 };
 
-// Q map: dims {192, Hq, L, B}; K map: {192, Hkv, L, B}; V map: {128, Hkv, L, B}; 128-byte
+// Q map: dims {192, Hq, L, B}; K map: {192, Hkv, q_off + L, B}; V map: {128, Hkv, q_off + L, B}; 128-byte
 // swizzle, 64-element inner box.
 cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                 const CUtensorMap &tmV, const PrefillParams &p,

@@ -6,7 +6,9 @@
 //     O_i = sum_j exp(a_ij - m_i) v_j / (exp(sink_h - m_i) + sum_j exp(a_ij - m_i)),
 //     a_ij = scale <q_i, k_j>, m_i = max(sink_h, max_j a_ij), LSE_i = m_i + ln(denominator).
 //
-// Band kernel. One CTA = 128 query rows of one head against the 128-key tiles of its band:
+// Band kernel. One CTA = 128 query rows of one head against the 128-key tiles of its band (row
+// i sits at position q_off + i: q_off = 0 for whole sequences, the prefix length for a chunk
+// prefilled against cached keys):
 // tiles j_lo .. j_hi where the band is [i - W + 1, i] (SWA, at most 2 tiles for W = 128:
 // "MiMo-V2-Flash 架构 QA" Q3.6) or [0, i] (GA; tiles above the diagonal are never visited).
 //
@@ -96,11 +98,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     const int b = rem / p.Hq;
     const int h = rem - b * p.Hq;
     const int g = h / p.G;
-    const int r0 = qt * BM;
+    const int r0 = qt * BM;                     // first query row of the tile (of the L rows)
     const int r_last = min(r0 + BM, p.L) - 1;
-    const int k_lo = (p.window > 0) ? max(0, r0 - p.window + 1) : 0;
+    const int a0 = p.q_off + r0;                // its position in the sequence (keys index it)
+    const int k_lo = (p.window > 0) ? max(0, a0 - p.window + 1) : 0;
     const int j_lo = k_lo / BN;
-    const int j_hi = r_last / BN;
+    const int j_hi = (p.q_off + r_last) / BN;
     const int n_tiles = j_hi - j_lo + 1;
 
     if (threadIdx.x == 0) {
@@ -227,7 +230,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
     } else {
         // ---------------- softmax warps: thread = query row ----------------
         const int row = threadIdx.x;          // 0..127
-        const int rp = r0 + row;              // position of this query row
+        const int rp = r0 + row;              // this query row (of the L rows)
+        const int ap = p.q_off + rp;          // its position in the sequence
         const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
         const float sink_l2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
         const float c_l2 = p.scale_log2; // > 0, so max(s) * c = max(s * c)
@@ -250,16 +254,16 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             tmem_ld128(tmem + lane_addr + (s ? TMEM_S1 : TMEM_S0), raw);
             float x[128]; // raw scores q.k; masked keys -inf
             // mask only on tiles that cross the diagonal or the window's lower edge
-            const bool need_mask = (kbase + BN - 1 > r0) ||
-                                   (p.window > 0 && kbase < r0 + BM - p.window);
+            const bool need_mask = (kbase + BN - 1 > a0) ||
+                                   (p.window > 0 && kbase < a0 + BM - p.window);
             // eight independent running maxima: short dependency chains
             float mx8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 mx8[i] = -INFINITY;
             if (need_mask) {
-                const int hi = rp - kbase;                                   // keep c <= hi
-                const int lo = (p.window > 0) ? rp - p.window + 1 - kbase : -BN; // keep c >= lo
+                const int hi = ap - kbase;                                   // keep c <= hi
+                const int lo = (p.window > 0) ? ap - p.window + 1 - kbase : -BN; // keep c >= lo
 #pragma unroll
                 for (int c = 0; c < 128; ++c) {
                     x[c] = (c <= hi && c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;

@@ -184,27 +184,33 @@ int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *str
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 
-int run_prefill(const sinkattn_prefill_args *a, int window, void *stream)
+// Prefill of the L query rows at positions prefix .. prefix + L - 1 against keys 0 .. prefix +
+// L - 1 (prefix = 0: whole sequences).
+int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *stream)
 {
     int st = validate_prefill(a);
     if (st != SINKATTN_OK || a->B == 0 || a->L == 0)
         return st;
-    if (window > 0) {
+    if (prefix < 0 || (int64_t)prefix + a->L > 0x7fffffff)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (window > 0 && prefix == 0) {
         bool done = false;
         st = try_prefill_swa_packed(a, window, stream, &done);
         if (st != SINKATTN_OK || done)
             return st;
     }
+    const int n_kv = prefix + a->L;
     CUtensorMap tq, tk, tv;
     if ((st = make_map(&tq, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, 1, 128)))
         return st;
-    if ((st = make_map(&tk, a->k, kDQ, a->Hkv, a->L, a->B, a->k_sh, a->k_sl, a->k_sb, 1, 128)))
+    if ((st = make_map(&tk, a->k, kDQ, a->Hkv, n_kv, a->B, a->k_sh, a->k_sl, a->k_sb, 1, 128)))
         return st;
-    if ((st = make_map(&tv, a->v, kDV, a->Hkv, a->L, a->B, a->v_sh, a->v_sl, a->v_sb, 1, 128)))
+    if ((st = make_map(&tv, a->v, kDV, a->Hkv, n_kv, a->B, a->v_sh, a->v_sl, a->v_sb, 1, 128)))
         return st;
     PrefillParams p;
     p.B = a->B;
     p.L = a->L;
+    p.q_off = prefix;
     p.Hq = a->Hq;
     p.Hkv = a->Hkv;
     p.G = a->Hq / a->Hkv;
@@ -535,12 +541,20 @@ int sinkattn_prefill_swa(const sinkattn_prefill_args *args, int32_t window, void
 {
     if (window < 1)
         return SINKATTN_ERR_INVALID_ARG;
-    return run_prefill(args, window, stream);
+    return run_prefill(args, window, 0, stream);
 }
 
 int sinkattn_prefill_ga(const sinkattn_prefill_args *args, void *stream)
 {
-    return run_prefill(args, 0, stream);
+    return run_prefill(args, 0, 0, stream);
+}
+
+int sinkattn_prefill_chunk(const sinkattn_prefill_args *args, int32_t prefix, int32_t window,
+                           void *stream)
+{
+    if (window < 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    return run_prefill(args, window, prefix, stream);
 }
 
 size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args)

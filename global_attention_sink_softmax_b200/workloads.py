@@ -39,6 +39,7 @@ class PrefillWorkload:
     neg_inf_heads: List[int] = field(default_factory=list)
     dq: int = DQ
     dv: int = DV
+    prefix: int = 0  # chunked prefill: L query tokens after `prefix` cached positions
 
 
 @dataclass
@@ -67,6 +68,11 @@ SWA_PREFILL = PrefillWorkload("swa_prefill_b2_l32768_64q8kv", B=2, L=32768, Hq=6
                               window=128, seed=1236)
 GA_PREFILL = PrefillWorkload("ga_prefill_b1_l32768_64q4kv", B=1, L=32768, Hq=64, Hkv=4, window=0,
                              seed=1237, neg_inf_heads=[h for h in range(64) if h % 8 == 7])
+# Chunked prefill (the serving command's --chunked-prefill-size 16384): the second 16384-token
+# chunk of a 32768-token GA prompt, against the first chunk's cached keys.
+GA_CHUNK = PrefillWorkload("ga_chunk_prefill_b1_p16384_l16384_64q4kv", B=1, L=16384, Hq=64, Hkv=4,
+                           window=0, seed=1300, neg_inf_heads=[h for h in range(64) if h % 8 == 7],
+                           prefix=16384)
 GA_DECODE = DecodeWorkload("ga_decode_b8_ctx262144_64q4kv", kind=KV_CONTIG, B=8, T=1, Hq=64,
                            Hkv=4, window=0, seed=1238, ctx=262144)
 SWA_DECODE = DecodeWorkload("swa_decode_b256_ring128_64q8kv", kind=KV_RING, B=256, T=1, Hq=64,

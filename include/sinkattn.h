@@ -107,6 +107,19 @@ int sinkattn_prefill_swa(const sinkattn_prefill_args *args, int32_t window, void
 /* Global (full causal) prefill (GA). Key tiles above the diagonal are skipped. */
 int sinkattn_prefill_ga(const sinkattn_prefill_args *args, void *stream);
 
+/* Chunked prefill against cached keys: a long prompt prefilled in chunks (the serving command of
+ * the "MiMo-V2-Flash" model card, --chunked-prefill-size 16384), or a new turn after a cached
+ * prefix ("MiMo-V2-Flash 模型架构深度拆解" §7.4, request-level prefix cache).
+ *   args->q, o, lse: the L query rows, at positions prefix .. prefix + L - 1 of their sequences
+ *                    ([B, L, Hq, ...] and lse [B, Hq, L], as for whole sequences);
+ *   args->k, v:      all prefix + L positions of the sequences (the cached prefix followed by
+ *                    the chunk's own keys), [B, prefix + L, Hkv, ...] with args' k / v strides;
+ *   prefix >= 0;     window = 0: full causal (GA), window >= 1: sliding window (SWA).
+ * The result equals rows prefix .. prefix + L - 1 of the whole-sequence prefill.
+ * Errors: as for the whole-sequence calls; prefix < 0 or window < 0 is INVALID_ARG. */
+int sinkattn_prefill_chunk(const sinkattn_prefill_args *args, int32_t prefix, int32_t window,
+                           void *stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Decode / speculative verify: T (1..4) new query tokens per sequence attend to that sequence's
  * cached tokens plus new tokens 0..t. The new tokens' K/V are passed separately and are NOT yet

@@ -154,3 +154,42 @@ def test_full_size_workloads_sampled_rows(w):
     lg = lse.cpu().permute(0, 2, 1)[idx_b, idx_i]
     assert_close(og, ro, lg, rl, w.name)
     assert sa.sinkattn_take_device_error() == 0
+
+
+@pytest.mark.parametrize("B,P,L,Hq,Hkv,window", [
+    (1, 0, 200, 16, 1, 0), (2, 1, 129, 16, 1, 0), (1, 127, 1, 8, 1, 0), (1, 128, 128, 16, 4, 0),
+    (1, 300, 257, 16, 1, 0), (2, 1000, 300, 8, 2, 0), (1, 200, 300, 8, 1, 128),
+    (1, 50, 77, 4, 1, 7), (1, 129, 64, 8, 8, 200),
+])
+@pytest.mark.parametrize("sink_mode", ["rand", "none"])
+def test_chunked_prefill(B, P, L, Hq, Hkv, window, sink_mode):
+    """A chunk of L tokens after a P-token prefix equals rows P .. P+L-1 of the whole-sequence
+    prefill of the concatenated sequence (the oracle, restricted to those rows)."""
+    q, k, v, s = rand_inputs(B, P + L, Hq, Hkv, 31 * P + L + window, sink_mode)
+    dev = "cuda"
+    o, lse = sa.sinkattn_prefill_chunk(q[:, P:].to(dev), k.to(dev), v.to(dev),
+                                       None if s is None else s.to(dev), prefix=P, window=window)
+    torch.cuda.synchronize()
+    rows = [[b, P + i] for b in range(B) for i in range(L)]
+    ro, rl, _ = oracle.prefill(q, k, v, s, 1 / math.sqrt(192), window, rows=rows)
+    assert_close(o.reshape(B * L, Hq, 128), ro, lse.permute(0, 2, 1).reshape(B * L, Hq), rl,
+                 f"chunk P{P} L{L} W{window}")
+    assert sa.sinkattn_take_device_error() == 0
+
+
+def test_chunked_prefill_full_size_sampled():
+    """The chunk workload of the benchmark (GA, B=1, a 16384-token chunk after a 16384-token
+    prefix, 64 Q / 4 KV), on sampled rows."""
+    w = W.GA_CHUNK
+    d = W.prefill_inputs(w, device="cuda", L=w.prefix + w.L)
+    o, lse = sa.sinkattn_prefill_chunk(d["q"][:, w.prefix:], d["k"], d["v"], d["sink"],
+                                       prefix=w.prefix)
+    torch.cuda.synchronize()
+    g = torch.Generator().manual_seed(5)
+    sample = sorted(set([0, 1, 127, 128, 129, w.L - 1] + torch.randint(0, w.L, (26,), generator=g).tolist()))
+    rows = [[0, w.prefix + i] for i in sample]
+    ro, rl, _ = oracle.prefill(d["q"].cpu(), d["k"].cpu(), d["v"].cpu(), d["sink"].cpu(),
+                               1 / math.sqrt(192), 0, rows=rows)
+    idx = torch.tensor(sample)
+    assert_close(o[0, idx].cpu(), ro, lse[0][:, idx].permute(1, 0).cpu(), rl, w.name)
+    assert sa.sinkattn_take_device_error() == 0
