@@ -245,14 +245,26 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
     } else if (warp == WARP_MMA) {
         if (lane == 0 && cnt > 0) {
             const uint32_t idesc_o = umma_idesc_bf16(128, 128, 1);
-            const uint32_t sK = smem_u32(smem + off_k());
-            const uint32_t sV = smem_u32(smem + off_v(p.P));
-            int base_s = 0, base_pv = 0;
+            // Operand descriptors are built once; a k-step or a ring slot only advances the
+            // start-address field (16-byte units; shared memory < 256 KB, so it never carries).
+            // This thread shares its SMSP with two softmax warps, so it issues few instructions;
+            // its loops stay rolled (the kernel's code must fit the instruction caches).
+            const uint64_t kd0 = smem_desc_sw128(smem_u32(smem + off_k()), 16, 1024);
+            const uint64_t vd0 = smem_desc_sw128(smem_u32(smem + off_v(p.P)), R * CHUNK, 1024);
+            const uint64_t qd0 = smem_desc_sw128(smem_u32(smem), 16, 1024);
+            const uint64_t qd1 = smem_desc_sw128(smem_u32(smem + Q_BYTES), 16, 1024);
+            const uint32_t region16 = (uint32_t)(R * CHUNK) >> 4; // one 64-dim region of a ring
+            int base_s = 0;
+            int base_even = 0, base_odd = 0; // ring slot of the span's first key, per item parity
             // S of item n into S buffer n & 1 (warpgroup n & 1). The span is ring slots
             // base .. base + SC - 1: one MMA per k-step, or two where it wraps.
             auto issue_s = [&](int n) -> bool {
                 const SwaItem it = swa_item(p, it0 + n, n == 0);
                 base_s = swa_next_base(p, it, base_s);
+                if (n & 1)
+                    base_odd = base_s;
+                else
+                    base_even = base_s;
                 const int sb = n & 1;
                 if (!mbar_wait(&bars[Q_FULL + sb], (n >> 1) & 1, abort, 1u) ||
                     !mbar_wait(&bars[K_FULL + (n & 1)], (n >> 1) & 1, abort, 1u))
@@ -261,21 +273,20 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                 if (n >= 2 && !mbar_wait(&bars[S_FREE + sb], ((n >> 1) - 1) & 1, abort, 1u))
                     return false;
                 tc_fence_after();
-                const uint32_t sQ = smem_u32(smem + sb * Q_BYTES);
                 const int ca = min(SC, R - base_s); // chunks before the wrap
                 const int na = ca * 16, nb = NSC - na;
                 const uint32_t idesc_a = umma_idesc_bf16(128, na, 0);
                 const uint32_t idesc_b = nb > 0 ? umma_idesc_bf16(128, nb, 0) : 0u;
+                const uint64_t qd = sb ? qd1 : qd0;
+                const uint64_t ka = kd0 + (uint32_t)((base_s * CHUNK) >> 4);
+                const uint32_t d = tmem + sb * NSC;
 #pragma unroll 1
                 for (int kk = 0; kk < 12; ++kk) {
-                    const uint32_t koff = (kk & 3) * 32;
-                    const uint64_t adesc = smem_desc_sw128(sQ + (kk >> 2) * Q_REGION + koff, 16, 1024);
-                    const uint32_t kreg = sK + (kk >> 2) * R * CHUNK + koff;
-                    umma_ss(tmem + sb * NSC, adesc, smem_desc_sw128(kreg + base_s * CHUNK, 16, 1024),
-                            idesc_a, kk > 0);
+                    const uint32_t qo = (uint32_t)((kk >> 2) * Q_REGION + (kk & 3) * 32) >> 4;
+                    const uint32_t ko = (kk >> 2) * region16 + (((kk & 3) * 32) >> 4);
+                    umma_ss(d, qd + qo, ka + ko, idesc_a, kk > 0);
                     if (nb > 0)
-                        umma_ss(tmem + sb * NSC + na, adesc, smem_desc_sw128(kreg, 16, 1024),
-                                idesc_b, kk > 0);
+                        umma_ss(d + na, qd + qo, kd0 + ko, idesc_b, kk > 0);
                 }
                 umma_commit(&bars[S_FULL + sb]);
                 umma_commit(&bars[Q_EMPTY + sb]);
@@ -285,8 +296,7 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             // issue order S_0, {S_{n+1}, PV_n}
             bool ok = issue_s(0);
             for (int n = 0; ok && n < cnt; ++n) {
-                const SwaItem it = swa_item(p, it0 + n, n == 0);
-                base_pv = swa_next_base(p, it, base_pv);
+                const int base_pv = (n & 1) ? base_odd : base_even; // set by issue_s(n)
                 if (n + 1 < cnt && !issue_s(n + 1))
                     break;
                 if (!mbar_wait(&bars[P_FULL + (n & 1)], (n >> 1) & 1, abort, 1u) ||
@@ -297,10 +307,12 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                     break;
                 tc_fence_after();
                 const uint32_t pt = tmem + (n & 1) * NSC; // P: 16 keys per 8 columns
+#pragma unroll 1
                 for (int kk = 0; kk < SC; ++kk) {
-                    const int slot = (base_pv + kk) % R;
-                    umma_ts(tmem + TMEM_O, pt + kk * 8,
-                            smem_desc_sw128(sV + slot * CHUNK, R * CHUNK, 1024), idesc_o, kk > 0);
+                    int slot = base_pv + kk;
+                    slot = slot >= R ? slot - R : slot;
+                    umma_ts(tmem + TMEM_O, pt + kk * 8, vd0 + (uint32_t)((slot * CHUNK) >> 4), idesc_o,
+                            kk > 0);
                 }
                 umma_commit(&bars[PV_DONE + (n & 1)]);
                 umma_commit(&bars[V_EMPTY + (n & 1)]);
