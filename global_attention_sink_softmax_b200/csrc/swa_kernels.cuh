@@ -256,11 +256,14 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             const uint32_t region16 = (uint32_t)(R * CHUNK) >> 4; // one 64-dim region of a ring
             int base_s = 0;
             int base_even = 0, base_odd = 0; // ring slot of the span's first key, per item parity
+            int pblk = (it0 % p.n_pblk) - 1; // position block of the last item issued
             // S of item n into S buffer n & 1 (warpgroup n & 1). The span is ring slots
-            // base .. base + SC - 1: one MMA per k-step, or two where it wraps.
+            // base .. base + SC - 1: one MMA per k-step, or two where it wraps. A CTA's items
+            // are consecutive, so the position block and the ring base advance without division.
             auto issue_s = [&](int n) -> bool {
-                const SwaItem it = swa_item(p, it0 + n, n == 0);
-                base_s = swa_next_base(p, it, base_s);
+                pblk = (pblk + 1 == p.n_pblk) ? 0 : pblk + 1;
+                const int nb_ = base_s + p.P / 16;
+                base_s = (n == 0 || pblk == 0) ? 0 : (nb_ >= R ? nb_ - R : nb_);
                 if (n & 1)
                     base_odd = base_s;
                 else
