@@ -108,6 +108,18 @@ def test_prefill_rejects_bad_arguments(L, kw, status):
     a = _prefill_args(**kw)
     assert L.sinkattn_prefill_ga(ctypes.byref(a), None) == status
     assert L.sinkattn_prefill_swa(ctypes.byref(a), 128, None) == status
+    assert L.sinkattn_prefill_chunk(ctypes.byref(a), 100, 0, None) == status
+
+
+def test_chunk_checks_prefix_and_window(L):
+    """Rejected before any device work: a negative prefix or window, and a sequence whose
+    positions overflow int32; an empty chunk is a no-op."""
+    a = _prefill_args()
+    assert L.sinkattn_prefill_chunk(ctypes.byref(a), -1, 0, None) == 1
+    assert L.sinkattn_prefill_chunk(ctypes.byref(a), 0, -1, None) == 1
+    assert L.sinkattn_prefill_chunk(ctypes.byref(a), 0x7fffffff - 10, 0, None) == 1
+    assert L.sinkattn_prefill_chunk(ctypes.byref(_prefill_args(L=0)), 5, 0, None) == 0
+    assert L.sinkattn_prefill_chunk(None, 0, 0, None) == 1
 
 
 def test_prefill_empty_is_ok_and_window_checked(L):
