@@ -15,15 +15,17 @@
 // Roles (224 threads):
 //   warps 0-3  softmax + epilogue: thread t owns query row t (TMEM lane t). It reads its row of
 //              S from TMEM, runs the online softmax seeded with the sink (m0 = sink, l0 = 1),
-//              writes P (bf16) into shared memory in the UMMA 128B-swizzled K-major layout,
+//              writes P (bf16 pairs) back over its S row in TMEM (the A operand of P.V),
 //              rescales its O row in TMEM when needed, and at the end normalises O and writes
 //              O (bf16) and LSE.
 //   warp 4     TMA producer for Q (once) and K tiles (2-stage ring).
-//   warp 5     TMA producer for V tiles (1 stage).
+//   warp 5     TMA producer for V tiles (2-stage ring).
 //   warp 6     TMEM allocator and the single UMMA issuer: S = Q K^T (M128 N128 K16 x 12) into
-//              a double-buffered S in TMEM, O += P V (M128 N128 K16 x 8) into O in TMEM.
+//              one of three S buffers in TMEM, O += P V (M128 N128 K16 x 8, A = P from TMEM)
+//              into O in TMEM (3 x 128 S columns + 128 O columns fill the 512). S_{j+3}
+//              reuses the buffer of P_j once P_j V_j is done, long after it was issued.
 // The issue order S_0, {S_{j+1}, PV_j} lets the tensor cores compute S_{j+1} while the softmax
-// warps work on S_j.
+// warps work on S_j; the softmax waits for PV_{j-1} only when it has to rescale O.
 //
 // Two row sums: O is normalised by the sum of the bf16-rounded P values (the ones the P.V MMA
 // multiplies), so numerator and denominator use identical weights; LSE uses the fp32 sum.
@@ -46,31 +48,31 @@ constexpr int Q_BYTES = 3 * Q_REGION;    // 192 dims
 constexpr int K_REGION = BN * ROW_BYTES;
 constexpr int K_BYTES = 3 * K_REGION;
 constexpr int V_BYTES = 2 * K_REGION;    // 128 dims
-constexpr int P_BYTES = 2 * BM * ROW_BYTES;
 constexpr int K_STAGES = 2;
+constexpr int V_STAGES = 2;
 constexpr int OFF_Q = 0;
 constexpr int OFF_K = OFF_Q + Q_BYTES;
 constexpr int OFF_V = OFF_K + K_STAGES * K_BYTES;
-constexpr int OFF_P = OFF_V + V_BYTES;
-constexpr int OFF_BAR = OFF_P + P_BYTES;
+constexpr int OFF_BAR = OFF_V + V_STAGES * V_BYTES;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024; // barriers + 1 KB for aligning the base
 constexpr int THREADS = 224;
 constexpr int WARP_KLOAD = 4, WARP_VLOAD = 5, WARP_MMA = 6;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O = 256;
+constexpr int S_BUFS = 3;                   // S / P buffers in TMEM, 128 columns each
+constexpr uint32_t TMEM_O = S_BUFS * BN;    // O: the last 128 columns
 constexpr float TAU = 8.0f;
 
 enum Bar {
     B_Q = 0,
-    B_KFULL = 1,   // + stage
-    B_KEMPTY = 3,  // + stage
-    B_VFULL = 5,
-    B_VEMPTY = 6,
-    B_SFULL = 7,   // + buffer
-    B_PFULL = 9,
-    B_PVDONE = 10,
-    B_DRAIN = 11,
-    NUM_BARS = 12
+    B_KFULL = 1,   // + K stage
+    B_KEMPTY = 3,  // + K stage
+    B_VFULL = 5,   // + V stage
+    B_VEMPTY = 7,  // + V stage
+    B_SFULL = 9,   // + S buffer
+    B_PFULL = 12,  // + S buffer
+    B_PVDONE = 15, // + S buffer
+    B_DRAIN = 18,
+    NUM_BARS = 19
 };
 } // namespace pf
 
@@ -108,16 +110,17 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 
     if (threadIdx.x == 0) {
         mbar_init(&bars[B_Q], 1);
-        mbar_init(&bars[B_KFULL + 0], 1);
-        mbar_init(&bars[B_KFULL + 1], 1);
-        mbar_init(&bars[B_KEMPTY + 0], 1);
-        mbar_init(&bars[B_KEMPTY + 1], 1);
-        mbar_init(&bars[B_VFULL], 1);
-        mbar_init(&bars[B_VEMPTY], 1);
-        mbar_init(&bars[B_SFULL + 0], 1);
-        mbar_init(&bars[B_SFULL + 1], 1);
-        mbar_init(&bars[B_PFULL], 128);
-        mbar_init(&bars[B_PVDONE], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bars[B_KFULL + i], 1);
+            mbar_init(&bars[B_KEMPTY + i], 1);
+            mbar_init(&bars[B_VFULL + i], 1);
+            mbar_init(&bars[B_VEMPTY + i], 1);
+        }
+        for (int i = 0; i < S_BUFS; ++i) {
+            mbar_init(&bars[B_SFULL + i], 1);
+            mbar_init(&bars[B_PFULL + i], 128);
+            mbar_init(&bars[B_PVDONE + i], 1);
+        }
         mbar_init(&bars[B_DRAIN], 1);
         *abort = 0;
         fence_mbar_init();
@@ -161,17 +164,18 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             tma_prefetch_desc(&tmV);
             int issued = 0;
             for (int idx = 0; idx < n_tiles; ++idx) {
-                if (idx >= 1 && !mbar_wait(&bars[B_VEMPTY], (idx - 1) & 1, abort, 1u))
+                const int vs = idx & 1;
+                if (idx >= 2 && !mbar_wait(&bars[B_VEMPTY + vs], ((idx >> 1) - 1) & 1, abort, 1u))
                     break;
                 const int j = j_lo + idx;
-                mbar_arrive_expect_tx(&bars[B_VFULL], V_BYTES);
+                mbar_arrive_expect_tx(&bars[B_VFULL + vs], V_BYTES);
                 for (int c = 0; c < 2; ++c)
-                    tma_load_4d(smem + OFF_V + c * K_REGION, &tmV, &bars[B_VFULL], c * 64, g,
-                                j * BN, b);
+                    tma_load_4d(smem + OFF_V + vs * V_BYTES + c * K_REGION, &tmV,
+                                &bars[B_VFULL + vs], c * 64, g, j * BN, b);
                 issued = idx + 1;
             }
-            if (issued > 0)
-                mbar_wait_drain(&bars[B_VFULL], (issued - 1) & 1);
+            for (int idx = max(0, issued - 2); idx < issued; ++idx)
+                mbar_wait_drain(&bars[B_VFULL + (idx & 1)], (idx >> 1) & 1);
         }
         __syncwarp();
     } else if (warp == WARP_MMA) {
@@ -181,23 +185,26 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             const uint32_t sQ = smem_u32(smem + OFF_Q);
             const uint32_t sK = smem_u32(smem + OFF_K);
             const uint32_t sV = smem_u32(smem + OFF_V);
-            const uint32_t sP = smem_u32(smem + OFF_P);
             bool ok = mbar_wait(&bars[B_Q], 0, abort, 1u);
-            // S_idx = Q K_idx^T into S buffer idx & 1
+            // S_idx = Q K_idx^T into S buffer idx % 3, from K stage idx & 1
             auto issue_s = [&](int idx) -> bool {
-                const int s = idx & 1;
-                if (!mbar_wait(&bars[B_KFULL + s], (idx >> 1) & 1, abort, 1u))
+                const int ks = idx & 1, sb = idx % S_BUFS;
+                if (!mbar_wait(&bars[B_KFULL + ks], (idx >> 1) & 1, abort, 1u))
+                    return false;
+                // the buffer holds P of tile idx - 3 until its P.V is done
+                if (idx >= S_BUFS &&
+                    !mbar_wait(&bars[B_PVDONE + sb], (idx / S_BUFS - 1) & 1, abort, 1u))
                     return false;
                 tc_fence_after();
-                const uint32_t d = tmem + (s ? TMEM_S1 : TMEM_S0);
+                const uint32_t d = tmem + sb * BN;
 #pragma unroll
                 for (int kk = 0; kk < 12; ++kk) {
                     const uint32_t off = (kk >> 2) * Q_REGION + (kk & 3) * 32;
                     umma_ss(d, smem_desc_sw128(sQ + off, 16, 1024),
-                            smem_desc_sw128(sK + s * K_BYTES + off, 16, 1024), idesc_s, kk > 0);
+                            smem_desc_sw128(sK + ks * K_BYTES + off, 16, 1024), idesc_s, kk > 0);
                 }
-                umma_commit(&bars[B_SFULL + s]);
-                umma_commit(&bars[B_KEMPTY + s]);
+                umma_commit(&bars[B_SFULL + sb]);
+                umma_commit(&bars[B_KEMPTY + ks]);
                 return true;
             };
             if (ok)
@@ -205,22 +212,24 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             for (int idx = 0; ok && idx < n_tiles; ++idx) {
                 if (idx + 1 < n_tiles && !issue_s(idx + 1))
                     break;
-                if (!mbar_wait(&bars[B_PFULL], idx & 1, abort, 1u))
+                const int sb = idx % S_BUFS, vs = idx & 1;
+                if (!mbar_wait(&bars[B_PFULL + sb], (idx / S_BUFS) & 1, abort, 1u))
                     break;
-                if (!mbar_wait(&bars[B_VFULL], idx & 1, abort, 1u))
+                if (!mbar_wait(&bars[B_VFULL + vs], (idx >> 1) & 1, abort, 1u))
                     break;
                 tc_fence_after();
+                const uint32_t pt = tmem + sb * BN; // P over S
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
-                    // A = P (128 rows x 16 keys, K-major); B = V (16 keys x 128 dims, dims
-                    // contiguous: MN-major, dims 64..127 one 16 KB region further on)
-                    umma_ss(tmem + TMEM_O,
-                            smem_desc_sw128(sP + (kk >> 2) * Q_REGION + (kk & 3) * 32, 16, 1024),
-                            smem_desc_sw128(sV + kk * 16 * ROW_BYTES, K_REGION, 1024), idesc_o,
-                            (idx > 0 || kk > 0) ? 1u : 0u);
+                    // A = P (128 rows x 16 keys: 8 TMEM columns of bf16 pairs); B = V (16 keys x
+                    // 128 dims, dims contiguous: MN-major, dims 64..127 one 16 KB region further on)
+                    umma_ts(tmem + TMEM_O, pt + kk * 8,
+                            smem_desc_sw128(sV + vs * V_BYTES + kk * 16 * ROW_BYTES, K_REGION,
+                                            1024),
+                            idesc_o, (idx > 0 || kk > 0) ? 1u : 0u);
                 }
-                umma_commit(&bars[B_PVDONE]);
-                umma_commit(&bars[B_VEMPTY]);
+                umma_commit(&bars[B_PVDONE + sb]);
+                umma_commit(&bars[B_VEMPTY + vs]);
             }
             // every MMA of ours has finished before TMEM is released
             umma_commit(&bars[B_DRAIN]);
@@ -241,17 +250,16 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         float m_run = sink_l2;
         float l_exact = (sink_l2 > -INFINITY) ? 1.f : 0.f;
         float l_round = l_exact;
-        uint8_t *prow = smem + OFF_P + row * ROW_BYTES;
         bool ok = true;
         for (int idx = 0; idx < n_tiles; ++idx) {
-            const int s = idx & 1;
+            const int sb = idx % S_BUFS;
             const int kbase = (j_lo + idx) * BN;
-            ok = warp_wait(&bars[B_SFULL + s], (idx >> 1) & 1, abort);
+            ok = warp_wait(&bars[B_SFULL + sb], (idx / S_BUFS) & 1, abort);
             if (!ok)
                 break;
             tc_fence_after();
             uint32_t raw[128];
-            tmem_ld128(tmem + lane_addr + (s ? TMEM_S1 : TMEM_S0), raw);
+            tmem_ld128(tmem + lane_addr + sb * BN, raw);
             float x[128]; // raw scores q.k; masked keys -inf
             // mask only on tiles that cross the diagonal or the window's lower edge
             const bool need_mask = (kbase + BN - 1 > a0) ||
@@ -289,57 +297,52 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 l_round *= alpha;
                 m_run = mx;
             }
-            if (idx > 0) {
-                // PV of the previous tile is done: P buffer free, O up to date
-                ok = warp_wait(&bars[B_PVDONE], (idx - 1) & 1, abort);
+            // O is only touched when one of this warp's rows raises its max: then wait for the
+            // P.V of the previous tile (O up to date) and rescale. Otherwise P of this tile goes
+            // into its own S buffer while that P.V may still run.
+            if (idx > 0 && __any_sync(0xffffffffu, rescale)) {
+                const int pb = (idx - 1) % S_BUFS;
+                ok = warp_wait(&bars[B_PVDONE + pb], ((idx - 1) / S_BUFS) & 1, abort);
                 if (!ok)
                     break;
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * 32, o);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * 32, o);
 #pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tmem_st32(tmem + lane_addr + TMEM_O + c * 32, o);
-                    }
-                    tmem_st_wait();
+                    for (int e = 0; e < 32; ++e)
+                        o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32(tmem + lane_addr + TMEM_O + c * 32, o);
                 }
+                tmem_st_wait();
             }
             const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
             float pe[4] = {0.f, 0.f, 0.f, 0.f}, pr[4] = {0.f, 0.f, 0.f, 0.f};
+            // P (bf16 pairs: keys 2c, 2c + 1 in column c) over this row's S in TMEM
+            const uint32_t paddr = tmem + lane_addr + sb * BN;
 #pragma unroll
-            for (int c8 = 0; c8 < 16; ++c8) {
-                float e[8];
+            for (int c16 = 0; c16 < 8; ++c16) {
+                uint32_t pk[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u)
-                    e[u] = fast_exp2(fmaf(x[c8 * 8 + u], c_l2, neg_m));
-                uint4 pk;
-                pk.x = pack_bf16x2(e[0], e[1]);
-                pk.y = pack_bf16x2(e[2], e[3]);
-                pk.z = pack_bf16x2(e[4], e[5]);
-                pk.w = pack_bf16x2(e[6], e[7]);
-                pe[0] += e[0] + e[1];
-                pe[1] += e[2] + e[3];
-                pe[2] += e[4] + e[5];
-                pe[3] += e[6] + e[7];
-                pr[0] += sum_bf16x2(pk.x);
-                pr[1] += sum_bf16x2(pk.y);
-                pr[2] += sum_bf16x2(pk.z);
-                pr[3] += sum_bf16x2(pk.w);
-                const int region = c8 >> 3, chunk = (c8 & 7) ^ (row & 7);
-                *reinterpret_cast<uint4 *>(prow + region * Q_REGION + chunk * 16) = pk;
+                for (int u = 0; u < 8; ++u) {
+                    const float e0 = fast_exp2(fmaf(x[c16 * 16 + 2 * u], c_l2, neg_m));
+                    const float e1 = fast_exp2(fmaf(x[c16 * 16 + 2 * u + 1], c_l2, neg_m));
+                    pk[u] = pack_bf16x2(e0, e1);
+                    pe[u & 3] += e0 + e1;
+                    pr[u & 3] += sum_bf16x2(pk[u]);
+                }
+                tmem_st8(paddr + c16 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
             }
             l_exact += (pe[0] + pe[1]) + (pe[2] + pe[3]);
             l_round += (pr[0] + pr[1]) + (pr[2] + pr[3]);
-            fence_async_smem();
+            tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&bars[B_PFULL]);
+            mbar_arrive(&bars[B_PFULL + sb]);
         }
         if (ok && n_tiles > 0)
-            ok = warp_wait(&bars[B_PVDONE], (n_tiles - 1) & 1, abort);
+            ok = warp_wait(&bars[B_PVDONE + (n_tiles - 1) % S_BUFS],
+                           ((n_tiles - 1) / S_BUFS) & 1, abort);
         if (ok) {
             tc_fence_after();
             const float inv_l = 1.f / l_round;
