@@ -65,6 +65,10 @@ def _load():
             lib.sinkattn_oracle_commit.argtypes = [i32, P, P, P, P, P, P, P, i32, P, i32, P, i32,
                                                    i32, i32, i32, i32, i32, i32]
             lib.sinkattn_oracle_commit.restype = i32
+            lib.sinkattn_oracle_rope.argtypes = [P, P, i64, i32, i32, i32, f64, P]
+            lib.sinkattn_oracle_rope.restype = i32
+            lib.sinkattn_oracle_vscale.argtypes = [P, i64, f64, P]
+            lib.sinkattn_oracle_vscale.restype = None
             _lib = lib
     return _lib
 
@@ -219,3 +223,31 @@ def commit(kind, k_new, v_new, n_accept, k_cache, v_cache, *, ring_head=None, ri
 
     to_t = (lambda a: None if a is None else torch.from_numpy(a))
     return back(kcb, k_cache), back(vcb, v_cache), to_t(rh), to_t(rl), to_t(cl)
+
+
+def rope(x, pos, theta, rope_dim=64):
+    """Partial rotary embedding of the first rope_dim dims of every head.
+
+    x [..., H, d] bf16 (any leading dims); pos: positions with x's leading shape (one per row
+    of H heads). Returns float64 [..., H, d]."""
+    lib = _load()
+    *lead, H, d = x.shape
+    n = int(np.prod(lead)) if lead else 1
+    xb = _bits(x)
+    p = np.ascontiguousarray(np.broadcast_to(np.asarray(pos.cpu() if isinstance(pos, torch.Tensor)
+                                                        else pos, dtype=np.int64), lead)).reshape(-1)
+    out = np.zeros((n, H, d), np.float64)
+    rc = lib.sinkattn_oracle_rope(_ptr(xb), _ptr(p), n, H, d, int(rope_dim), float(theta),
+                                  _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle rope: bad arguments")
+    return torch.from_numpy(out.reshape(x.shape))
+
+
+def vscale(v, v_scale):
+    """Every element of v (bf16) times v_scale, float64."""
+    lib = _load()
+    vb = _bits(v)
+    out = np.zeros(vb.size, np.float64)
+    lib.sinkattn_oracle_vscale(_ptr(vb), vb.size, float(v_scale), _ptr(out))
+    return torch.from_numpy(out.reshape(v.shape))

@@ -31,7 +31,10 @@
  *
  * "Parity pinned": every function here is checked, in tests/test_oracle_pins.py, against the
  * worked example's printed numbers, a library softmax/logsumexp, a library attention routine,
- * and invariants the mathematics fixes.
+ * closed-form rotation angles, and invariants the mathematics fixes.
+ *
+ * The last two functions restate the steps that precede the attention core (the value scale
+ * and partial rotary position embedding), which the library fuses into one pass.
  *
  * Inputs are bf16 bit patterns (uint16). Each is converted exactly to fp64; all arithmetic is
  * fp64. Arrays are contiguous, token-major: [B, L, H, d].
@@ -376,4 +379,56 @@ int sinkattn_oracle_commit(int kind, const uint16_t *k_new, const uint16_t *v_ne
         }
     }
     return 0;
+}
+
+/*
+ * The two steps just before the attention core: the value scale and partial rotary position
+ * embedding. [ARCH] CH10.3 lists the attention module's order: Q/K/V projection, value_states
+ * times v_scale (0.707), split Q/K into 64 rotary | 128 no-pe dims, rotate the first 64,
+ * concatenate, then attention. [ARCH] CH3.5 and CH8.1: partial_rotary_factor 0.334 (64 of the
+ * 192 Q/K dims), rope_theta 5,000,000 on GA layers and swa_rope_theta 10,000 on SWA layers
+ * ([ARCH] CH10.5; [QA] Q2.7). [QA] Q2.7: at position m, dimension i turns by m * theta^(-2i/d).
+ *
+ * Readings where the pages leave it open:
+ *   - d in that angle is the rotated width rope_dim, and i counts dimension PAIRS,
+ *     0 <= i < rope_dim/2: pair i turns at w_i = theta^(-2i/rope_dim);
+ *   - pair i is dims (i, i + rope_dim/2) ("rotate half"), turned counter-clockwise:
+ *         y_i              = x_i cos(m w_i) - x_{i+rope_dim/2} sin(m w_i)
+ *         y_{i+rope_dim/2} = x_{i+rope_dim/2} cos(m w_i) + x_i sin(m w_i)
+ *   - the rotary embedding scales nothing else (its attention scaling is 1);
+ *   - dims rope_dim .. d-1 pass unchanged.
+ *
+ *   x [n, H, d] bf16 bits; pos [n]: the position of row n (all H heads); out [n, H, d] fp64.
+ * Returns 0, or -1 on a bad argument.
+ */
+int sinkattn_oracle_rope(const uint16_t *x, const int64_t *pos, int64_t n, int H, int d,
+                         int rope_dim, double theta, double *out)
+{
+    if (n < 0 || H < 0 || rope_dim < 2 || rope_dim % 2 != 0 || rope_dim > d || !(theta > 0.0))
+        return -1;
+    const int half = rope_dim / 2;
+    for (int64_t r = 0; r < n; ++r) {
+        for (int h = 0; h < H; ++h) {
+            const uint16_t *xr = x + (r * H + h) * d;
+            double *yr = out + (r * H + h) * d;
+            for (int c = 0; c < d; ++c)
+                yr[c] = bf16_to_f64(xr[c]);
+            for (int i = 0; i < half; ++i) {
+                const double w = pow(theta, -2.0 * i / rope_dim);
+                const double angle = (double)pos[r] * w;
+                const double cs = cos(angle), sn = sin(angle);
+                const double a = bf16_to_f64(xr[i]), b = bf16_to_f64(xr[i + half]);
+                yr[i] = a * cs - b * sn;
+                yr[i + half] = b * cs + a * sn;
+            }
+        }
+    }
+    return 0;
+}
+
+/* The value scale, [ARCH] CH10.3: every value element times v_scale. v [n] bf16 bits. */
+void sinkattn_oracle_vscale(const uint16_t *v, int64_t n, double v_scale, double *out)
+{
+    for (int64_t e = 0; e < n; ++e)
+        out[e] = bf16_to_f64(v[e]) * v_scale;
 }

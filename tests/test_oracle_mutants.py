@@ -36,6 +36,15 @@ MUTANTS = [
     ("paged row ignores the page size", "*\n                                      page_size + c % page_size;",
      "+ c % page_size;", 0),
     ("commit ring overwrites the newest", "slot = ring_head[b];\n", "slot = (ring_head[b] + ring_cap - 1) % ring_cap;\n", 0),
+    ("rope sine sign flipped", "yr[i] = a * cs - b * sn;", "yr[i] = a * cs + b * sn;", 0),
+    ("rope frequency over the whole head dim", "pow(theta, -2.0 * i / rope_dim)",
+     "pow(theta, -2.0 * i / d)", 0),
+    ("rope frequency exponent without the 2", "pow(theta, -2.0 * i / rope_dim)",
+     "pow(theta, -1.0 * i / rope_dim)", 0),
+    ("rope pairs one full width apart", "const int half = rope_dim / 2;", "const int half = rope_dim;", 0),
+    ("rope also turns the no-pe dims", "for (int i = 0; i < half; ++i) {\n                const double w",
+     "for (int i = 0; i < d / 2; ++i) {\n                const double w", 0),
+    ("value scale dropped", "out[e] = bf16_to_f64(v[e]) * v_scale;", "out[e] = bf16_to_f64(v[e]);", 0),
 ]
 
 

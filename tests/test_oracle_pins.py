@@ -399,3 +399,83 @@ def test_workload_generators_are_seeded():
     s = W.prefill_inputs(W.GA_PREFILL, L=8)["sink"]
     assert torch.isinf(s[7::8]).all() and torch.isfinite(s[0::8]).all()
     assert float(s[torch.isfinite(s)].min()) >= 0 and float(s[torch.isfinite(s)].max()) <= 6
+
+
+# ----------------------------------------------------------------------------------------------
+# partial rotary embedding and the value scale ("MiMo-V2-Flash 模型架构深度拆解" CH3.5, CH10.3,
+# CH10.5; "MiMo-V2-Flash 架构 QA" Q2.7)
+# ----------------------------------------------------------------------------------------------
+
+COS1, SIN1 = 0.5403023058681398, 0.8414709848078965  # cos(1 rad), sin(1 rad)
+
+
+def unit_rows(d, dims):
+    """One bf16 row of d dims per entry of dims, 1.0 in that dim."""
+    x = torch.zeros(len(dims), 1, d, dtype=torch.bfloat16)
+    for r, c in enumerate(dims):
+        x[r, 0, c] = 1.0
+    return x
+
+
+def test_rope_position_zero_is_identity():
+    g = torch.Generator().manual_seed(11)
+    x = rand_bf16((5, 3, 192), g)
+    for theta in (1e4, 5e6):
+        y = oracle.rope(x, np.zeros(5, np.int64), theta)
+        assert torch.equal(y, x.double())
+
+
+def test_rope_closed_form_angles():
+    # pair 0 turns at frequency 1: position 1 -> 1 rad; e_0 -> (cos, sin), e_32 -> (-sin, cos)
+    y = oracle.rope(unit_rows(192, [0, 32]), np.array([1, 1]), 1e4)[:, 0]
+    assert abs(y[0, 0] - COS1) < 1e-15 and abs(y[0, 32] - SIN1) < 1e-15
+    assert abs(y[1, 0] + SIN1) < 1e-15 and abs(y[1, 32] - COS1) < 1e-15
+    # pair 16 of 32 turns at theta^(-1/2): 0.01 for theta 1e4, so position 100 -> 1 rad
+    y = oracle.rope(unit_rows(192, [16]), np.array([100]), 1e4)[0, 0]
+    assert abs(y[16] - COS1) < 1e-13 and abs(y[48] - SIN1) < 1e-13
+    # GA theta 5e6: pair 16 turns at 1/sqrt(5e6) = 1/2236.0679774997896
+    y = oracle.rope(unit_rows(192, [16]), np.array([2236]), 5e6)[0, 0]
+    a = 2236 / 2236.0679774997896
+    assert abs(y[16] - math.cos(a)) < 1e-13 and abs(y[48] - math.sin(a)) < 1e-13
+    # last pair (31) at 1e4^(-62/64) = 10^(-3.875)
+    y = oracle.rope(unit_rows(192, [31]), np.array([7499]), 1e4)[0, 0]
+    a = 7499 * 10 ** -3.875
+    assert abs(y[31] - math.cos(a)) < 1e-12 and abs(y[63] - math.sin(a)) < 1e-12
+    # nothing else moves
+    mask = torch.ones(192, dtype=torch.bool)
+    mask[[31, 63]] = False
+    assert torch.all(y[mask] == 0)
+
+
+@pytest.mark.parametrize("theta", [1e4, 5e6])
+def test_rope_rotation_invariants(theta):
+    g = torch.Generator().manual_seed(12)
+    n = 64
+    q = rand_bf16((n, 4, 192), g)
+    k = rand_bf16((n, 4, 192), g)
+    m = torch.randint(0, 262144, (n,), generator=g).numpy()
+    s = torch.randint(0, 4096, (n,), generator=g).numpy()
+    yq = oracle.rope(q, m, theta)
+    # the no-pe dims pass unchanged
+    assert torch.equal(yq[..., 64:], q.double()[..., 64:])
+    # each pair (i, i + 32) keeps its length
+    xd = q.double()
+    n_in = xd[..., :32] ** 2 + xd[..., 32:64] ** 2
+    n_out = yq[..., :32] ** 2 + yq[..., 32:64] ** 2
+    assert torch.allclose(n_out, n_in, rtol=1e-12, atol=1e-12)
+    # relative position: <R(m) q, R(n) k> depends on m - n only
+    nk = torch.randint(0, 262144, (n,), generator=g).numpy()
+    d1 = (yq[..., :64] * oracle.rope(k, nk, theta)[..., :64]).sum(-1)
+    d2 = (oracle.rope(q, m + s, theta)[..., :64] * oracle.rope(k, nk + s, theta)[..., :64]).sum(-1)
+    assert torch.allclose(d1, d2, rtol=1e-9, atol=1e-9)
+    # and it is not position-free: a shifted query alone changes the score
+    d3 = (oracle.rope(q, m + 1, theta)[..., :64] * oracle.rope(k, nk, theta)[..., :64]).sum(-1)
+    assert (d3 - d1).abs().max() > 1e-3
+
+
+def test_vscale_multiplies_every_element():
+    g = torch.Generator().manual_seed(13)
+    v = rand_bf16((3, 7, 2, 128), g)
+    y = oracle.vscale(v, 0.707)
+    assert y.shape == v.shape
+    assert torch.equal(y, v.double() * 0.707)
