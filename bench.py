@@ -6,7 +6,8 @@
 Headline workload (one "step" = one call over one batch of synthetic input): SWA sink-attention
 prefill at model width, B=2, L=32768, 64 Q / 8 KV heads, d_qk=192, d_v=128, W=128. Metric:
 attention TFLOP/s counting only the band-limited (visible) pairs at 640 FLOP per (row, head,
-key), with its roofline fraction. The other workloads (GA prefill, GA and SWA decode, the hybrid
+key), with its roofline fraction. The other workloads (GA prefill, GA chunked prefill, the fused
+RoPE + value-scale pass over the headline Q/K/V, GA and SWA decode, the hybrid
 speculative-verify step) are measured after it and reported under "secondary".
 
 With N > 1 (torchrun) every rank runs the same per-GPU workload on its own GPU (independent
@@ -195,6 +196,37 @@ class DecodeRunner:
                 delattr(self, k)
 
 
+class RopeRunner:
+    """The fused partial-RoPE + value-scale pass (in place) over a prefill workload's Q, K, V:
+    the step the attention module runs just before the attention core."""
+
+    ROPE_DIM = 64
+
+    def __init__(self, w, dev, theta):
+        import global_attention_sink_softmax_b200 as sa
+        self.sa, self.w, self.theta = sa, w, theta
+        self.d = W.prefill_inputs(w, device=dev)
+        ntok = w.B * w.L
+        # read + write of the rotary part of every Q / K head and of all of V, bf16
+        self.bytes = 2 * ntok * ((w.Hq + w.Hkv) * self.ROPE_DIM * 2 + w.Hkv * w.dv * 2)
+        # 6 FLOP per rotated pair, 1 per scaled value
+        self.flops = ntok * ((w.Hq + w.Hkv) * (self.ROPE_DIM // 2) * 6 + w.Hkv * w.dv)
+        self.launches = 1
+        self.kernel = "rope_qkv_kernel"
+        self.workload = "rope_vscale_" + w.name
+        self.config = dict(B=w.B, L=w.L, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
+                           rope_dim=self.ROPE_DIM, theta=theta, v_scale=sa.V_SCALE,
+                           in_place=True)
+
+    def step(self):
+        d = self.d
+        self.sa.sinkattn_rope_qkv(d["q"], d["k"], d["v"], theta=self.theta)
+
+    def release(self):
+        if hasattr(self, "d"):
+            del self.d
+
+
 class HybridRunner:
     """One speculative-verify step of the hybrid stack: every layer's decode call in order."""
 
@@ -370,7 +402,8 @@ def measured_traffic(kernel):
              "decode_umma_kernel": ["common.cuh", "decode_kernels.cuh",
                                     "decode_tma_kernels.cuh", "decode_umma_kernels.cuh"],
              "decode_ring_kernel": ["common.cuh", "decode_kernels.cuh",
-                                    "decode_ring_kernels.cuh"]}[kernel]
+                                    "decode_ring_kernels.cuh"],
+             "rope_qkv_kernel": ["common.cuh", "rope_kernels.cuh"]}[kernel]
     m = hashlib.sha256()
     for f in files:
         m.update(open(os.path.join(csrc, f), "rb").read())
@@ -499,7 +532,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default=None,
                     help="run one workload only: swa_prefill, ga_prefill, ga_chunk_prefill, "
-                         "ga_decode, swa_decode, hybrid")
+                         "ga_decode, swa_decode, hybrid, rope")
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--ref-L", type=int, default=0, help="reference arm: shorter sequences (tests)")
     ap.add_argument("--small", action="store_true",
@@ -586,6 +619,8 @@ def main():
             jobs.append(("ga_prefill", lambda: PrefillRunner(ga_w, dev), None))
         if only in (None, "ga_chunk_prefill"):
             jobs.append(("ga_chunk_prefill", lambda: PrefillRunner(gac_w, dev), None))
+        if only in (None, "rope"):
+            jobs.append(("rope_qkv", lambda: RopeRunner(swa_w, dev, 1e4), None))
         if only in (None, "ga_decode"):
             jobs.append(("ga_decode", lambda: DecodeRunner(gad_w, dev), None))
         if only in (None, "swa_decode"):
@@ -604,7 +639,8 @@ def main():
             with ClockSampler(local) as clk:
                 ms = measure(r, steps, max(3, args.warmup), flush, world)
             ms_step = ms / steps
-            rl = roofline(r, ms_step, peaks, peak_src)
+            rl = roofline(r, ms_step, peaks, peak_src,
+                          bound="hbm" if isinstance(r, RopeRunner) else None)
             entry = {"workload": r.workload, "config": r.config, "ms_per_step": round(ms_step, 4),
                      "tflops": round(r.flops / (ms_step * 1e-3) / 1e12, 3),
                      "gbs": round(r.bytes / (ms_step * 1e-3) / 1e9, 2), "roofline": rl,

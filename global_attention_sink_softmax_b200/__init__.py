@@ -26,17 +26,20 @@ __all__ = [
     "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_prefill_chunk", "sinkattn_decode",
     "sinkattn_decode_workspace_size", "sinkattn_kv_commit", "sinkattn_take_device_error",
     "sinkattn_status_string", "sinkattn_version", "EXPORTED_SYMBOLS",
-    "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES",
+    "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES", "sinkattn_rope_qkv",
+    "ROPE_THETA_GA", "ROPE_THETA_SWA", "V_SCALE",
 ]
 
 KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
 DQ, DV = 192, 128
+# The model's rotary thetas (GA / SWA layers), rotated width and value scale.
+ROPE_THETA_GA, ROPE_THETA_SWA, ROPE_DIM, V_SCALE = 5_000_000.0, 10_000.0, 64, 0.707
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libsinkattn.so")
 EXPORTED_SYMBOLS = [
     "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_prefill_chunk",
     "sinkattn_decode_workspace_size", "sinkattn_decode", "sinkattn_kv_commit", "sinkattn_status_string", "sinkattn_version",
-    "sinkattn_take_device_error", "sinkattn_decode_noalloc",
+    "sinkattn_take_device_error", "sinkattn_decode_noalloc", "sinkattn_rope_qkv",
 ]
 # Size of the library's own split-KV workspace used by sinkattn_decode_noalloc.
 NOALLOC_WORKSPACE_BYTES = 16 << 20
@@ -60,6 +63,16 @@ class PrefillArgs(ctypes.Structure):
                 ("k_sb", _I64), ("k_sl", _I64), ("k_sh", _I64),
                 ("v_sb", _I64), ("v_sl", _I64), ("v_sh", _I64),
                 ("o_sb", _I64), ("o_sl", _I64), ("o_sh", _I64)]
+
+
+class RopeArgs(ctypes.Structure):
+    _fields_ = [("q", _P), ("k", _P), ("v", _P), ("pos_base", _P), ("pos0", _I64),
+                ("B", _I32), ("L", _I32), ("Hq", _I32), ("Hkv", _I32), ("dq", _I32),
+                ("dv", _I32), ("rope_dim", _I32), ("theta", ctypes.c_double),
+                ("v_scale", _F32),
+                ("q_sb", _I64), ("q_sl", _I64), ("q_sh", _I64),
+                ("k_sb", _I64), ("k_sl", _I64), ("k_sh", _I64),
+                ("v_sb", _I64), ("v_sl", _I64), ("v_sh", _I64)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -111,6 +124,8 @@ def lib() -> ctypes.CDLL:
             L.sinkattn_version.restype = ctypes.c_int
             L.sinkattn_take_device_error.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
             L.sinkattn_take_device_error.restype = ctypes.c_int
+            L.sinkattn_rope_qkv.argtypes = [ctypes.POINTER(RopeArgs), _P]
+            L.sinkattn_rope_qkv.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -349,6 +364,45 @@ def sinkattn_kv_commit(kind, k_new, v_new, n_accept, k_cache, v_cache, *, ring_h
                      ring_len, ctx_len, max_ctx, page_table, None, num_pages, None, None)
     st = lib().sinkattn_kv_commit(ctypes.byref(a), _ptr(n_accept), _stream(stream))
     _raise(st, "sinkattn_kv_commit")
+
+
+def sinkattn_rope_qkv(q=None, k=None, v=None, *, theta, rope_dim=ROPE_DIM, v_scale=V_SCALE,
+                      pos0=0, pos_base=None, stream=None):
+    """Partial RoPE on the first rope_dim dims of q [B,L,Hq,dq] and k [B,L,Hkv,dq], and v
+    [B,L,Hkv,dv] times v_scale, all in place (any of the three may be None). Token l of
+    sequence b sits at position pos0 + pos_base[b] + l (pos_base: CUDA int32 [B] or None).
+    theta: ROPE_THETA_GA or ROPE_THETA_SWA for the pages' model."""
+    given = [t for t in (q, k, v) if t is not None]
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        if t is not None:
+            _check_bf16(n, t)
+    _check_vec("pos_base", pos_base, torch.int32)
+    if not given:
+        return
+    B, L = given[0].shape[:2]
+    if any(tuple(t.shape[:2]) != (B, L) for t in given):
+        raise ValueError("q, k and v must share [B, L]")
+    if q is not None and k is not None and q.shape[3] != k.shape[3]:
+        raise ValueError("q and k must share the head dim")
+    if k is not None and v is not None and k.shape[2] != v.shape[2]:
+        raise ValueError("k and v must share the KV head count")
+    if pos_base is not None and pos_base.numel() != B:
+        raise ValueError("pos_base must have B entries")
+    a = RopeArgs()
+    a.B, a.L = B, L
+    a.Hq = q.shape[2] if q is not None else 0
+    a.Hkv = k.shape[2] if k is not None else (v.shape[2] if v is not None else 0)
+    a.dq = (q if q is not None else k).shape[3] if (q is not None or k is not None) else 0
+    a.dv = v.shape[3] if v is not None else 0
+    a.rope_dim, a.theta, a.v_scale = int(rope_dim), float(theta), float(v_scale)
+    a.pos0, a.pos_base = int(pos0), _ptr(pos_base)
+    if q is not None:
+        a.q, a.q_sb, a.q_sl, a.q_sh = _ptr(q), q.stride(0), q.stride(1), q.stride(2)
+    if k is not None:
+        a.k, a.k_sb, a.k_sl, a.k_sh = _ptr(k), k.stride(0), k.stride(1), k.stride(2)
+    if v is not None:
+        a.v, a.v_sb, a.v_sl, a.v_sh = _ptr(v), v.stride(0), v.stride(1), v.stride(2)
+    _raise(lib().sinkattn_rope_qkv(ctypes.byref(a), _stream(stream)), "sinkattn_rope_qkv")
 
 
 def sinkattn_take_device_error() -> int:

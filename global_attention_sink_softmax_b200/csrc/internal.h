@@ -109,6 +109,20 @@ struct CommitParams {
 
 cudaError_t launch_commit(const CommitParams &p, cudaStream_t stream);
 
+// Fused partial RoPE + value scale, in place (rope_kernels.cuh).
+constexpr int kRopeMaxHalf = 64; // rope_dim <= 128
+struct RopeParams {
+    uint16_t *q, *k, *v; // any may be null (skipped)
+    const int32_t *pos_base;
+    int64_t pos0;
+    int B, L, Hq, Hkv, half, dv;
+    float v_scale;
+    int64_t q_sb, q_sl, q_sh, k_sb, k_sl, k_sh, v_sb, v_sl, v_sh;
+    double inv_freq[kRopeMaxHalf]; // w_i = theta^(-2i/rope_dim)
+};
+
+cudaError_t launch_rope_qkv(const RopeParams &p, cudaStream_t stream);
+
 cudaError_t read_and_clear_device_error(uint32_t *flag);
 
 } // namespace sinkattn

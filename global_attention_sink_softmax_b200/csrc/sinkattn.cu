@@ -14,6 +14,7 @@
 #include "decode_ring_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
+#include "rope_kernels.cuh"
 #include "swa_kernels.cuh"
 
 namespace {
@@ -666,6 +667,73 @@ int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, v
     p.num_pages = a->num_pages;
     p.n_accept = n_accept;
     const cudaError_t e = launch_commit(p, (cudaStream_t)stream);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+int sinkattn_rope_qkv(const sinkattn_rope_args *a, void *stream)
+{
+    if (!a || a->B < 0 || a->L < 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (!(a->theta > 0.0) || !isfinite(a->theta) || !isfinite(a->v_scale))
+        return SINKATTN_ERR_INVALID_ARG;
+    if ((a->q && a->Hq <= 0) || ((a->k || a->v) && a->Hkv <= 0))
+        return SINKATTN_ERR_INVALID_ARG;
+    if ((a->q || a->k) && (a->rope_dim < 16 || a->rope_dim > 2 * kRopeMaxHalf ||
+                           a->rope_dim % 16 != 0 || a->dq < a->rope_dim || a->dq % 8 != 0))
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (a->v && (a->dv <= 0 || a->dv % 16 != 0))
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->L == 0 || (!a->q && !a->k && !a->v))
+        return SINKATTN_OK;
+    const void *ptrs[3] = {a->q, a->k, a->v};
+    const int64_t s[9] = {a->q_sb, a->q_sl, a->q_sh, a->k_sb, a->k_sl, a->k_sh,
+                          a->v_sb, a->v_sl, a->v_sh};
+    for (int i = 0; i < 3; ++i) {
+        if (!ptrs[i])
+            continue;
+        if (!aligned16(ptrs[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+        for (int j = 0; j < 3; ++j) {
+            if (s[3 * i + j] <= 0)
+                return SINKATTN_ERR_INVALID_ARG;
+            if (!stride_ok(s[3 * i + j]))
+                return SINKATTN_ERR_ALIGNMENT;
+        }
+    }
+    {
+        // 32-byte units per token; the kernel indexes TOK tokens' worth of them with an int
+        const int64_t nc = (a->q || a->k) ? a->rope_dim / 16 : 0;
+        const int64_t per_tok = (a->q ? (int64_t)a->Hq * nc : 0) +
+                                (a->k ? (int64_t)a->Hkv * nc : 0) +
+                                (a->v ? (int64_t)a->Hkv * (a->dv / 16) : 0);
+        if (per_tok * 8 > 0x3fffffff)
+            return SINKATTN_ERR_UNSUPPORTED;
+    }
+    RopeParams p;
+    p.q = static_cast<uint16_t *>(a->q);
+    p.k = static_cast<uint16_t *>(a->k);
+    p.v = static_cast<uint16_t *>(a->v);
+    p.pos_base = a->pos_base;
+    p.pos0 = a->pos0;
+    p.B = a->B;
+    p.L = a->L;
+    p.Hq = a->Hq;
+    p.Hkv = a->Hkv;
+    p.half = (a->q || a->k) ? a->rope_dim / 2 : 8;
+    p.dv = a->dv;
+    p.v_scale = a->v_scale;
+    p.q_sb = a->q_sb;
+    p.q_sl = a->q_sl;
+    p.q_sh = a->q_sh;
+    p.k_sb = a->k_sb;
+    p.k_sl = a->k_sl;
+    p.k_sh = a->k_sh;
+    p.v_sb = a->v_sb;
+    p.v_sl = a->v_sl;
+    p.v_sh = a->v_sh;
+    for (int i = 0; i < kRopeMaxHalf; ++i)
+        p.inv_freq[i] = i < p.half ? pow(a->theta, -2.0 * i / (2.0 * p.half)) : 0.0;
+    const cudaError_t e = launch_rope_qkv(p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

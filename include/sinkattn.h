@@ -229,6 +229,47 @@ int sinkattn_decode_noalloc(const sinkattn_decode_args *args, void *stream);
  * ------------------------------------------------------------------------------------------- */
 int sinkattn_kv_commit(const sinkattn_decode_args *args, const int32_t *n_accept, void *stream);
 
+
+/* ---------------------------------------------------------------------------------------------
+ * Partial rotary position embedding and the value scale, fused into one in-place pass: the
+ * steps the attention module runs between the Q/K/V projection and attention ("MiMo-V2-Flash
+ * 模型架构深度拆解" CH10.3: V times v_scale = 0.707, then RoPE on the first 64 of the 192 Q/K
+ * dims; CH3.5 and CH8.1: partial_rotary_factor 0.334, rope_theta 5,000,000 on GA layers and
+ * swa_rope_theta 10,000 on SWA layers; "MiMo-V2-Flash 架构 QA" Q2.7: angle m * theta^(-2i/d)).
+ *
+ * Token l of sequence b sits at position m = pos0 + pos_base[b] + l (pos_base NULL: 0), so a
+ * whole prompt uses pos0 = 0, a chunk after P cached tokens pos0 = P, and decode's new tokens
+ * pos_base = the tokens each sequence has seen. Dimension pair i (0 <= i < rope_dim/2) of
+ * every Q and K head is dims (i, i + rope_dim/2) and turns by m * theta^(-2i/rope_dim):
+ *     y_i = x_i cos - x_{i+rope_dim/2} sin,   y_{i+rope_dim/2} = x_{i+rope_dim/2} cos + x_i sin
+ * (the pages leave the pairing open; this is the "rotate half" arrangement). Dims rope_dim..dq-1
+ * are neither read nor written. Every V element is multiplied by v_scale. Results are rounded
+ * once to bf16 (nearest even); angles are reduced in fp64, so large positions stay exact.
+ *
+ *   q [B, L, Hq, dq], k [B, L, Hkv, dq], v [B, L, Hkv, dv]: bf16, modified in place; any of the
+ *       three may be NULL (skipped). Strides as for prefill; rows must not overlap.
+ *   pos_base: device int32 [B] or NULL.
+ *   rope_dim: a multiple of 16 in 16..128, <= dq (64 for the pages' model); dq a multiple of 8;
+ *   dv a multiple of 16.  theta > 0 and finite; v_scale finite.
+ * Errors: INVALID_ARG (negative sizes, theta <= 0, non-finite values, non-positive strides,
+ * Hq / Hkv <= 0 for a given tensor), UNSUPPORTED (rope_dim / dq / dv out of range), ALIGNMENT.
+ * ------------------------------------------------------------------------------------------- */
+typedef struct sinkattn_rope_args {
+    void *q;
+    void *k;
+    void *v;
+    const int32_t *pos_base;
+    int64_t pos0;
+    int32_t B, L, Hq, Hkv, dq, dv, rope_dim;
+    double theta;
+    float v_scale;
+    int64_t q_sb, q_sl, q_sh;
+    int64_t k_sb, k_sl, k_sh;
+    int64_t v_sb, v_sl, v_sh;
+} sinkattn_rope_args;
+
+int sinkattn_rope_qkv(const sinkattn_rope_args *args, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *sinkattn_status_string(int status);
 

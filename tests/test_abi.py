@@ -59,6 +59,7 @@ C_LAYOUT = r"""
 int main(void) {
   printf("sinkattn_prefill_args %zu\n", sizeof(sinkattn_prefill_args));
   printf("sinkattn_decode_args %zu\n", sizeof(sinkattn_decode_args));
+  printf("sinkattn_rope_args %zu\n", sizeof(sinkattn_rope_args));
   %FIELDS%
   return 0;
 }
@@ -67,7 +68,9 @@ int main(void) {
 
 def test_struct_layout_matches_header(tmp_path):
     lines = []
-    for cname, py in (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs)):
+    structs = (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs),
+               ("sinkattn_rope_args", sa.RopeArgs))
+    for cname, py in structs:
         for f, _ in py._fields_:
             lines.append(f"F({cname}, {f})")
     src = C_LAYOUT.replace("%FIELDS%", "\n  ".join(lines))
@@ -78,7 +81,8 @@ def test_struct_layout_matches_header(tmp_path):
     got = dict(l.rsplit(" ", 1) for l in subprocess.check_output([str(exe)], text=True).splitlines())
     assert int(got["sinkattn_prefill_args"]) == ctypes.sizeof(sa.PrefillArgs)
     assert int(got["sinkattn_decode_args"]) == ctypes.sizeof(sa.DecodeArgs)
-    for cname, py in (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs)):
+    assert int(got["sinkattn_rope_args"]) == ctypes.sizeof(sa.RopeArgs)
+    for cname, py in structs:
         for f, _ in py._fields_:
             assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
 
@@ -188,6 +192,44 @@ def test_commit_rejects_bad_arguments(L):
     assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(dv=64)), ctypes.c_void_p(0x60000), None) == 2
     assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(kind=0)), ctypes.c_void_p(0x60000), None) == 1
     assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(B=0)), None, None) == 0
+
+
+def _rope_args(**kw):
+    a = sa.RopeArgs()
+    a.q, a.k, a.v = 0x10000, 0x20000, 0x30000
+    a.B, a.L, a.Hq, a.Hkv, a.dq, a.dv, a.rope_dim = 2, 64, 64, 8, 192, 128, 64
+    a.theta, a.v_scale = 1e4, 0.707
+    for f, d, h in (("q", 192, 64), ("k", 192, 8), ("v", 128, 8)):
+        setattr(a, f + "_sh", d)
+        setattr(a, f + "_sl", d * h)
+        setattr(a, f + "_sb", d * h * 64)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(B=-1), 1), (dict(L=-3), 1), (dict(theta=0.0), 1), (dict(theta=-1e4), 1),
+    (dict(theta=float("inf")), 1), (dict(theta=float("nan")), 1), (dict(v_scale=float("nan")), 1),
+    (dict(Hq=0), 1), (dict(Hkv=0), 1), (dict(q_sl=0), 1), (dict(v_sh=-128), 1),
+    (dict(rope_dim=8), 2), (dict(rope_dim=72), 2), (dict(rope_dim=144), 2), (dict(dq=48), 2),
+    (dict(dq=196), 2), (dict(dv=120), 2),
+    (dict(q=0x10004), 3), (dict(v=0x30002), 3), (dict(k_sl=100), 3),
+])
+def test_rope_rejects_bad_arguments(L, kw, status):
+    assert L.sinkattn_rope_qkv(ctypes.byref(_rope_args(**kw)), None) == status
+
+
+def test_rope_empty_and_partial_calls_need_no_device(L):
+    """Empty work, or no tensor at all, returns OK before any CUDA call; a tensor that is not
+    given is not checked (its head count and strides may be anything)."""
+    assert L.sinkattn_rope_qkv(ctypes.byref(_rope_args(B=0)), None) == 0
+    assert L.sinkattn_rope_qkv(ctypes.byref(_rope_args(L=0)), None) == 0
+    assert L.sinkattn_rope_qkv(ctypes.byref(_rope_args(q=None, k=None, v=None)), None) == 0
+    assert L.sinkattn_rope_qkv(ctypes.byref(_rope_args(B=0, q=None, Hq=0, q_sl=0)), None) == 0
+    assert L.sinkattn_rope_qkv(ctypes.byref(_rope_args(B=0, v=None, dv=120)), None) == 0
+    assert L.sinkattn_rope_qkv(ctypes.byref(_rope_args(B=0, q=None, k=None, rope_dim=0)), None) == 0
+    assert L.sinkattn_rope_qkv(None, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
