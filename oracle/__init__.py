@@ -69,6 +69,12 @@ def _load():
             lib.sinkattn_oracle_rope.restype = i32
             lib.sinkattn_oracle_vscale.argtypes = [P, i64, f64, P]
             lib.sinkattn_oracle_vscale.restype = None
+            lib.sinkattn_oracle_fp8_encode.argtypes = [P, i64, ctypes.c_float, P]
+            lib.sinkattn_oracle_fp8_encode.restype = None
+            lib.sinkattn_oracle_fp8_decode.argtypes = [P, i64, P]
+            lib.sinkattn_oracle_fp8_decode.restype = None
+            lib.sinkattn_oracle_e4m3_encode.argtypes = [ctypes.c_float]
+            lib.sinkattn_oracle_e4m3_encode.restype = ctypes.c_uint8
             _lib = lib
     return _lib
 
@@ -251,3 +257,52 @@ def vscale(v, v_scale):
     out = np.zeros(vb.size, np.float64)
     lib.sinkattn_oracle_vscale(_ptr(vb), vb.size, float(v_scale), _ptr(out))
     return torch.from_numpy(out.reshape(v.shape))
+
+
+def fp8_encode(x, scale):
+    """FP8 (E4M3) cache codes of a bf16 tensor: encode(x / scale), the division in fp32.
+    Returns a torch.uint8 tensor of x's shape."""
+    lib = _load()
+    xb = _bits(x)
+    codes = np.zeros(xb.size, np.uint8)
+    lib.sinkattn_oracle_fp8_encode(_ptr(xb), xb.size, float(np.float32(scale)), _ptr(codes))
+    return torch.from_numpy(codes.reshape(x.shape))
+
+
+def e4m3_encode_f32(y):
+    """E4M3 code of each fp32 value in y (numpy or torch), as a uint8 numpy array."""
+    lib = _load()
+    ya = np.asarray(y.cpu() if isinstance(y, torch.Tensor) else y, dtype=np.float32).reshape(-1)
+    return np.array([lib.sinkattn_oracle_e4m3_encode(float(v)) for v in ya], np.uint8)
+
+
+def fp8_decode(codes):
+    """E4M3 values (without the scale) of a uint8 code tensor, float64."""
+    lib = _load()
+    c = np.ascontiguousarray(np.asarray(codes.cpu() if isinstance(codes, torch.Tensor) else codes,
+                                        dtype=np.uint8))
+    out = np.zeros(c.size, np.float64)
+    lib.sinkattn_oracle_fp8_decode(_ptr(c), c.size, _ptr(out))
+    return torch.from_numpy(out.reshape(c.shape))
+
+
+def decode_fp8(kind, q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, sink, scale, window=0,
+               **kw):
+    """Decode against an FP8 (E4M3) cache: cached token values are e(code) * scale.
+
+    The T new tokens are quantised as the cache will store them (fp8_encode), so every key is
+    e(c_k) * k_scale and every value e(c_v) * v_scale. By linearity
+        a_j = scale * <q, k_scale e(c_j)> = (scale * k_scale) * <q, e(c_j)>,
+        O   = sum_j w_j v_scale e(c_vj) = v_scale * sum_j w_j e(c_vj),
+    and e(c) is exact in bf16 (4 significant bits, exponents -9..8), so this is the bf16 decode
+    above on the E4M3 values with the scale scale * k_scale, and O times v_scale. LSE is the
+    one of those logits. Returns (o, lse, wsink) as decode()."""
+    def values_bf16(codes):
+        return fp8_decode(codes).to(torch.bfloat16)
+
+    kn = values_bf16(fp8_encode(k_new, k_scale))
+    vn = values_bf16(fp8_encode(v_new, v_scale))
+    kc, vc = values_bf16(k_codes), values_bf16(v_codes)
+    f32 = lambda s: float(np.float32(s))
+    o, lse, ws = decode(kind, q, kn, vn, kc, vc, sink, scale * f32(k_scale), window, **kw)
+    return o * f32(v_scale), lse, ws

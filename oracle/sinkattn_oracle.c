@@ -432,3 +432,62 @@ void sinkattn_oracle_vscale(const uint16_t *v, int64_t n, double v_scale, double
     for (int64_t e = 0; e < n; ++e)
         out[e] = bf16_to_f64(v[e]) * v_scale;
 }
+
+/*
+ * FP8 KV cache codes. The pages size a KV slot at one byte ([NOTES] §2 memory arithmetic) and
+ * speak of FP8 inference ([BLOG]); they name no format or scaling. Readings:
+ *   - the E4M3 "fn" format: 1 sign, 4 exponent bits (bias 7), 3 mantissa bits, no infinities,
+ *     S.1111.111 is NaN; largest finite 448 = 1.75 * 2^8, smallest normal 2^-6, subnormals
+ *     k * 2^-9;
+ *   - one fp32 scale per cache tensor (K and V separately): a stored code c means e(c) * scale;
+ *   - storing x: y = x / scale in fp32 (correctly rounded), then the nearest E4M3 value, ties
+ *     to the even code, saturating to +-448 (NaN stays NaN).
+ */
+double sinkattn_oracle_e4m3_value(uint8_t c)
+{
+    const int s = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7)
+        return NAN;
+    const double v = (e == 0) ? ldexp((double)m, -9)        /* subnormal: m/8 * 2^-6 */
+                              : ldexp((double)(8 + m), e - 10); /* (1 + m/8) * 2^(e-7) */
+    return s ? -v : v;
+}
+
+uint8_t sinkattn_oracle_e4m3_encode(float y)
+{
+    if (isnan(y))
+        return 0x7f;
+    const uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    const double a = fabs((double)y);
+    if (a >= 448.0)
+        return sign | 0x7e;
+    /* the nearest of the 127 non-negative finite values; on a tie the even code (its last
+       bit is the mantissa's last bit) */
+    int best = 0;
+    double best_d = INFINITY;
+    for (int c = 0; c <= 0x7e; ++c) {
+        const double d = fabs(sinkattn_oracle_e4m3_value((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = c;
+            best_d = d;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* codes[i] = encode(x[i] / scale), the division in fp32. x: bf16 bits. */
+void sinkattn_oracle_fp8_encode(const uint16_t *x, int64_t n, float scale, uint8_t *codes)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        const float xi = (float)bf16_to_f64(x[i]);
+        const float y = xi / scale;
+        codes[i] = sinkattn_oracle_e4m3_encode(y);
+    }
+}
+
+/* out[i] = e(codes[i]) (the scale is applied by the caller). */
+void sinkattn_oracle_fp8_decode(const uint8_t *codes, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = sinkattn_oracle_e4m3_value(codes[i]);
+}

@@ -45,6 +45,12 @@ MUTANTS = [
     ("rope also turns the no-pe dims", "for (int i = 0; i < half; ++i) {\n                const double w",
      "for (int i = 0; i < d / 2; ++i) {\n                const double w", 0),
     ("value scale dropped", "out[e] = bf16_to_f64(v[e]) * v_scale;", "out[e] = bf16_to_f64(v[e]);", 0),
+    ("e4m3 ties toward zero", "(d == best_d && (c & 1) == 0)", "(d == best_d && 0)", 0),
+    ("e4m3 exponent bias 8", "ldexp((double)(8 + m), e - 10)", "ldexp((double)(8 + m), e - 11)", 0),
+    ("e4m3 subnormal step 2^-10", "ldexp((double)m, -9)", "ldexp((double)m, -10)", 0),
+    ("e4m3 without saturation", "if (a >= 448.0)\n        return sign | 0x7e;",
+     "if (a >= 464.0)\n        return sign | 0x7f;", 0),
+    ("fp8 encode multiplies by the scale", "const float y = xi / scale;", "const float y = xi * scale;", 0),
 ]
 
 

@@ -479,3 +479,106 @@ def test_vscale_multiplies_every_element():
     y = oracle.vscale(v, 0.707)
     assert y.shape == v.shape
     assert torch.equal(y, v.double() * 0.707)
+
+
+# ----------------------------------------------------------------------------------------------
+# FP8 (E4M3) cache codes and decode against an FP8 cache
+# ----------------------------------------------------------------------------------------------
+
+def test_e4m3_values_equal_the_library_for_every_code():
+    codes = torch.arange(256, dtype=torch.uint8)
+    ours = oracle.fp8_decode(codes)
+    lib = codes.view(torch.float8_e4m3fn).to(torch.float64)
+    nan = torch.isnan(lib)
+    assert torch.equal(torch.isnan(ours), nan) and nan.sum() == 2  # 0x7f and 0xff
+    assert torch.equal(ours[~nan], lib[~nan])
+
+
+def test_e4m3_closed_forms():
+    v = oracle.fp8_decode(torch.tensor([0x00, 0x01, 0x07, 0x08, 0x38, 0xb8, 0x7e, 0xfe, 0x57, 0x58],
+                                       dtype=torch.uint8)).tolist()
+    assert v == [0.0, 2.0 ** -9, 7 * 2.0 ** -9, 2.0 ** -6, 1.0, -1.0, 448.0, -448.0, 15.0, 16.0]
+
+
+def test_e4m3_encode_rounds_to_nearest_even_and_saturates():
+    enc = lambda xs: oracle.e4m3_encode_f32(np.array(xs, np.float32)).tolist()
+    # ties go to the even code: 1.0625 between 1 (0x38) and 1.125 (0x39); 1.1875 between 1.125
+    # and 1.25 (0x3a); 2^-10 between 0 and 2^-9; 3 * 2^-10 between 2^-9 and 2^-8 (0x02);
+    # 15.5 between 15 (0x57) and 16 (0x58), across a binade
+    assert enc([1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, 15.5]) == [0x38, 0x3a, 0x00, 0x02, 0x58]
+    assert enc([1.0626, 1.1874, -1.0626]) == [0x39, 0x39, 0xb9]
+    # beyond the largest finite value: +-448 (satfinite), NaN stays NaN
+    assert enc([448.0, 449.0, 464.0, 1e30, float("inf"), -500.0, float("-inf")]) == \
+        [0x7e, 0x7e, 0x7e, 0x7e, 0x7e, 0xfe, 0xfe]
+    assert enc([float("nan")]) == [0x7f]
+    # every finite code round-trips
+    finite = [c for c in range(256) if c not in (0x7f, 0xff)]
+    vals = oracle.fp8_decode(torch.tensor(finite, dtype=torch.uint8)).numpy().astype(np.float32)
+    assert oracle.e4m3_encode_f32(vals).tolist() == finite
+
+
+def test_e4m3_encode_equals_the_library_cast_in_range():
+    g = torch.Generator().manual_seed(21)
+    mag = torch.exp2(torch.rand(20000, generator=g) * 20 - 12)  # 2^-12 .. 2^8
+    y = (mag * torch.where(torch.rand(20000, generator=g) < 0.5, -1.0, 1.0)).float()
+    y = y.clamp(-448.0, 448.0)
+    lib = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.e4m3_encode_f32(y), lib)
+
+
+def test_fp8_encode_divides_in_fp32():
+    g = torch.Generator().manual_seed(22)
+    x = rand_bf16((3, 5, 64), g)
+    for s in (0.013, 0.5, 1 / 3):
+        codes = oracle.fp8_encode(x, s)
+        y = x.float().numpy() / np.float32(s)  # IEEE fp32 division
+        assert np.array_equal(codes.numpy().reshape(-1), oracle.e4m3_encode_f32(y))
+
+
+def eager_fp8_decode(q, k_new, v_new, kc_codes, vc_codes, ks, vs, ctx, sink, scale, window):
+    """Contiguous-cache FP8 decode written out directly: dequantise (library cast for the new
+    tokens), concatenate, softmax with the sink column (library), drop it."""
+    B, T, Hq, _ = q.shape
+    Hkv = k_new.shape[2]
+    G = Hq // Hkv
+    f32 = lambda s: float(np.float32(s))
+    deq = lambda c, s: c.view(torch.float8_e4m3fn).to(torch.float64) * f32(s)
+    quant = lambda x, s: (x.float() / torch.tensor(s, dtype=torch.float32)).to(torch.float8_e4m3fn).view(torch.uint8)
+    kn, vn = deq(quant(k_new, ks), ks), deq(quant(v_new, vs), vs)
+    kc, vc = deq(kc_codes, ks), deq(vc_codes, vs)
+    o = torch.zeros(B, T, Hq, v_new.shape[3], dtype=torch.float64)
+    lse = torch.zeros(B, T, Hq, dtype=torch.float64)
+    for b in range(B):
+        n = int(ctx[b])
+        K = torch.cat([kc[b, :n], kn[b]], 0)      # [n + T, Hkv, dq], positions -n .. T-1
+        V = torch.cat([vc[b, :n], vn[b]], 0)
+        pos = torch.arange(-n, T)
+        for t in range(T):
+            vis = (pos <= t) & ((pos > t - window) if window > 0 else True)
+            for h in range(Hq):
+                a = scale * (K[vis, h // G] @ q[b, t, h].double())
+                logits = torch.cat([a, torch.tensor([float(sink[h])], dtype=torch.float64)])
+                w = torch.softmax(logits, 0)[:-1]
+                o[b, t, h] = w @ V[vis, h // G]
+                lse[b, t, h] = torch.logsumexp(logits, 0)
+    return o, lse
+
+
+@pytest.mark.parametrize("window", [0, 7])
+def test_decode_fp8_equals_eager_dequantised(window):
+    g = torch.Generator().manual_seed(23)
+    B, T, Hq, Hkv, max_ctx = 2, 3, 4, 2, 24
+    ks, vs = 0.021, 0.017
+    q = rand_bf16((B, T, Hq, 192), g)
+    k_new, v_new = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    lib_codes = lambda x, s: (x.float() / s).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+    kc = lib_codes(torch.randn(B, max_ctx, Hkv, 192, generator=g), ks)
+    vc = lib_codes(torch.randn(B, max_ctx, Hkv, 128, generator=g), vs)
+    ctx = torch.tensor([17, 0], dtype=torch.int32)
+    sink = torch.tensor([0.5, -1.0, float("-inf"), 2.0])
+    scale = 1.0 / math.sqrt(192)
+    o, lse, _ = oracle.decode_fp8(oracle.KV_CONTIG, q, k_new, v_new, kc, vc, ks, vs, sink, scale,
+                                  window, ctx_len=ctx)
+    eo, el = eager_fp8_decode(q, k_new, v_new, kc, vc, ks, vs, ctx, sink, scale, window)
+    assert torch.allclose(o, eo, rtol=0, atol=1e-12)
+    assert torch.allclose(lse, el, rtol=0, atol=1e-12)
