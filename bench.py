@@ -7,7 +7,8 @@ Headline workload (one "step" = one call over one batch of synthetic input): SWA
 prefill at model width, B=2, L=32768, 64 Q / 8 KV heads, d_qk=192, d_v=128, W=128. Metric:
 attention TFLOP/s counting only the band-limited (visible) pairs at 640 FLOP per (row, head,
 key), with its roofline fraction. The other workloads (GA prefill, GA chunked prefill, the fused
-RoPE + value-scale pass over the headline Q/K/V, GA and SWA decode, the hybrid
+RoPE + value-scale pass over the headline Q/K/V, GA decode with a bf16 and with an FP8 cache,
+SWA decode, the hybrid
 speculative-verify step) are measured after it and reported under "secondary".
 
 With N > 1 (torchrun) every rank runs the same per-GPU workload on its own GPU (independent
@@ -84,7 +85,8 @@ def decode_counts(w, d):
         pairs += int(vis.sum()) * w.Hq
     flops = pairs * FLOP_PER_PAIR
     kv_row = w.Hkv * (w.dq + w.dv) * 2
-    nbytes = int(n_used.sum()) * kv_row
+    cache_row = w.Hkv * (w.dq + w.dv) * d["k_cache"].element_size()  # 1 byte for an FP8 cache
+    nbytes = int(n_used.sum()) * cache_row
     nbytes += w.B * T * (kv_row + w.Hq * (w.dq + w.dv) * 2 + w.Hq * 4)
     return flops, nbytes
 
@@ -167,13 +169,18 @@ class DecodeRunner:
             self.kw.update(ctx_len=d["ctx_len"], max_ctx=d["max_ctx"])
         if w.kind == W.KV_PAGED:
             self.kw.update(page_table=d["page_table"])
+        fp8 = "k_scale" in d
         need = sa.sinkattn_decode_workspace_size(w.kind, d["q"], d["k_new"], d["v_new"],
                                                  d["k_cache"], d["v_cache"], **self.kw)
         self.ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         self.launches = 1 if need == 0 else 2
         # the kernel the library dispatches this workload to
+        if fp8:
+            self.kw.update(k_scale=d["k_scale"], v_scale=d["v_scale"])
         rows = w.T * (w.Hq // w.Hkv)
-        if w.kind == W.KV_RING:
+        if fp8:
+            self.kernel = "decode_fp8_kernel"
+        elif w.kind == W.KV_RING:
             self.kernel = "decode_ring_kernel" if rows <= 16 else "decode_split_kernel"
         elif w.kind == W.KV_PAGED and w.page_size % 64 != 0:
             self.kernel = "decode_split_kernel"
@@ -183,6 +190,9 @@ class DecodeRunner:
         self.workload = w.name
         self.config = dict(B=w.B, T=w.T, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
                            window=w.window, cache=["ring", "contiguous", "paged"][w.kind])
+        if fp8:
+            self.config.update(cache_dtype="fp8_e4m3", k_scale=d["k_scale"], v_scale=d["v_scale"])
+            self.workload = w.name + "_fp8"
 
     def step(self):
         d = self.d
@@ -403,7 +413,9 @@ def measured_traffic(kernel):
                                     "decode_tma_kernels.cuh", "decode_umma_kernels.cuh"],
              "decode_ring_kernel": ["common.cuh", "decode_kernels.cuh",
                                     "decode_ring_kernels.cuh"],
-             "rope_qkv_kernel": ["common.cuh", "rope_kernels.cuh"]}[kernel]
+             "rope_qkv_kernel": ["common.cuh", "rope_kernels.cuh"],
+             "decode_fp8_kernel": ["common.cuh", "decode_kernels.cuh",
+                                   "decode_fp8_kernels.cuh"]}[kernel]
     m = hashlib.sha256()
     for f in files:
         m.update(open(os.path.join(csrc, f), "rb").read())
@@ -532,7 +544,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default=None,
                     help="run one workload only: swa_prefill, ga_prefill, ga_chunk_prefill, "
-                         "ga_decode, swa_decode, hybrid, rope")
+                         "ga_decode, ga_decode_fp8, swa_decode, hybrid, rope")
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--ref-L", type=int, default=0, help="reference arm: shorter sequences (tests)")
     ap.add_argument("--small", action="store_true",
@@ -623,6 +635,10 @@ def main():
             jobs.append(("rope_qkv", lambda: RopeRunner(swa_w, dev, 1e4), None))
         if only in (None, "ga_decode"):
             jobs.append(("ga_decode", lambda: DecodeRunner(gad_w, dev), None))
+        if only in (None, "ga_decode_fp8"):
+            jobs.append(("ga_decode_fp8",
+                         lambda: DecodeRunner(gad_w, dev, W.decode_inputs(gad_w, device=dev, fp8=True)),
+                         None))
         if only in (None, "swa_decode"):
             jobs.append(("swa_decode", lambda: DecodeRunner(swad_w, dev), "flush"))
         if only in (None, "hybrid") and not args.small:

@@ -27,10 +27,11 @@ __all__ = [
     "sinkattn_decode_workspace_size", "sinkattn_kv_commit", "sinkattn_take_device_error",
     "sinkattn_status_string", "sinkattn_version", "EXPORTED_SYMBOLS",
     "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES", "sinkattn_rope_qkv",
-    "ROPE_THETA_GA", "ROPE_THETA_SWA", "V_SCALE",
+    "ROPE_THETA_GA", "ROPE_THETA_SWA", "V_SCALE", "KV_BF16", "KV_FP8_E4M3",
 ]
 
 KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
+KV_BF16, KV_FP8_E4M3 = 0, 1  # cache element types; an FP8 cache is a uint8 / float8_e4m3fn tensor
 DQ, DV = 192, 128
 # The model's rotary thetas (GA / SWA layers), rotated width and value scale.
 ROPE_THETA_GA, ROPE_THETA_SWA, ROPE_DIM, V_SCALE = 5_000_000.0, 10_000.0, 64, 0.707
@@ -87,7 +88,8 @@ class DecodeArgs(ctypes.Structure):
                 ("ctx_len", _P), ("max_ctx", _I32),
                 ("page_table", _P), ("page_size", _I32), ("max_pages", _I32),
                 ("num_pages", _I32),
-                ("o", _P), ("o_sb", _I64), ("o_st", _I64), ("o_sh", _I64), ("lse", _P)]
+                ("o", _P), ("o_sb", _I64), ("o_st", _I64), ("o_sh", _I64), ("lse", _P),
+                ("kv_dtype", _I32), ("k_scale", _F32), ("v_scale", _F32)]
 
 
 _lock = threading.Lock()
@@ -248,11 +250,23 @@ def sinkattn_prefill_chunk(q, k, v, sink=None, *, prefix, window=0, o=None, lse=
 # decode
 # ----------------------------------------------------------------------------------------------
 
+def _is_fp8_cache(t):
+    return isinstance(t, torch.Tensor) and t.dtype in (torch.uint8, torch.float8_e4m3fn)
+
+
 def _decode_args(kind, q, k_new, v_new, k_cache, v_cache, sink, window, scale, ring_head,
-                 ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse):
-    for n, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
-                 ("v_cache", v_cache)):
+                 ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse,
+                 k_scale=None, v_scale=None):
+    for n, t in (("q", q), ("k_new", k_new), ("v_new", v_new)):
         _check_bf16(n, t)
+    fp8 = _is_fp8_cache(k_cache)
+    for n, t in (("k_cache", k_cache), ("v_cache", v_cache)):
+        if fp8:
+            if not _is_fp8_cache(t) or not t.is_cuda or t.dim() != 4 or t.stride(-1) != 1:
+                raise ValueError(f"{n}: an FP8 cache is a 4-D CUDA uint8 / float8_e4m3fn tensor "
+                                 "with a contiguous last dim (both caches alike)")
+        else:
+            _check_bf16(n, t)
     if o is not None:
         _check_bf16("o", o)
     _check_vec("sink", sink, torch.float32)
@@ -291,6 +305,10 @@ def _decode_args(kind, q, k_new, v_new, k_cache, v_cache, sink, window, scale, r
     if o is not None:
         a.o, a.o_sb, a.o_st, a.o_sh = _ptr(o), o.stride(0), o.stride(1), o.stride(2)
     a.lse = _ptr(lse)
+    if fp8:
+        if k_scale is None or v_scale is None:
+            raise ValueError("an FP8 cache needs k_scale and v_scale")
+        a.kv_dtype, a.k_scale, a.v_scale = KV_FP8_E4M3, float(k_scale), float(v_scale)
     return a
 
 
@@ -298,19 +316,21 @@ def sinkattn_decode_workspace_size(kind, q, k_new, v_new, k_cache, v_cache, *, w
                                    ring_head=None, ring_len=None, ctx_len=None, max_ctx=None,
                                    page_table=None, page_size=None, num_pages=None) -> int:
     a = _decode_args(kind, q, k_new, v_new, k_cache, v_cache, None, window, 1.0, ring_head,
-                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, None, None)
+                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, None, None,
+                     1.0, 1.0)
     return int(lib().sinkattn_decode_workspace_size(ctypes.byref(a)))
 
 
 def sinkattn_decode(kind, q, k_new, v_new, k_cache, v_cache, sink=None, *, window=0,
                     ring_head=None, ring_len=None, ctx_len=None, max_ctx=None, page_table=None,
                     page_size=None, num_pages=None, o=None, lse=None, workspace=None,
-                    scale=None, stream=None, want_lse=True):
+                    scale=None, stream=None, want_lse=True, k_scale=None, v_scale=None):
     """Decode / speculative verify of T (1..4) new tokens per sequence against a KV cache.
 
     kind: KV_RING (k_cache [B,cap,Hkv,192] with ring_head/ring_len int32 [B]), KV_CONTIG
     (k_cache [B,max_ctx,Hkv,192] with ctx_len [B]) or KV_PAGED (k_cache [pages,page,Hkv,192]
     with page_table [B,max_pages] and ctx_len [B]). The new tokens' K/V are not in the cache.
+    A uint8 / float8_e4m3fn cache holds E4M3 codes scaled by k_scale / v_scale (FP8 cache).
     Returns (o [B,T,Hq,128] bf16, lse [B,T,Hq] fp32 or None)."""
     B, T, Hq, dq = q.shape
     if scale is None:
@@ -320,7 +340,8 @@ def sinkattn_decode(kind, q, k_new, v_new, k_cache, v_cache, sink=None, *, windo
     if lse is None and want_lse:
         lse = torch.empty(B, T, Hq, dtype=torch.float32, device=q.device)
     a = _decode_args(kind, q, k_new, v_new, k_cache, v_cache, sink, window, scale, ring_head,
-                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse)
+                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse,
+                     k_scale, v_scale)
     L_ = lib()
     need = int(L_.sinkattn_decode_workspace_size(ctypes.byref(a)))
     if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
@@ -335,7 +356,7 @@ def sinkattn_decode(kind, q, k_new, v_new, k_cache, v_cache, sink=None, *, windo
 def sinkattn_decode_noalloc(kind, q, k_new, v_new, k_cache, v_cache, sink=None, *, window=0,
                             ring_head=None, ring_len=None, ctx_len=None, max_ctx=None,
                             page_table=None, page_size=None, num_pages=None, o=None, lse=None,
-                            scale=None, stream=None):
+                            scale=None, stream=None, k_scale=None, v_scale=None):
     """Decode without a workspace, for callers that cannot allocate device memory (a plugin host
     that passes only input/output buffers, a serving loop with all memory reserved up front).
     The library keeps the split-KV partials in its own fixed 16 MiB device array; larger
@@ -347,7 +368,8 @@ def sinkattn_decode_noalloc(kind, q, k_new, v_new, k_cache, v_cache, sink=None, 
     if scale is None:
         scale = 1.0 / math.sqrt(dq)
     a = _decode_args(kind, q, k_new, v_new, k_cache, v_cache, sink, window, scale, ring_head,
-                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse)
+                     ring_len, ctx_len, max_ctx, page_table, page_size, num_pages, o, lse,
+                     k_scale, v_scale)
     _raise(lib().sinkattn_decode_noalloc(ctypes.byref(a), _stream(stream)),
            "sinkattn_decode_noalloc")
     return o, lse
@@ -355,13 +377,16 @@ def sinkattn_decode_noalloc(kind, q, k_new, v_new, k_cache, v_cache, sink=None, 
 
 def sinkattn_kv_commit(kind, k_new, v_new, n_accept, k_cache, v_cache, *, ring_head=None,
                        ring_len=None, ctx_len=None, max_ctx=None, page_table=None,
-                       num_pages=None, stream=None):
-    """Append the first n_accept[b] of each sequence's T new tokens to its cache, in place."""
+                       num_pages=None, stream=None, k_scale=None, v_scale=None):
+    """Append the first n_accept[b] of each sequence's T new tokens to its cache, in place.
+    Into an FP8 cache (uint8 / float8_e4m3fn) each element x is stored as the E4M3 code of
+    x / scale (k_scale for K, v_scale for V)."""
     _check_vec("n_accept", n_accept, torch.int32)
     B, T, Hkv, dq = k_new.shape
     q_dummy = k_new  # only the cache-related fields are read
     a = _decode_args(kind, q_dummy, k_new, v_new, k_cache, v_cache, None, 0, 1.0, ring_head,
-                     ring_len, ctx_len, max_ctx, page_table, None, num_pages, None, None)
+                     ring_len, ctx_len, max_ctx, page_table, None, num_pages, None, None,
+                     k_scale, v_scale)
     st = lib().sinkattn_kv_commit(ctypes.byref(a), _ptr(n_accept), _stream(stream))
     _raise(st, "sinkattn_kv_commit")
 

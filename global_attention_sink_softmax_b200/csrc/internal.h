@@ -71,6 +71,12 @@ struct DecodeParams {
     float *lse;
     float *ws_o;    // [B, Hkv, splits, R, 128] (splits > 1)
     float *ws_ml;   // [B, Hkv, splits, R, 4]: max, sum of rounded P, sum of fp32 P, pad
+    // FP8 (E4M3) cache: k8 / v8 are the caches as bytes (strides above count bytes); the new
+    // tokens are quantised with k_scale / v_scale, scale_log2 includes k_scale and O is
+    // multiplied by v_scale
+    int fp8;
+    float k_scale, v_scale;
+    const uint8_t *k8, *v8;
 };
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream);
@@ -105,9 +111,13 @@ struct CommitParams {
     const int32_t *page_table;
     int page_size, max_pages, num_pages;
     const int32_t *n_accept;
+    int fp8;               // quantise into an E4M3 cache (strides count bytes)
+    float k_scale, v_scale;
 };
 
 cudaError_t launch_commit(const CommitParams &p, cudaStream_t stream);
+cudaError_t launch_decode_fp8(const DecodeParams &p, cudaStream_t stream);
+cudaError_t launch_commit_fp8(const CommitParams &p, cudaStream_t stream);
 
 // Fused partial RoPE + value scale, in place (rope_kernels.cuh).
 constexpr int kRopeMaxHalf = 64; // rope_dim <= 128

@@ -9,6 +9,7 @@
 
 #include "common.cuh"
 #include "decode_kernels.cuh"
+#include "decode_fp8_kernels.cuh"
 #include "decode_tma_kernels.cuh"
 #include "decode_umma_kernels.cuh"
 #include "decode_ring_kernels.cuh"
@@ -48,6 +49,8 @@ EncodeTiledFn encode_fn()
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 // element strides of bf16 tensors: positive and a whole number of 16-byte units
 bool stride_ok(int64_t s) { return s > 0 && (s % 8) == 0; }
+// byte strides (one-byte elements): positive multiples of 16
+bool stride_ok_bytes(int64_t s) { return s > 0 && (s % 16) == 0; }
 
 // 4-D bf16 map over [B, tokens, heads, d] given as dims {d, heads, tokens, B}; box
 // {64, box_heads, box_tokens, 1}, 128-byte swizzle, zero fill outside the tensor.
@@ -293,6 +296,19 @@ int validate_decode_shape(const sinkattn_decode_args *a)
     return SINKATTN_OK;
 }
 
+// The cache element type and, for FP8, its two scales (finite, > 0).
+int kv_dtype_check(const sinkattn_decode_args *a)
+{
+    if (a->kv_dtype == SINKATTN_KV_BF16)
+        return SINKATTN_OK;
+    if (a->kv_dtype != SINKATTN_KV_FP8_E4M3)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (!isfinite(a->k_scale) || !(a->k_scale > 0.f) || !isfinite(a->v_scale) ||
+        !(a->v_scale > 0.f))
+        return SINKATTN_ERR_INVALID_ARG;
+    return SINKATTN_OK;
+}
+
 int validate_decode(const sinkattn_decode_args *a)
 {
     if (!a)
@@ -307,6 +323,8 @@ int validate_decode(const sinkattn_decode_args *a)
     if (G > 16 || a->T * G > 64)
         return SINKATTN_ERR_UNSUPPORTED;
     if (!isfinite(a->scale) || !(a->scale > 0.f))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (kv_dtype_check(a) != SINKATTN_OK)
         return SINKATTN_ERR_INVALID_ARG;
     if (a->kind == SINKATTN_KV_RING) {
         if (a->ring_cap <= 0 || !a->ring_head || !a->ring_len)
@@ -332,10 +350,12 @@ int validate_decode(const sinkattn_decode_args *a)
     const int64_t s[15] = {a->q_sb,  a->q_st,  a->q_sh,  a->kn_sb, a->kn_st,
                            a->kn_sh, a->vn_sb, a->vn_st, a->vn_sh, a->kc_sb,
                            a->kc_ss, a->kc_sh, a->vc_sb, a->vc_ss, a->vc_sh};
+    const bool fp8 = a->kv_dtype == SINKATTN_KV_FP8_E4M3;
     for (int i = 0; i < 15; ++i) {
         if (s[i] <= 0)
             return SINKATTN_ERR_INVALID_ARG;
-        if (!stride_ok(s[i]))
+        // cache strides (the last six) of an FP8 cache count bytes
+        if ((fp8 && i >= 9) ? !stride_ok_bytes(s[i]) : !stride_ok(s[i]))
             return SINKATTN_ERR_ALIGNMENT;
     }
     const int64_t so[3] = {a->o_sb, a->o_st, a->o_sh};
@@ -361,7 +381,13 @@ void fill_decode_params(DecodeParams &p, const sinkattn_decode_args *a, const Sp
     p.window = a->window;
     p.splits = s.splits;
     p.chunk = s.chunk;
-    p.scale_log2 = a->scale * kLog2e;
+    p.fp8 = a->kv_dtype == SINKATTN_KV_FP8_E4M3;
+    p.k_scale = p.fp8 ? a->k_scale : 1.f;
+    p.v_scale = p.fp8 ? a->v_scale : 1.f;
+    p.k8 = static_cast<const uint8_t *>(a->k_cache);
+    p.v8 = static_cast<const uint8_t *>(a->v_cache);
+    // an FP8 cache's logits are scale * k_scale * <q, e(c)>
+    p.scale_log2 = a->scale * kLog2e * p.k_scale;
     p.sink = a->sink;
     p.q = static_cast<const uint16_t *>(a->q);
     p.k_new = static_cast<const uint16_t *>(a->k_new);
@@ -455,6 +481,10 @@ bool decode_tma_ok(const sinkattn_decode_args *a, const DecodeParams &)
 int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *stream)
 {
     cudaError_t e;
+    if (p.fp8) {
+        e = launch_decode_fp8(p, (cudaStream_t)stream);
+        return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+    }
     if (a->kind == SINKATTN_KV_RING && p.R <= 16 && a->ring_cap % 32 == 0 && p.splits == 1) {
         // a ring item per warp, streamed in 32-key chunks (units of more than 16 rows, as in a
         // 4-token verify, measured faster on the cp.async kernel, whose CTA serves all rows)
@@ -612,6 +642,8 @@ int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, v
         return SINKATTN_ERR_INVALID_ARG;
     if (a->dq != kDQ || a->dv != kDV)
         return SINKATTN_ERR_UNSUPPORTED;
+    if (kv_dtype_check(a) != SINKATTN_OK)
+        return SINKATTN_ERR_INVALID_ARG;
     if (a->B == 0 || a->T == 0)
         return SINKATTN_OK;
     if (!n_accept || !a->k_new || !a->v_new || !a->k_cache || !a->v_cache)
@@ -629,13 +661,17 @@ int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, v
             return SINKATTN_ERR_ALIGNMENT;
     const int64_t s[12] = {a->kn_sb, a->kn_st, a->kn_sh, a->vn_sb, a->vn_st, a->vn_sh,
                            a->kc_sb, a->kc_ss, a->kc_sh, a->vc_sb, a->vc_ss, a->vc_sh};
+    const bool fp8 = a->kv_dtype == SINKATTN_KV_FP8_E4M3;
     for (int i = 0; i < 12; ++i) {
         if (s[i] <= 0)
             return SINKATTN_ERR_INVALID_ARG;
-        if (!stride_ok(s[i]))
+        if ((fp8 && i >= 6) ? !stride_ok_bytes(s[i]) : !stride_ok(s[i]))
             return SINKATTN_ERR_ALIGNMENT;
     }
     CommitParams p;
+    p.fp8 = fp8;
+    p.k_scale = fp8 ? a->k_scale : 1.f;
+    p.v_scale = fp8 ? a->v_scale : 1.f;
     p.kind = a->kind;
     p.B = a->B;
     p.T = a->T;
@@ -666,7 +702,8 @@ int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, v
     p.max_pages = a->max_pages;
     p.num_pages = a->num_pages;
     p.n_accept = n_accept;
-    const cudaError_t e = launch_commit(p, (cudaStream_t)stream);
+    const cudaError_t e = fp8 ? launch_commit_fp8(p, (cudaStream_t)stream)
+                              : launch_commit(p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

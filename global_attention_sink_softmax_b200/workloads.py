@@ -104,6 +104,17 @@ def normal_bf16(shape, g: torch.Generator, device) -> torch.Tensor:
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
 
 
+# Per-tensor scales of the synthetic FP8 caches: N(0, 1) values up to ~6 fill the E4M3 range.
+FP8_K_SCALE, FP8_V_SCALE = 6.0 / 448.0, 5.0 / 448.0
+
+
+def fp8_codes(shape, g: torch.Generator, device, scale: float) -> torch.Tensor:
+    """One-byte E4M3 codes of N(0, 1) draws divided by `scale`, made with torch's float8 cast
+    (a library conversion, as torch.randn is a library draw), clamped to the finite range."""
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32) / scale
+    return x.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+
+
 def sinks(Hq: int, g: torch.Generator, device, neg_inf_heads=()) -> torch.Tensor:
     s = torch.rand(Hq, generator=g, device=device, dtype=torch.float32) * 6.0
     for h in neg_inf_heads:
@@ -126,25 +137,32 @@ def prefill_inputs(w: PrefillWorkload, device="cpu", L: Optional[int] = None,
 
 def decode_inputs(w: DecodeWorkload, device="cpu", B: Optional[int] = None,
                   ctx: Optional[int] = None, ctx_hi: Optional[int] = None,
-                  seed: Optional[int] = None):
+                  seed: Optional[int] = None, fp8: bool = False):
     """Seeded decode inputs. Returns a dict with q/k_new/v_new [B,T,H,d], the cache tensors and
-    the cache metadata of the workload's kind (ring_head/ring_len, ctx_len, page_table)."""
+    the cache metadata of the workload's kind (ring_head/ring_len, ctx_len, page_table).
+    fp8=True: the caches are uint8 E4M3 codes (fp8_codes, scales FP8_K_SCALE / FP8_V_SCALE,
+    also returned as k_scale / v_scale)."""
     B = w.B if B is None else B
     g = _gen(w.seed if seed is None else seed, device)
+
+    def cache(shape, which):
+        if not fp8:
+            return normal_bf16(shape, g, device)
+        return fp8_codes(shape, g, device, FP8_K_SCALE if which == "k" else FP8_V_SCALE)
     d = dict(q=normal_bf16((B, w.T, w.Hq, w.dq), g, device),
              k_new=normal_bf16((B, w.T, w.Hkv, w.dq), g, device),
              v_new=normal_bf16((B, w.T, w.Hkv, w.dv), g, device),
              sink=sinks(w.Hq, g, device))
     if w.kind == KV_RING:
-        d["k_cache"] = normal_bf16((B, w.ring_cap, w.Hkv, w.dq), g, device)
-        d["v_cache"] = normal_bf16((B, w.ring_cap, w.Hkv, w.dv), g, device)
+        d["k_cache"] = cache((B, w.ring_cap, w.Hkv, w.dq), "k")
+        d["v_cache"] = cache((B, w.ring_cap, w.Hkv, w.dv), "v")
         d["ring_head"] = torch.randint(0, w.ring_cap, (B,), generator=g, device=device,
                                        dtype=torch.int32)
         d["ring_len"] = torch.full((B,), w.ring_cap, dtype=torch.int32, device=device)
     elif w.kind == KV_CONTIG:
         c = w.ctx if ctx is None else ctx
-        d["k_cache"] = normal_bf16((B, c, w.Hkv, w.dq), g, device)
-        d["v_cache"] = normal_bf16((B, c, w.Hkv, w.dv), g, device)
+        d["k_cache"] = cache((B, c, w.Hkv, w.dq), "k")
+        d["v_cache"] = cache((B, c, w.Hkv, w.dv), "v")
         d["ctx_len"] = torch.full((B,), c, dtype=torch.int32, device=device)
         d["max_ctx"] = c
     else:
@@ -162,10 +180,12 @@ def decode_inputs(w: DecodeWorkload, device="cpu", B: Optional[int] = None,
         for b, n in enumerate(pages_per):
             table[b, :n] = perm[off:off + n]
             off += n
-        d["k_cache"] = normal_bf16((total, P, w.Hkv, w.dq), g, device)
-        d["v_cache"] = normal_bf16((total, P, w.Hkv, w.dv), g, device)
+        d["k_cache"] = cache((total, P, w.Hkv, w.dq), "k")
+        d["v_cache"] = cache((total, P, w.Hkv, w.dv), "v")
         d["ctx_len"] = ctx_len
         d["page_table"] = table
         d["max_ctx"] = max_pages * P
         d["page_size"] = P
+    if fp8:
+        d["k_scale"], d["v_scale"] = FP8_K_SCALE, FP8_V_SCALE
     return d

@@ -75,6 +75,16 @@ typedef enum sinkattn_kv_kind {
     SINKATTN_KV_PAGED = 2    /* page pool + per-sequence page table (GA) */
 } sinkattn_kv_kind;
 
+/* Element type of a KV cache (decode and commit). The new tokens' k_new / v_new are bf16 with
+ * either. FP8 reading: the pages size a KV slot at one byte ("MiMo-V2-Flash Technical Report"
+ * paper notes, KV-memory arithmetic) and speak of FP8 inference, naming no format; the library
+ * stores E4M3 ("fn": bias 7, no infinities, largest finite 448) codes with one fp32 scale per
+ * cache tensor, a code c meaning e4m3(c) * scale. */
+typedef enum sinkattn_kv_dtype {
+    SINKATTN_KV_BF16 = 0,     /* bf16 elements (the default of a zero-initialised struct) */
+    SINKATTN_KV_FP8_E4M3 = 1  /* one-byte E4M3 codes, scaled by k_scale / v_scale */
+} sinkattn_kv_dtype;
+
 /* ---------------------------------------------------------------------------------------------
  * Prefill: every position of every sequence attends to its own sequence.
  *
@@ -171,6 +181,15 @@ typedef struct sinkattn_decode_args {
     void *o;
     int64_t o_sb, o_st, o_sh;
     float *lse;
+    /* Cache element type (sinkattn_kv_dtype). With SINKATTN_KV_FP8_E4M3, k_cache / v_cache hold
+     * one-byte codes in the same [.., Hkv, d] layouts, their strides count bytes and must be
+     * multiples of 16, and a K (V) code c stands for e4m3(c) * k_scale (v_scale); both scales
+     * must be finite and > 0. Decode then attends to the T new tokens as the commit will store
+     * them: each new K / V element x becomes the E4M3 value nearest to x / scale (the division
+     * in fp32, ties to even, saturating to +-448). Q is rounded to fp16 for the tensor cores, so
+     * |q| must stay below 65504 on this path. */
+    int32_t kv_dtype;
+    float k_scale, v_scale;
 } sinkattn_decode_args;
 
 /* Bytes of device workspace sinkattn_decode needs for these arguments (split-KV partials:

@@ -297,8 +297,11 @@ def decode_fp8(kind, q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, sink, 
     and e(c) is exact in bf16 (4 significant bits, exponents -9..8), so this is the bf16 decode
     above on the E4M3 values with the scale scale * k_scale, and O times v_scale. LSE is the
     one of those logits. Returns (o, lse, wsink) as decode()."""
-    def values_bf16(codes):
-        return fp8_decode(codes).to(torch.bfloat16)
+    lut = fp8_decode(torch.arange(256, dtype=torch.uint8)).to(torch.bfloat16)
+
+    def values_bf16(codes):  # e(c), exact in bf16; one leading index at a time bounds memory
+        return torch.stack([lut[c.long()] for c in codes.cpu()]) if codes.shape[0] else \
+            torch.empty(codes.shape, dtype=torch.bfloat16)
 
     kn = values_bf16(fp8_encode(k_new, k_scale))
     vn = values_bf16(fp8_encode(v_new, v_scale))

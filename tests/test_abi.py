@@ -232,6 +232,34 @@ def test_rope_empty_and_partial_calls_need_no_device(L):
     assert L.sinkattn_rope_qkv(None, None) == 1
 
 
+FP8 = dict(kv_dtype=1, k_scale=0.02, v_scale=0.02)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kv_dtype=2), 1), (dict(kv_dtype=-1), 1),
+    (dict(FP8, k_scale=0.0), 1), (dict(FP8, v_scale=-0.5), 1),
+    (dict(FP8, k_scale=float("nan")), 1), (dict(FP8, v_scale=float("inf")), 1),
+    # an FP8 cache's strides count bytes: 200 is a whole number of 16-byte bf16 units (8-element
+    # multiples) but not of 16 bytes
+    (dict(FP8, kc_ss=200), 3), (dict(FP8, vc_sh=136), 3),
+])
+def test_fp8_cache_arguments_are_checked(L, kw, status):
+    a = _decode_args(**kw)
+    assert L.sinkattn_decode(ctypes.byref(a), None, 0, None) == status
+    assert L.sinkattn_decode_noalloc(ctypes.byref(a), None) == status
+    assert L.sinkattn_kv_commit(ctypes.byref(a), ctypes.c_void_p(0x60000), None) == status
+
+
+def test_fp8_strides_fine_for_bf16_and_workspace_independent_of_dtype(L):
+    # the bf16 reading of the same 200-element stride is aligned: that call fails only later,
+    # on the missing workspace (a GA context of 4096 tokens needs a split)
+    a = _decode_args(kc_ss=200, B=8, max_ctx=262144)
+    assert L.sinkattn_decode(ctypes.byref(a), None, 0, None) == 4
+    b = _decode_args(B=8, max_ctx=262144, **FP8)
+    assert L.sinkattn_decode_workspace_size(ctypes.byref(b)) == \
+        L.sinkattn_decode_workspace_size(ctypes.byref(_decode_args(B=8, max_ctx=262144)))
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sa, "library_path", str(tmp_path / "missing.so"))
     monkeypatch.setattr(sa, "_lib", None)
