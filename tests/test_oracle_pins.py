@@ -582,3 +582,63 @@ def test_decode_fp8_equals_eager_dequantised(window):
     eo, el = eager_fp8_decode(q, k_new, v_new, kc, vc, ks, vs, ctx, sink, scale, window)
     assert torch.allclose(o, eo, rtol=0, atol=1e-12)
     assert torch.allclose(lse, el, rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------------------------
+# brute force: a second, naive fp64 double loop over tiny inputs
+# ----------------------------------------------------------------------------------------------
+
+def naive_row(qv, keys, vals, sink, scale):
+    """One query row by hand: plain Python floats, math.exp / math.log, nothing shared."""
+    a = [scale * sum(x * y for x, y in zip(qv, kv)) for kv in keys]
+    m = max([sink] + a)
+    ws = math.exp(sink - m) if sink != -math.inf else 0.0
+    es = [math.exp(x - m) for x in a]
+    D = ws + sum(es)
+    o = [sum(e * vv[c] for e, vv in zip(es, vals)) / D for c in range(len(vals[0]))]
+    return o, m + math.log(D)
+
+
+@pytest.mark.parametrize("L,window", [(1, 0), (2, 0), (5, 0), (8, 0), (8, 3), (7, 1), (6, 128)])
+def test_brute_force_tiny_prefill(L, window):
+    g = torch.Generator().manual_seed(31 + L + window)
+    B, Hq, Hkv = 2, 4, 2
+    q, k, v = rand_bf16((B, L, Hq, 192), g), rand_bf16((B, L, Hkv, 192), g), rand_bf16((B, L, Hkv, 128), g)
+    sink = torch.tensor([1.5, float("-inf"), -2.0, 4.0])
+    scale = 1.0 / math.sqrt(192)
+    o, lse, _ = oracle.prefill(q, k, v, sink, scale, window)
+    qd, kd, vd = q.double().tolist(), k.double().tolist(), v.double().tolist()
+    for b in range(B):
+        for i in range(L):
+            lo = max(0, i - window + 1) if window > 0 else 0
+            for h in range(Hq):
+                gk = h // (Hq // Hkv)
+                keys = [kd[b][j][gk] for j in range(lo, i + 1)]
+                vals = [vd[b][j][gk] for j in range(lo, i + 1)]
+                ro, rl = naive_row(qd[b][i][h], keys, vals, float(sink[h]), scale)
+                assert max(abs(x - y) for x, y in zip(o[b, i, h].tolist(), ro)) < 1e-12
+                assert abs(lse[b, i, h].item() - rl) < 1e-12
+
+
+def test_brute_force_tiny_decode():
+    """Decode over a 5-token contiguous cache + T = 3 new tokens, window 4, by hand."""
+    g = torch.Generator().manual_seed(37)
+    B, T, Hq, Hkv, n = 1, 3, 2, 1, 5
+    q = rand_bf16((B, T, Hq, 192), g)
+    kn, vn = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    kc, vc = rand_bf16((B, n + 2, Hkv, 192), g), rand_bf16((B, n + 2, Hkv, 128), g)
+    sink = torch.tensor([0.7, -1.0])
+    scale = 1.0 / math.sqrt(192)
+    for window in (0, 4):
+        o, lse, _ = oracle.decode(oracle.KV_CONTIG, q, kn, vn, kc, vc, sink, scale, window,
+                                  ctx_len=torch.tensor([n], dtype=torch.int32))
+        # positions: cached token c at c - n, new token u at u
+        K = [(c - n, kc[0, c, 0].double().tolist(), vc[0, c, 0].double().tolist()) for c in range(n)]
+        K += [(u, kn[0, u, 0].double().tolist(), vn[0, u, 0].double().tolist()) for u in range(T)]
+        for t in range(T):
+            vis = [(kk, vv) for p, kk, vv in K if p <= t and (window == 0 or p > t - window)]
+            for h in range(Hq):
+                ro, rl = naive_row(q[0, t, h].double().tolist(), [x[0] for x in vis],
+                                   [x[1] for x in vis], float(sink[h]), scale)
+                assert max(abs(x - y) for x, y in zip(o[0, t, h].tolist(), ro)) < 1e-12
+                assert abs(lse[0, t, h].item() - rl) < 1e-12
