@@ -474,6 +474,92 @@ def cpu_baseline_prefill(w, d_cpu, target_s=12.0):
             "sample": f"{n} random (batch, position) rows x all {w.Hq} heads of {w.name}"}
 
 
+def _cpu(t):
+    return t.cpu() if isinstance(t, torch.Tensor) else t
+
+
+def cpu_oracle_sample(kind, w, d, n, seed=0):
+    """One timed oracle call on a sample of size n of a secondary workload (inputs on any
+    device; only the sample is copied to the host). Returns (work, seconds, what) where work is
+    FLOPs for prefill and bytes (the job's algorithmic bytes per unit) otherwise."""
+    import oracle
+    g = torch.Generator().manual_seed(seed)
+    if kind == "prefill":
+        P = getattr(w, "prefix", 0)
+        q = d["q"]
+        if P:  # the chunk's queries sit at positions P.. of sequences of P + L positions
+            qf = torch.zeros((w.B, P + w.L) + tuple(q.shape[2:]), dtype=q.dtype)
+            qf[:, P:] = _cpu(q)
+        else:
+            qf = _cpu(q)
+        rows = torch.stack([torch.randint(0, w.B, (n,), generator=g),
+                            P + torch.randint(0, w.L, (n,), generator=g)], 1)
+        t0 = time.perf_counter()
+        oracle.prefill(qf, _cpu(d["k"]), _cpu(d["v"]), _cpu(d["sink"]), W.SCALE, w.window,
+                       rows=rows)
+        dt = time.perf_counter() - t0
+        pairs = sum((min(i + 1, w.window) if w.window else i + 1) for i in rows[:, 1].tolist())
+        return pairs * w.Hq * FLOP_PER_PAIR, dt, f"{n} random (batch, position) rows x {w.Hq} heads"
+    if kind == "rope":
+        b = torch.randint(0, w.B, (n,), generator=g)
+        l = torch.randint(0, w.L, (n,), generator=g)
+        qs, ks, vs = _cpu(d["q"][b, l]), _cpu(d["k"][b, l]), _cpu(d["v"][b, l])
+        t0 = time.perf_counter()
+        oracle.rope(qs, l.numpy(), 1e4)
+        oracle.rope(ks, l.numpy(), 1e4)
+        oracle.vscale(vs, 0.707)
+        dt = time.perf_counter() - t0
+        per_tok = 2 * ((w.Hq + w.Hkv) * 64 * 2 + w.Hkv * w.dv * 2)
+        return n * per_tok, dt, f"{n} random tokens (all heads)"
+    # decode against a contiguous or ring cache, bf16 or FP8: n sampled sequences
+    seqs = torch.randperm(w.B, generator=g)[:n]
+    per_seq = ("q", "k_new", "v_new", "k_cache", "v_cache", "ring_head", "ring_len", "ctx_len")
+    sub = {k: (_cpu(v[seqs.to(v.device)]) if k in per_seq else _cpu(v)) for k, v in d.items()}
+    kw = {}
+    if w.kind == W.KV_RING:
+        kw.update(ring_head=sub["ring_head"], ring_len=sub["ring_len"])
+    else:
+        kw.update(ctx_len=sub["ctx_len"])
+    t0 = time.perf_counter()
+    if "k_scale" in d:
+        oracle.decode_fp8(w.kind, sub["q"], sub["k_new"], sub["v_new"], sub["k_cache"],
+                          sub["v_cache"], d["k_scale"], d["v_scale"], sub["sink"], W.SCALE,
+                          w.window, **kw)
+    else:
+        oracle.decode(w.kind, sub["q"], sub["k_new"], sub["v_new"], sub["k_cache"],
+                      sub["v_cache"], sub["sink"], W.SCALE, w.window, **kw)
+    dt = time.perf_counter() - t0
+    return None, dt, f"{len(seqs)} random sequences of {w.B}"
+
+
+def cpu_baseline_secondary(kind, r, target_s=2.0):
+    """The oracle on the host cores, on a bounded sample of a secondary workload: its rate in
+    the job's unit and the whole workload's oracle time extrapolated from that rate (labelled
+    so). Never raises: a failure is reported in the entry instead."""
+    try:
+        w = r.w
+        if kind == "decode":
+            n = min(w.B, 2 if w.B <= 8 else 16)
+            _, dt, what = cpu_oracle_sample(kind, w, r.d, n)
+            work = r.bytes * n / w.B  # every sequence of these workloads holds the same context
+            rate, unit, full = work / dt / 1e9, "GB/s", r.bytes / (work / dt)
+        else:
+            n = 16
+            work, dt, what = cpu_oracle_sample(kind, w, r.d, n)
+            n = max(n, min(1 << 16, int(n * target_s / max(dt, 1e-3))))
+            work, dt, what = cpu_oracle_sample(kind, w, r.d, n, seed=n)
+            if kind == "prefill":
+                rate, unit, full = work / dt / 1e12, "TFLOP/s", r.flops / (work / dt)
+            else:
+                rate, unit, full = work / dt / 1e9, "GB/s", r.bytes / (work / dt)
+        cores = 1 if kind == "rope" else omp_threads()  # the RoPE oracle is one plain loop
+        return {"value": round(rate, 6), "unit": unit, "cores": cores, "kind": "oracle",
+                "seconds": round(dt, 2), "sample": f"{what} of {getattr(r, 'workload', w.name)}",
+                "full_workload_s_extrapolated": round(full, 3)}
+    except Exception as e:  # the baseline is a report; it must not cost the benchmark its line
+        return {"kind": "oracle", "error": f"{type(e).__name__}: {e}"[:200]}
+
+
 # ----------------------------------------------------------------------------------------------
 # main
 # ----------------------------------------------------------------------------------------------
@@ -662,6 +748,11 @@ def main():
                      "gbs": round(r.bytes / (ms_step * 1e-3) / 1e9, 2), "roofline": rl,
                      "gpu_launches_per_step": r.launches, "clocks": clk.summary(),
                      "l2": "flushed between steps" if fl else "working set larger than L2"}
+            cb_kind = {"ga_prefill": "prefill", "ga_chunk_prefill": "prefill", "rope_qkv": "rope",
+                       "ga_decode": "decode", "ga_decode_fp8": "decode",
+                       "swa_decode": "decode"}.get(name)
+            if cb_kind and rank == 0 and world == 1 and not args.no_cpu_baseline:
+                entry["cpu_baseline"] = cpu_baseline_secondary(cb_kind, r)
             if name == "hybrid":
                 entry["note"] = ("layer list taken literally: 49 layer calls (9 GA, 40 SWA); "
                                  "GB/s over all layers' algorithmic bytes")
