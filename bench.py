@@ -541,6 +541,10 @@ def cpu_baseline_secondary(kind, r, target_s=2.0):
         if kind == "decode":
             n = min(w.B, 2 if w.B <= 8 else 16)
             _, dt, what = cpu_oracle_sample(kind, w, r.d, n)
+            grown = max(n, min(w.B, int(n * target_s / max(dt, 1e-3))))
+            if grown > n:
+                n = grown
+                _, dt, what = cpu_oracle_sample(kind, w, r.d, n, seed=n)
             work = r.bytes * n / w.B  # every sequence of these workloads holds the same context
             rate, unit, full = work / dt / 1e9, "GB/s", r.bytes / (work / dt)
         else:
