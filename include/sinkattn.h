@@ -22,11 +22,13 @@
  * window W keeps i - W < j <= i (exactly W keys once i >= W - 1, the query included).
  *
  * Conventions shared by every entry point.
- *   - Element types: q, k, v, o and the caches are bf16; sink and lse are fp32.
+ *   - Element types: q, k, v, o and the caches are bf16 (a decode cache may instead hold
+ *     one-byte FP8 codes: see sinkattn_kv_dtype); sink and lse are fp32.
  *   - Layouts are token-major, [batch, token, head, dim], the dim contiguous; the other
  *     three dims are given as element strides (int64). Base pointers and every non-unit
  *     stride in bytes must be multiples of 16.
- *   - Head dims: dq = 192 and dv = 128 (the kernels are specialised for them).
+ *   - Head dims: dq = 192 and dv = 128 for attention and commit (the kernels are specialised
+ *     for them); sinkattn_rope_qkv states its own limits.
  *     GQA group G = Hq / Hkv must be an integer in 1..16 (prefill) or 1..16 (decode).
  *   - sink: fp32 [Hq] in post-scale logit units (not multiplied by scale). NULL means no sink
  *     for any head; an entry of -inf means plain softmax for that head. NaN or +inf entries
