@@ -75,6 +75,9 @@ def _load():
             lib.sinkattn_oracle_fp8_decode.restype = None
             lib.sinkattn_oracle_e4m3_encode.argtypes = [ctypes.c_float]
             lib.sinkattn_oracle_e4m3_encode.restype = ctypes.c_uint8
+            lib.sinkattn_oracle_prefill_backward.argtypes = [P, P, P, P, P, i32, i32, i32, i32,
+                                                             i32, i32, i32, f64, P, P, P, P]
+            lib.sinkattn_oracle_prefill_backward.restype = i32
             _lib = lib
     return _lib
 
@@ -309,3 +312,25 @@ def decode_fp8(kind, q, k_new, v_new, k_codes, v_codes, k_scale, v_scale, sink, 
     f32 = lambda s: float(np.float32(s))
     o, lse, ws = decode(kind, q, kn, vn, kc, vc, sink, scale * f32(k_scale), window, **kw)
     return o * f32(v_scale), lse, ws
+
+
+def prefill_backward(q, k, v, sink, dout, scale, window=0):
+    """Gradients of sum(O * dout) of the prefill (serial; small cases).
+
+    q [B,L,Hq,dq], k [B,L,Hkv,dq], v [B,L,Hkv,dv], dout [B,L,Hq,dv] bf16; sink [Hq] or None.
+    Returns (dq, dk, dv, dsink [Hq]) float64."""
+    lib = _load()
+    B, L, Hq, dq = q.shape
+    Hkv, dv = k.shape[2], v.shape[3]
+    qb, kb, vb, db = _bits(q), _bits(k), _bits(v), _bits(dout)
+    s = _f32(sink)
+    gq = np.zeros((B, L, Hq, dq), np.float64)
+    gk = np.zeros((B, L, Hkv, dq), np.float64)
+    gv = np.zeros((B, L, Hkv, dv), np.float64)
+    gs = np.zeros(Hq, np.float64)
+    rc = lib.sinkattn_oracle_prefill_backward(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(s), _ptr(db), B,
+                                              L, Hq, Hkv, dq, dv, int(window), float(scale),
+                                              _ptr(gq), _ptr(gk), _ptr(gv), _ptr(gs))
+    if rc != 0:
+        raise ValueError("oracle prefill_backward: bad arguments")
+    return tuple(torch.from_numpy(x) for x in (gq, gk, gv, gs))

@@ -491,3 +491,102 @@ void sinkattn_oracle_fp8_decode(const uint8_t *codes, int64_t n, double *out)
     for (int64_t i = 0; i < n; ++i)
         out[i] = sinkattn_oracle_e4m3_value(codes[i]);
 }
+
+/*
+ * Backward of the whole-sequence prefill: the training variant. [ARCH] CH10.1 creates the sink
+ * parameter with requires_grad=False (it is not trained by gradient); its gradient is given
+ * here all the same, for a caller that does train it.
+ *
+ * With the forward of sink_softmax_row for row i of head h (p_j = exp(a_j - m) / D for the
+ * visible keys, p_s = exp(sink - m) / D for the sink, O = sum_j p_j v_j), and the incoming
+ * gradient dO of that row:
+ *   dp_j  = <dO, v_j>
+ *   delta = sum_j p_j dp_j = <dO, O>          (the sink carries no value: its dp is 0)
+ *   da_j  = p_j (dp_j - delta)                (softmax backward over the keys and the sink)
+ *   dsink_h += p_s (0 - delta)
+ *   dq_i  = scale * sum_j da_j k_j;   dk_j += scale * da_j q_i;   dv_j += p_j dO
+ * GQA: dk / dv of KV head g sum over its G query heads.
+ *
+ *   q, k, v, dout as prefill (bf16 bits; dout [B, L, Hq, dv]); gq [B,L,Hq,dq], gk [B,L,Hkv,dq],
+ *   gv [B,L,Hkv,dv], gsink [Hq] fp64 (written). Serial: the key gradients accumulate across rows.
+ */
+int sinkattn_oracle_prefill_backward(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                                     const float *sink, const uint16_t *dout, int B, int L,
+                                     int Hq, int Hkv, int dq, int dv, int window, double scale,
+                                     double *gq, double *gk, double *gv, double *gsink)
+{
+    if (B < 0 || L < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || window < 0)
+        return -1;
+    const int G = Hq / Hkv;
+    memset(gq, 0, sizeof(double) * (size_t)B * L * Hq * dq);
+    memset(gk, 0, sizeof(double) * (size_t)B * L * Hkv * dq);
+    memset(gv, 0, sizeof(double) * (size_t)B * L * Hkv * dv);
+    memset(gsink, 0, sizeof(double) * (size_t)Hq);
+    double *a = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
+    double *dp = (double *)malloc(sizeof(double) * (L > 0 ? L : 1));
+    double *o = (double *)malloc(sizeof(double) * dv);
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < L; ++i) {
+            const int lo = (window > 0 && i - window + 1 > 0) ? i - window + 1 : 0;
+            for (int h = 0; h < Hq; ++h) {
+                const int g = h / G;
+                const double s = head_sink(sink, h);
+                const uint16_t *qi = q + (((int64_t)b * L + i) * Hq + h) * dq;
+                const uint16_t *di = dout + (((int64_t)b * L + i) * Hq + h) * dv;
+                /* forward of the row */
+                double m = s;
+                for (int j = lo; j <= i; ++j) {
+                    const uint16_t *kj = k + (((int64_t)b * L + j) * Hkv + g) * dq;
+                    double dot = 0.0;
+                    for (int d = 0; d < dq; ++d)
+                        dot += bf16_to_f64(qi[d]) * bf16_to_f64(kj[d]);
+                    a[j] = scale * dot;
+                    if (a[j] > m)
+                        m = a[j];
+                }
+                double D = exp(s - m);
+                for (int j = lo; j <= i; ++j)
+                    D += exp(a[j] - m);
+                for (int e = 0; e < dv; ++e)
+                    o[e] = 0.0;
+                for (int j = lo; j <= i; ++j) {
+                    const uint16_t *vj = v + (((int64_t)b * L + j) * Hkv + g) * dv;
+                    const double p = exp(a[j] - m) / D;
+                    for (int e = 0; e < dv; ++e)
+                        o[e] += p * bf16_to_f64(vj[e]);
+                }
+                /* backward */
+                double delta = 0.0;
+                for (int e = 0; e < dv; ++e)
+                    delta += bf16_to_f64(di[e]) * o[e];
+                for (int j = lo; j <= i; ++j) {
+                    const uint16_t *vj = v + (((int64_t)b * L + j) * Hkv + g) * dv;
+                    double x = 0.0;
+                    for (int e = 0; e < dv; ++e)
+                        x += bf16_to_f64(di[e]) * bf16_to_f64(vj[e]);
+                    dp[j] = x;
+                }
+                const double ps = exp(s - m) / D;
+                gsink[h] += ps * (0.0 - delta);
+                double *gqi = gq + (((int64_t)b * L + i) * Hq + h) * dq;
+                for (int j = lo; j <= i; ++j) {
+                    const double p = exp(a[j] - m) / D;
+                    const double da = p * (dp[j] - delta);
+                    const uint16_t *kj = k + (((int64_t)b * L + j) * Hkv + g) * dq;
+                    double *gkj = gk + (((int64_t)b * L + j) * Hkv + g) * dq;
+                    double *gvj = gv + (((int64_t)b * L + j) * Hkv + g) * dv;
+                    for (int d = 0; d < dq; ++d) {
+                        gqi[d] += scale * da * bf16_to_f64(kj[d]);
+                        gkj[d] += scale * da * bf16_to_f64(qi[d]);
+                    }
+                    for (int e = 0; e < dv; ++e)
+                        gvj[e] += p * bf16_to_f64(di[e]);
+                }
+            }
+        }
+    }
+    free(a);
+    free(dp);
+    free(o);
+    return 0;
+}

@@ -51,6 +51,14 @@ MUTANTS = [
     ("e4m3 without saturation", "if (a >= 448.0)\n        return sign | 0x7e;",
      "if (a >= 464.0)\n        return sign | 0x7f;", 0),
     ("fp8 encode multiplies by the scale", "const float y = xi / scale;", "const float y = xi * scale;", 0),
+    ("backward drops delta", "const double da = p * (dp[j] - delta);", "const double da = p * dp[j];", 0),
+    ("backward sink gradient sign", "gsink[h] += ps * (0.0 - delta);", "gsink[h] += ps * delta;", 0),
+    ("backward dk without the scale", "gkj[d] += scale * da * bf16_to_f64(qi[d]);",
+     "gkj[d] += da * bf16_to_f64(qi[d]);", 0),
+    ("backward dv weighted by da", "gvj[e] += p * bf16_to_f64(di[e]);", "gvj[e] += da * bf16_to_f64(di[e]);", 0),
+    ("backward window one key too wide",
+     "const int lo = (window > 0 && i - window + 1 > 0) ? i - window + 1 : 0;\n            for (int h = 0; h < Hq; ++h) {\n                const int g = h / G;\n                const double s",
+     "const int lo = (window > 0 && i - window > 0) ? i - window : 0;\n            for (int h = 0; h < Hq; ++h) {\n                const int g = h / G;\n                const double s", 0),
 ]
 
 

@@ -642,3 +642,77 @@ def test_brute_force_tiny_decode():
                                    [x[1] for x in vis], float(sink[h]), scale)
                 assert max(abs(x - y) for x, y in zip(o[0, t, h].tolist(), ro)) < 1e-12
                 assert abs(lse[0, t, h].item() - rl) < 1e-12
+
+
+# ----------------------------------------------------------------------------------------------
+# backward (the training variant): gradients of sum(O * dO)
+# ----------------------------------------------------------------------------------------------
+
+def eager_grads(q, k, v, sink, dout, scale, window):
+    """Library autograd (fp64) through the eager concat -> softmax -> drop formulation."""
+    B, L, Hq, _ = q.shape
+    G = Hq // k.shape[2]
+    qd, kd, vd = (x.double().clone().requires_grad_(True) for x in (q, k, v))
+    sd = sink.double().clone().requires_grad_(True)
+    kr = kd.repeat_interleave(G, 2).permute(0, 2, 1, 3)          # [B, Hq, L, dq]
+    vr = vd.repeat_interleave(G, 2).permute(0, 2, 1, 3)
+    a = scale * qd.permute(0, 2, 1, 3) @ kr.transpose(-1, -2)     # [B, Hq, L, L]
+    a = a.masked_fill(~band_mask(L, window), float("-inf"))
+    col = sd.view(1, Hq, 1, 1).expand(B, Hq, L, 1)
+    w = torch.softmax(torch.cat([a, col], -1), -1)[..., :-1]
+    o = (w @ vr).permute(0, 2, 1, 3)
+    (o * dout.double()).sum().backward()
+    return qd.grad, kd.grad, vd.grad, sd.grad
+
+
+@pytest.mark.parametrize("L,window,Hq,Hkv", [(9, 0, 4, 2), (9, 3, 4, 2), (6, 1, 2, 2), (7, 0, 8, 1)])
+def test_backward_equals_library_autograd(L, window, Hq, Hkv):
+    g = torch.Generator().manual_seed(41 + L + window)
+    B = 2
+    q, k, v = rand_bf16((B, L, Hq, 192), g), rand_bf16((B, L, Hkv, 192), g), rand_bf16((B, L, Hkv, 128), g)
+    dout = rand_bf16((B, L, Hq, 128), g)
+    sink = torch.rand(Hq, generator=g) * 4 - 1
+    scale = 1.0 / math.sqrt(192)
+    ours = oracle.prefill_backward(q, k, v, sink, dout, scale, window)
+    ref = eager_grads(q, k, v, sink, dout, scale, window)
+    for name, x, y in zip(("dq", "dk", "dv", "dsink"), ours, ref):
+        assert torch.allclose(x, y, rtol=1e-10, atol=1e-11), name
+
+
+def test_backward_sink_by_central_differences():
+    """d/ds_h of sum(O * dO) against central differences of the (separately pinned) forward."""
+    g = torch.Generator().manual_seed(47)
+    B, L, Hq, Hkv = 1, 6, 2, 1
+    q, k, v = rand_bf16((B, L, Hq, 192), g), rand_bf16((B, L, Hkv, 192), g), rand_bf16((B, L, Hkv, 128), g)
+    dout = rand_bf16((B, L, Hq, 128), g)
+    sink = torch.tensor([0.3, 1.7], dtype=torch.float64)
+    scale = 1.0 / math.sqrt(192)
+    ds = oracle.prefill_backward(q, k, v, sink.float(), dout, scale, 0)[3]
+
+    def f(s):  # the forward oracle takes fp32 sinks: step in fp32-exact increments
+        o, _, _ = oracle.prefill(q, k, v, s.float(), scale, 0)
+        return (o * dout.double()).sum().item()
+    h = 2.0 ** -12
+    for hh in range(Hq):
+        e = torch.zeros(Hq, dtype=torch.float64)
+        e[hh] = h
+        num = (f(sink + e) - f(sink - e)) / (2 * h)
+        assert abs(num - ds[hh].item()) < 1e-5 * max(1.0, abs(num)), (hh, num, ds[hh].item())
+
+
+def test_backward_without_sink_equals_library_attention_backward():
+    """sink = -inf: no sink gradient, and dq / dk / dv equal the library's fp64 attention
+    backward (scaled_dot_product_attention, GQA)."""
+    g = torch.Generator().manual_seed(43)
+    B, L, Hq, Hkv = 2, 8, 4, 2
+    q, k, v = rand_bf16((B, L, Hq, 192), g), rand_bf16((B, L, Hkv, 192), g), rand_bf16((B, L, Hkv, 128), g)
+    dout = rand_bf16((B, L, Hq, 128), g)
+    scale = 1.0 / math.sqrt(192)
+    ours = oracle.prefill_backward(q, k, v, torch.full((Hq,), float("-inf")), dout, scale, 0)
+    qd, kd, vd = (to_bhld(x).clone().requires_grad_(True) for x in (q, k, v))
+    o = F.scaled_dot_product_attention(qd, kd, vd, attn_mask=band_mask(L, 0), scale=scale,
+                                       enable_gqa=True)
+    (o * to_bhld(dout)).sum().backward()
+    for x, y in zip(ours[:3], (qd.grad, kd.grad, vd.grad)):
+        assert torch.allclose(x, y.permute(0, 2, 1, 3), rtol=1e-10, atol=1e-11)
+    assert torch.all(ours[3] == 0)
