@@ -471,7 +471,8 @@ def cpu_baseline_prefill(w, d_cpu, target_s=12.0):
     flops, dt = oracle_prefill_sample(w, d_cpu, n, seed=n)
     return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": omp_threads(),
             "kind": "oracle", "seconds": round(dt, 2),
-            "sample": f"{n} random (batch, position) rows x all {w.Hq} heads of {w.name}"}
+            "sample": f"{n} random (batch, position) rows x all {w.Hq} heads of {w.name}",
+            "full_workload_s_extrapolated": round(prefill_counts(w)[0] / (flops / dt), 3)}
 
 
 def _cpu(t):

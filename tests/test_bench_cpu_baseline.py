@@ -68,3 +68,11 @@ def test_failure_is_reported_not_raised(bench):
     w = dataclasses.replace(W.GA_DECODE, B=2, ctx=10)
     e = bench.cpu_baseline_secondary("decode", runner(w, {}, 1, 1, "broken"))
     assert e["kind"] == "oracle" and "error" in e
+
+
+def test_headline_baseline_reports_its_extrapolation(bench):
+    w = dataclasses.replace(W.SWA_PREFILL, B=1, L=512)
+    d = W.prefill_inputs(w)
+    e = bench.cpu_baseline_prefill(w, d, target_s=0.2)
+    assert e["unit"] == "TFLOP/s" and e["value"] > 0 and e["kind"] == "oracle"
+    assert e["full_workload_s_extrapolated"] > 0
