@@ -35,6 +35,12 @@ MUTANTS = [
      "D += l_p[p] * exp(m_p[p] - m) + exp(sink - m);", 0),
     ("paged row ignores the page size", "*\n                                      page_size + c % page_size;",
      "+ c % page_size;", 0),
+    ("paged commit takes the page index modulo the page size",
+     "row = (int64_t)page_table[(int64_t)b * max_pages + c / page_size] * page_size +\n                      c % page_size;",
+     "row = (int64_t)page_table[(int64_t)b * max_pages + c % page_size] * page_size +\n                      c % page_size;", 0),
+    ("paged commit ignores the sequence's page-table row",
+     "row = (int64_t)page_table[(int64_t)b * max_pages + c / page_size] * page_size +\n                      c % page_size;",
+     "row = (int64_t)page_table[c / page_size] * page_size +\n                      c % page_size;", 0),
     ("commit ring overwrites the newest", "slot = ring_head[b];\n", "slot = (ring_head[b] + ring_cap - 1) % ring_cap;\n", 0),
     ("rope sine sign flipped", "yr[i] = a * cs - b * sn;", "yr[i] = a * cs + b * sn;", 0),
     ("rope frequency over the whole head dim", "pow(theta, -2.0 * i / rope_dim)",

@@ -392,6 +392,53 @@ def test_commit_ring_and_contig_semantics():
         assert torch.equal(k3[b, int(c3[b]):], kc3[b, int(c3[b]):])
 
 
+@pytest.mark.parametrize("accept", ["none", "one", "all"])
+def test_commit_paged_equals_contig(accept):
+    """The paged commit stores what the contiguous commit stores, through the page table.
+
+    ("MiMo-V2-Flash 模型架构深度拆解" CH10.3, the "KV cache update" step; the page table of the
+    serving stack, "MiMo-V2-Flash" model card.) Pages are handed out in a random permutation;
+    contexts start just before, on and after page boundaries so the accepted tokens cross one.
+    Checked two ways: the pool read back row by row through the table equals the contiguous
+    cache (and pages no sequence owns are untouched), and the oracle's decode over the grown
+    paged cache (its paged addressing pinned against prefill above) equals the decode over the
+    grown contiguous cache."""
+    g = torch.Generator().manual_seed(59)
+    B, T, Hq, Hkv, P, maxc = 4, 4, 4, 2, 8, 32
+    n = {"none": 0, "one": 1, "all": T}[accept]
+    acc = torch.full((B,), n, dtype=torch.int32)
+    ctx = torch.tensor([6, 8, 15, 0], dtype=torch.int32)
+    kn, vn = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    kc, vc = rand_bf16((B, maxc, Hkv, 192), g), rand_bf16((B, maxc, Hkv, 128), g)
+    max_pages = maxc // P
+    spare = 3  # pages in the pool that no sequence owns
+    perm = torch.randperm(B * max_pages + spare, generator=g).to(torch.int32)
+    table = perm[:B * max_pages].reshape(B, max_pages).contiguous()
+    kp = rand_bf16((B * max_pages + spare, P, Hkv, 192), g)
+    vp = rand_bf16((B * max_pages + spare, P, Hkv, 128), g)
+    for b in range(B):
+        for c in range(maxc):
+            kp[table[b, c // P], c % P] = kc[b, c]
+            vp[table[b, c // P], c % P] = vc[b, c]
+    k1, v1, _, _, c1 = oracle.commit(oracle.KV_CONTIG, kn, vn, acc, kc, vc, ctx_len=ctx)
+    k2, v2, _, _, c2 = oracle.commit(oracle.KV_PAGED, kn, vn, acc, kp, vp, ctx_len=ctx,
+                                     page_table=table, page_size=P)
+    assert torch.equal(c1, c2) and torch.equal(c1, ctx + acc)
+    for b in range(B):
+        for c in range(maxc):
+            assert torch.equal(k2[table[b, c // P], c % P], k1[b, c]), (b, c)
+            assert torch.equal(v2[table[b, c // P], c % P], v1[b, c]), (b, c)
+    for pg in perm[B * max_pages:].tolist():
+        assert torch.equal(k2[pg], kp[pg]) and torch.equal(v2[pg], vp[pg])
+    q = rand_bf16((B, T, Hq, 192), g)
+    kn2, vn2 = rand_bf16((B, T, Hkv, 192), g), rand_bf16((B, T, Hkv, 128), g)
+    sink = torch.rand(Hq, generator=g) * 6
+    a = oracle.decode(oracle.KV_CONTIG, q, kn2, vn2, k1, v1, sink, 0.07, 0, ctx_len=c1)
+    b_ = oracle.decode(oracle.KV_PAGED, q, kn2, vn2, k2, v2, sink, 0.07, 0, ctx_len=c2,
+                       page_table=table, page_size=P)
+    assert torch.equal(a[0], b_[0]) and torch.equal(a[1], b_[1])
+
+
 def test_workload_generators_are_seeded():
     a = W.prefill_inputs(W.SWA_PREFILL_SMALL, L=64)
     b = W.prefill_inputs(W.SWA_PREFILL_SMALL, L=64)
