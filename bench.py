@@ -624,6 +624,22 @@ def measure(runner, steps, warmup, flush, world):
     return max_over_ranks(ms)
 
 
+def compact_summary(result, secondary):
+    """{workload key: [ms per step, roofline fraction, bound, achieved, unit]} for the headline
+    and every secondary workload, plus the hybrid step's GA and SWA layers apart."""
+    def short(ms, rl):
+        return [ms, rl.get("frac"), rl.get("bound"), rl.get("achieved"), rl.get("unit")]
+
+    out = {}
+    if result.get("roofline"):
+        out["headline"] = short(result.get("ms_per_step"), result["roofline"])
+    for name, e in secondary.items():
+        out[name] = short(e["ms_per_step"], e["roofline"])
+        for kind, sub in e.get("by_kind", {}).items():
+            out[f"{name}.{kind}"] = short(sub["ms_per_step"], sub["roofline"])
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -783,6 +799,9 @@ def main():
             result["cpu_baseline"] = cpu_base
         if secondary:
             result["secondary"] = secondary
+            # the same figures in short, as the line's last key: a reader that keeps only the
+            # end of the output still sees every workload's time and roofline fraction
+            result["summary"] = compact_summary(result, secondary)
         print(json.dumps(result), flush=True)
     if world > 1:
         import torch.distributed as dist

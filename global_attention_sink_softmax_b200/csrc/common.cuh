@@ -8,9 +8,70 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #define SA_DEV __device__ __forceinline__
 
 namespace sinkattn {
+
+// ---------------------------------------------------------------------------------------------
+// Host: set-up that must happen once per CUDA context (kernel attributes, symbol addresses)
+// ---------------------------------------------------------------------------------------------
+// Process-unique id of the CUDA context current on this thread (cuCtxGetId), or 0 when none is
+// current yet. A context created after a device reset gets a new id even if its handle value
+// repeats, so set-up keyed on it is redone for the new context.
+inline unsigned long long current_context_id()
+{
+    typedef CUresult (*GetCurrentFn)(CUcontext *);
+    typedef CUresult (*GetIdFn)(CUcontext, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Runs a set-up step once per CUDA context of each device, from any number of host threads.
+// The step runs with the device current; if it fails, it is tried again on the next call.
+class PerContextOnce {
+  public:
+    template <class F> cudaError_t run(F &&setup)
+    {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess)
+            return e;
+        const bool cached = dev >= 0 && dev < kMaxDevices;
+        std::lock_guard<std::mutex> lock(mu_);
+        const unsigned long long id = current_context_id();
+        if (cached && id != 0 && ctx_[dev] == id)
+            return cudaSuccess;
+        e = setup(dev);
+        if (e == cudaSuccess && cached)
+            ctx_[dev] = current_context_id(); // the step may have created the context
+        return e;
+    }
+
+  private:
+    static constexpr int kMaxDevices = 256;
+    std::mutex mu_;
+    unsigned long long ctx_[kMaxDevices] = {};
+};
 
 // Device-side error flag: bit 0 = a prefill wait gave up, bit 1 = a decode wait gave up.
 // The library is built as one translation unit, so this is its only definition.

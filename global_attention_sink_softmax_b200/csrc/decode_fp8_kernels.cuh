@@ -449,12 +449,9 @@ __global__ void __launch_bounds__(d8::THREADS, 2) decode_fp8_kernel(const Decode
 
 cudaError_t launch_decode_fp8(const DecodeParams &p, cudaStream_t stream)
 {
-    static int configured_devices = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
-    if (dev < 32 && !(configured_devices & (1 << dev))) {
+    static PerContextOnce configured; // shared-memory opt-in, once per context
+    cudaError_t e = configured.run([](int) {
+        cudaError_t e = cudaSuccess;
         const void *fns[3] = {(const void *)decode_fp8_kernel<4>, (const void *)decode_fp8_kernel<2>,
                               (const void *)decode_fp8_kernel<1>};
         for (int i = 0; i < 3; ++i) {
@@ -462,8 +459,10 @@ cudaError_t launch_decode_fp8(const DecodeParams &p, cudaStream_t stream)
             if (e != cudaSuccess)
                 return e;
         }
-        configured_devices |= (1 << dev);
-    }
+        return e;
+    });
+    if (e != cudaSuccess)
+        return e;
     dim3 grid(p.splits, p.Hkv, p.B);
     if (p.MT == 1)
         decode_fp8_kernel<4><<<grid, d8::THREADS, d8::SMEM, stream>>>(p);

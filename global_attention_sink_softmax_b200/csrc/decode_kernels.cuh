@@ -478,12 +478,9 @@ int decode_stages(const DecodeParams &p);
 
 cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream)
 {
-    static int configured_devices = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
-    if (dev < 32 && !(configured_devices & (1 << dev))) {
+    static PerContextOnce configured; // shared-memory opt-in, once per context
+    cudaError_t e = configured.run([](int) {
+        cudaError_t e = cudaSuccess;
         const void *fns[6] = {(const void *)decode_split_kernel<4, 4>,
                               (const void *)decode_split_kernel<2, 4>,
                               (const void *)decode_split_kernel<1, 4>,
@@ -496,8 +493,10 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream)
             if (e != cudaSuccess)
                 return e;
         }
-        configured_devices |= (1 << dev);
-    }
+        return e;
+    });
+    if (e != cudaSuccess)
+        return e;
     e = decode_stages(p) == 2 ? launch_decode_split<2>(p, stream) : launch_decode_split<4>(p, stream);
     if (e != cudaSuccess || p.splits == 1)
         return e;

@@ -307,18 +307,13 @@ cudaError_t launch_decode_ring(const CUtensorMap &kc, const CUtensorMap &vc, con
                                const CUtensorMap &vn, const DecodeParams &p, int sms,
                                cudaStream_t stream)
 {
-    static int configured_devices = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static PerContextOnce configured; // shared-memory opt-in, once per context
+    cudaError_t e = configured.run([](int) {
+        return cudaFuncSetAttribute(decode_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    dr::SMEM_BYTES);
+    });
     if (e != cudaSuccess)
         return e;
-    if (dev < 32 && !(configured_devices & (1 << dev))) {
-        e = cudaFuncSetAttribute(decode_ring_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dr::SMEM_BYTES);
-        if (e != cudaSuccess)
-            return e;
-        configured_devices |= (1 << dev);
-    }
     const int items = p.B * p.Hkv * p.MT;
     const int ctas = (items + dr::WARPS - 1) / dr::WARPS;
     decode_ring_kernel<<<ctas < sms ? ctas : sms, dr::THREADS, dr::SMEM_BYTES, stream>>>(kc, vc, kn, vn, p);

@@ -423,12 +423,9 @@ cudaError_t launch_decode_tma_split(const CUtensorMap &kc, const CUtensorMap &vc
 cudaError_t launch_decode_tma(const CUtensorMap &kc, const CUtensorMap &vc, const CUtensorMap &kn,
                               const CUtensorMap &vn, const DecodeParams &p, cudaStream_t stream)
 {
-    static int configured_devices = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
-    if (dev < 32 && !(configured_devices & (1 << dev))) {
+    static PerContextOnce configured; // shared-memory opt-in, once per context
+    cudaError_t e = configured.run([](int) {
+        cudaError_t e = cudaSuccess;
         const void *fns[6] = {(const void *)decode_tma_kernel<4, 4>, (const void *)decode_tma_kernel<2, 4>,
                               (const void *)decode_tma_kernel<1, 4>, (const void *)decode_tma_kernel<4, 2>,
                               (const void *)decode_tma_kernel<2, 2>, (const void *)decode_tma_kernel<1, 2>};
@@ -438,8 +435,10 @@ cudaError_t launch_decode_tma(const CUtensorMap &kc, const CUtensorMap &vc, cons
             if (e != cudaSuccess)
                 return e;
         }
-        configured_devices |= (1 << dev);
-    }
+        return e;
+    });
+    if (e != cudaSuccess)
+        return e;
     e = decode_stages(p) == 2 ? launch_decode_tma_split<2>(kc, vc, kn, vn, p, stream)
                               : launch_decode_tma_split<4>(kc, vc, kn, vn, p, stream);
     if (e != cudaSuccess || p.splits == 1)

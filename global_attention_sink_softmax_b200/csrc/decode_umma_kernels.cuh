@@ -708,21 +708,17 @@ cudaError_t launch_decode_umma(const CUtensorMap &q, const CUtensorMap &kc, cons
                                const CUtensorMap &kn, const CUtensorMap &vn, const DecodeParams &p,
                                int max_ctas, cudaStream_t stream)
 {
-    static int configured_devices = 0;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return e;
-    if (dev < 32 && !(configured_devices & (1 << dev))) {
-        e = cudaFuncSetAttribute(decode_umma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 du::SMEM_BYTES);
+    static PerContextOnce configured; // shared-memory opt-in, once per context
+    cudaError_t e = configured.run([](int) {
+        cudaError_t e = cudaFuncSetAttribute(
+            decode_umma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, du::SMEM_BYTES);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(decode_umma_kernel<4>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, du::SMEM_BYTES);
-        if (e != cudaSuccess)
-            return e;
-        configured_devices |= (1 << dev);
-    }
+        return e;
+    });
+    if (e != cudaSuccess)
+        return e;
     const int n_items = p.splits * p.Hkv * p.B;
     const int grid = (max_ctas > 0 && max_ctas < n_items) ? max_ctas : n_items;
     if (p.R > 32)

@@ -386,18 +386,13 @@ cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                 const CUtensorMap &tmV, const PrefillParams &p,
                                 cudaStream_t stream)
 {
-    static int configured_devices = 0; // bit per device: shared-memory opt-in done
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static PerContextOnce configured; // shared-memory opt-in, once per context
+    cudaError_t e = configured.run([](int) {
+        return cudaFuncSetAttribute(prefill_band_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    pf::SMEM_BYTES);
+    });
     if (e != cudaSuccess)
         return e;
-    if (dev < 32 && !(configured_devices & (1 << dev))) {
-        e = cudaFuncSetAttribute(prefill_band_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 pf::SMEM_BYTES);
-        if (e != cudaSuccess)
-            return e;
-        configured_devices |= (1 << dev);
-    }
     const int64_t blocks = (int64_t)p.n_qtiles * p.B * p.Hq;
     if (blocks <= 0)
         return cudaSuccess;

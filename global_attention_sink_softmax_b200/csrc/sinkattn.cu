@@ -437,30 +437,38 @@ void fill_decode_params(DecodeParams &p, const sinkattn_decode_args *a, const Sp
 constexpr size_t kNoAllocWorkspaceBytes = SINKATTN_NOALLOC_WORKSPACE_BYTES;
 static __device__ __align__(256) float g_noalloc_workspace[kNoAllocWorkspaceBytes / sizeof(float)];
 
-constexpr int kMaxCachedDevices = 64;
 std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[kMaxCachedDevices] = {};
+constexpr int kMaxCachedDevices = 256;
+struct NoAllocAddress {
+    unsigned long long ctx; // context the address belongs to (0: none cached)
+    void *ptr;
+};
+NoAllocAddress g_noalloc_addr[kMaxCachedDevices] = {};
 
-// Device address of g_noalloc_workspace on the current device. Host code cannot use the
-// array's name as a device pointer, so the address is looked up with cudaGetSymbolAddress the
-// first time a device needs it (with that device current) and kept per device.
+// Device address of g_noalloc_workspace in the current device's context. Host code cannot use
+// the array's name as a device pointer, so the address is looked up with cudaGetSymbolAddress
+// the first time a context needs it (with its device current) and kept per device together
+// with that context's id: after a device reset the new context's module is loaded afresh, its
+// id differs, and the address is looked up again.
 cudaError_t noalloc_workspace_ptr(void **out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
+    const bool cached = dev >= 0 && dev < kMaxCachedDevices;
     std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (dev >= 0 && dev < kMaxCachedDevices && g_noalloc_ptr[dev]) {
-        *out = g_noalloc_ptr[dev];
+    const unsigned long long ctx = current_context_id();
+    if (cached && ctx != 0 && g_noalloc_addr[dev].ctx == ctx) {
+        *out = g_noalloc_addr[dev].ptr;
         return cudaSuccess;
     }
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_workspace);
     if (e != cudaSuccess)
         return e;
-    if (dev >= 0 && dev < kMaxCachedDevices)
-        g_noalloc_ptr[dev] = p;
+    if (cached)
+        g_noalloc_addr[dev] = NoAllocAddress{current_context_id(), p};
     *out = p;
     return cudaSuccess;
 }

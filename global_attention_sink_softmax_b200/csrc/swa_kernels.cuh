@@ -449,22 +449,17 @@ cudaError_t launch_prefill_swa_packed(const CUtensorMap &tmQ, const CUtensorMap 
                                       const CUtensorMap &tmVc, const SwaParams &p, int grid,
                                       cudaStream_t stream)
 {
-    static int configured_devices = 0; // bit per device: shared-memory opt-in done
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static PerContextOnce configured; // shared-memory opt-in, once per context
+    cudaError_t e = configured.run([](int dev) {
+        int optin = 0;
+        cudaError_t e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess)
+            return e;
+        return cudaFuncSetAttribute(prefill_swa_packed_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
+    });
     if (e != cudaSuccess)
         return e;
-    if (dev < 32 && !(configured_devices & (1 << dev))) {
-        int optin = 0;
-        e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-        if (e != cudaSuccess)
-            return e;
-        e = cudaFuncSetAttribute(prefill_swa_packed_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, optin);
-        if (e != cudaSuccess)
-            return e;
-        configured_devices |= (1 << dev);
-    }
     if (grid <= 0)
         return cudaSuccess;
     prefill_swa_packed_kernel<<<grid, sw::THREADS, sw::smem_bytes(p.P), stream>>>(

@@ -29,7 +29,8 @@
  *     stride in bytes must be multiples of 16.
  *   - Head dims: dq = 192 and dv = 128 for attention and commit (the kernels are specialised
  *     for them); sinkattn_rope_qkv states its own limits.
- *     GQA group G = Hq / Hkv must be an integer in 1..16 (prefill) or 1..16 (decode).
+ *     GQA group G = Hq / Hkv must be an integer; decode and commit take G in 1..16 with
+ *     T * G <= 64 query rows per KV head, prefill any G.
  *   - sink: fp32 [Hq] in post-scale logit units (not multiplied by scale). NULL means no sink
  *     for any head; an entry of -inf means plain softmax for that head. NaN or +inf entries
  *     give unspecified results (not checked).
@@ -37,8 +38,11 @@
  *     May be NULL.
  *   - scale: finite and > 0 (1/sqrt(192) for the pages' model).
  *   - Ownership: the caller allocates and owns every buffer, host- and device-side. The
- *     library allocates nothing and keeps no per-call state; decode scratch is a caller
- *     workspace. All device pointers must be device memory of the current device.
+ *     library allocates nothing at run time and keeps no state between calls in the caller's
+ *     memory; decode scratch is a caller workspace. Its only device state is process-wide and
+ *     lives in the library's own module: the wait-timeout flag read by
+ *     sinkattn_take_device_error, and the fixed scratch array of sinkattn_decode_noalloc. All
+ *     device pointers must be device memory of the current device.
  *   - Streams: `stream` is a cudaStream_t (NULL = legacy default stream). Work is enqueued on
  *     it; nothing synchronises the host. Returns after the launch.
  *   - Errors: every entry point returns a sinkattn_status. Arguments are validated on the host
@@ -116,7 +120,10 @@ typedef struct sinkattn_prefill_args {
  * QA" Q3.6). */
 int sinkattn_prefill_swa(const sinkattn_prefill_args *args, int32_t window, void *stream);
 
-/* Global (full causal) prefill (GA). Key tiles above the diagonal are skipped. */
+/* Global (full causal) prefill (GA): every position sees itself and all earlier positions
+ * ("MiMo-V2-Flash 模型架构深度拆解" CH10.3, the GA layers' causal mask; CH10.1, the GA layers'
+ * sink is optional and off in the model's config, so a NULL or -inf sink gives plain causal
+ * softmax). Key tiles above the diagonal are skipped. */
 int sinkattn_prefill_ga(const sinkattn_prefill_args *args, void *stream);
 
 /* Chunked prefill against cached keys: a long prompt prefilled in chunks (the serving command of
@@ -194,7 +201,11 @@ typedef struct sinkattn_decode_args {
     float k_scale, v_scale;
 } sinkattn_decode_args;
 
-/* Bytes of device workspace sinkattn_decode needs for these arguments (split-KV partials:
+/* Bytes of device workspace sinkattn_decode needs for these arguments. The pages give no
+ * decode algorithm, only its setting: contexts of up to 256K tokens, where decode time goes to
+ * reading the KV cache ("MiMo-V2-Flash Technical Report" paper notes §1.1). A long GA context is
+ * therefore split into key spans read in parallel, whose sink-free partials the merge described
+ * at sinkattn_decode combines; this is the room those partials take (split-KV partials:
  * per split and query row, an unnormalised fp32 O row, its running max and two running sums,
  * one over the bf16-rounded P that multiplied V and one over fp32 P). 0 when no split is
  * needed. Depends only on kind, B, T, Hq, Hkv, dq, dv, window, ring_cap / max_ctx and the page
