@@ -181,7 +181,8 @@ class DecodeRunner:
         if fp8:
             self.kernel = "decode_fp8_kernel"
         elif w.kind == W.KV_RING:
-            self.kernel = "decode_ring_kernel" if rows <= 16 else "decode_split_kernel"
+            self.kernel = ("decode_ring_kernel" if rows <= 16 and w.ring_cap % 32 == 0
+                           else "decode_split_kernel")
         elif w.kind == W.KV_PAGED and w.page_size % 64 != 0:
             self.kernel = "decode_split_kernel"
         else:
@@ -657,7 +658,7 @@ def main():
     ap.add_argument("--small", action="store_true",
                     help="profiling case: prefill workloads at B=1 (SWA L=16384, GA L=8192), "
                          "decode at B=2, SWA decode at B=64, hybrid verify as its first GA "
-                         "layer alone at B=8")
+                         "layer alone at B=8 and its first SWA layer alone")
     args = ap.parse_args()
     world, rank, local = init_dist(args)
     args.gpus = max(args.gpus, world)
@@ -755,6 +756,9 @@ def main():
             hyb0 = W.hybrid_layer_workload(0)
             hyb0 = dataclasses.replace(hyb0, B=8, name=hyb0.name + "_small_B8")
             jobs.append(("hybrid_ga_layer", lambda: DecodeRunner(hyb0, dev), None))
+            # one SWA layer of the step at its full size (B=64; 43 MB, flushed between steps)
+            jobs.append(("hybrid_swa_layer",
+                         lambda: DecodeRunner(W.hybrid_layer_workload(1), dev), "flush"))
         for name, make, fl in jobs:
             r = make()
             flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev) if fl else None

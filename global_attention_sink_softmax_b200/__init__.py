@@ -28,6 +28,7 @@ __all__ = [
     "sinkattn_status_string", "sinkattn_version", "EXPORTED_SYMBOLS",
     "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES", "sinkattn_rope_qkv",
     "ROPE_THETA_GA", "ROPE_THETA_SWA", "V_SCALE", "KV_BF16", "KV_FP8_E4M3",
+    "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward",
 ]
 
 KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
@@ -41,6 +42,8 @@ EXPORTED_SYMBOLS = [
     "sinkattn_prefill_swa", "sinkattn_prefill_ga", "sinkattn_prefill_chunk",
     "sinkattn_decode_workspace_size", "sinkattn_decode", "sinkattn_kv_commit", "sinkattn_status_string", "sinkattn_version",
     "sinkattn_take_device_error", "sinkattn_decode_noalloc", "sinkattn_rope_qkv",
+    "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward_workspace_size",
+    "sinkattn_prefill_backward",
 ]
 # Size of the library's own split-KV workspace used by sinkattn_decode_noalloc.
 NOALLOC_WORKSPACE_BYTES = 16 << 20
@@ -76,6 +79,15 @@ class RopeArgs(ctypes.Structure):
                 ("v_sb", _I64), ("v_sl", _I64), ("v_sh", _I64)]
 
 
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [("q", _P), ("k", _P), ("v", _P), ("o", _P), ("dout", _P), ("lse", _P),
+                ("sink", _P), ("dq", _P), ("dk", _P), ("dv", _P), ("dsink", _P),
+                ("B", _I32), ("L", _I32), ("Hq", _I32), ("Hkv", _I32), ("d_qk", _I32),
+                ("d_v", _I32), ("scale", _F32)] + [
+                (f"{t}_{s}", _I64) for t in ("q", "k", "v", "o", "do", "dq", "dk", "dv")
+                for s in ("sb", "sl", "sh")]
+
+
 class DecodeArgs(ctypes.Structure):
     _fields_ = [("kind", _I32), ("B", _I32), ("T", _I32), ("Hq", _I32), ("Hkv", _I32),
                 ("dq", _I32), ("dv", _I32), ("window", _I32), ("scale", _F32), ("sink", _P),
@@ -89,7 +101,9 @@ class DecodeArgs(ctypes.Structure):
                 ("page_table", _P), ("page_size", _I32), ("max_pages", _I32),
                 ("num_pages", _I32),
                 ("o", _P), ("o_sb", _I64), ("o_st", _I64), ("o_sh", _I64), ("lse", _P),
-                ("kv_dtype", _I32), ("k_scale", _F32), ("v_scale", _F32)]
+                ("kv_dtype", _I32), ("k_scale", _F32), ("v_scale", _F32),
+                ("commit_rope", _I32), ("rope_dim", _I32), ("rope_theta", ctypes.c_double),
+                ("commit_v_scale", _F32), ("commit_pos", _P)]
 
 
 _lock = threading.Lock()
@@ -128,6 +142,12 @@ def lib() -> ctypes.CDLL:
             L.sinkattn_take_device_error.restype = ctypes.c_int
             L.sinkattn_rope_qkv.argtypes = [ctypes.POINTER(RopeArgs), _P]
             L.sinkattn_rope_qkv.restype = ctypes.c_int
+            L.sinkattn_prefill_backward_workspace_size.argtypes = [ctypes.POINTER(BackwardArgs)]
+            L.sinkattn_prefill_backward_workspace_size.restype = _SZ
+            L.sinkattn_prefill_backward.argtypes = [ctypes.POINTER(BackwardArgs), _I32, _P, _SZ, _P]
+            L.sinkattn_prefill_backward.restype = ctypes.c_int
+            L.sinkattn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.sinkattn_set_wait_limit_ns.restype = ctypes.c_int
             _lib = L
     return _lib
 
@@ -377,16 +397,24 @@ def sinkattn_decode_noalloc(kind, q, k_new, v_new, k_cache, v_cache, sink=None, 
 
 def sinkattn_kv_commit(kind, k_new, v_new, n_accept, k_cache, v_cache, *, ring_head=None,
                        ring_len=None, ctx_len=None, max_ctx=None, page_table=None,
-                       num_pages=None, stream=None, k_scale=None, v_scale=None):
+                       num_pages=None, stream=None, k_scale=None, v_scale=None,
+                       rope_theta=None, rope_dim=ROPE_DIM, commit_v_scale=V_SCALE, pos=None):
     """Append the first n_accept[b] of each sequence's T new tokens to its cache, in place.
     Into an FP8 cache (uint8 / float8_e4m3fn) each element x is stored as the E4M3 code of
-    x / scale (k_scale for K, v_scale for V)."""
+    x / scale (k_scale for K, v_scale for V).
+    rope_theta given: K is stored with the partial rotary embedding of its first rope_dim dims at
+    position pos[b] + u (pos: int32 [B]; None = ctx_len before the commit, not for a ring) and V
+    multiplied by commit_v_scale, as sinkattn_rope_qkv would; k_new / v_new are not modified."""
     _check_vec("n_accept", n_accept, torch.int32)
+    _check_vec("pos", pos, torch.int32)
     B, T, Hkv, dq = k_new.shape
     q_dummy = k_new  # only the cache-related fields are read
     a = _decode_args(kind, q_dummy, k_new, v_new, k_cache, v_cache, None, 0, 1.0, ring_head,
                      ring_len, ctx_len, max_ctx, page_table, None, num_pages, None, None,
                      k_scale, v_scale)
+    if rope_theta is not None:
+        a.commit_rope, a.rope_dim, a.rope_theta = 1, int(rope_dim), float(rope_theta)
+        a.commit_v_scale, a.commit_pos = float(commit_v_scale), _ptr(pos)
     st = lib().sinkattn_kv_commit(ctypes.byref(a), _ptr(n_accept), _stream(stream))
     _raise(st, "sinkattn_kv_commit")
 
@@ -435,3 +463,52 @@ def sinkattn_take_device_error() -> int:
     flag = ctypes.c_uint32(0)
     _raise(lib().sinkattn_take_device_error(ctypes.byref(flag)), "sinkattn_take_device_error")
     return int(flag.value)
+
+
+def sinkattn_prefill_backward(q, k, v, o, lse, dout, sink=None, *, window=0, scale=None,
+                              dq=None, dk=None, dv=None, dsink=True, workspace=None, stream=None):
+    """Gradients of the whole-sequence prefill (the training variant): given the forward's
+    q, k, v, its output o and lse ([B, Hq, L]) and dout = dLoss/dO, returns (dq, dk, dv, dsink)
+    as fp32 tensors (dq [B,L,Hq,192], dk [B,L,Hkv,192], dv [B,L,Hkv,128], dsink [Hq] or None
+    when dsink=False). window 0: GA, >= 1: SWA."""
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _check_bf16(n, t)
+    _check_vec("sink", sink, torch.float32)
+    if lse.dtype != torch.float32 or not lse.is_cuda or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous CUDA float32 tensor [B, Hq, L]")
+    B, L, Hq, dqk = q.shape
+    Hkv, dvv = k.shape[2], v.shape[3]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dqk)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(B, L, Hq, dqk, **f32) if dq is None else dq
+    dk = torch.empty(B, L, Hkv, dqk, **f32) if dk is None else dk
+    dv = torch.empty(B, L, Hkv, dvv, **f32) if dv is None else dv
+    ds = (torch.empty(Hq, **f32) if dsink is True else dsink) if dsink is not False else None
+    a = BackwardArgs()
+    a.q, a.k, a.v, a.o, a.dout, a.lse = _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse)
+    a.sink, a.dq, a.dk, a.dv, a.dsink = _ptr(sink), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ds)
+    a.B, a.L, a.Hq, a.Hkv, a.d_qk, a.d_v, a.scale = B, L, Hq, Hkv, dqk, dvv, float(scale)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("do", dout), ("dq", dq), ("dk", dk),
+                    ("dv", dv)):
+        if t.stride(-1) != 1:
+            raise ValueError(f"{name}: the last dim must be contiguous")
+        setattr(a, f"{name}_sb", t.stride(0))
+        setattr(a, f"{name}_sl", t.stride(1))
+        setattr(a, f"{name}_sh", t.stride(2))
+    L_ = lib()
+    need = int(L_.sinkattn_prefill_backward_workspace_size(ctypes.byref(a)))
+    if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if need > 0 else None
+    ws_bytes = workspace.numel() * workspace.element_size() if need > 0 else 0
+    _raise(L_.sinkattn_prefill_backward(ctypes.byref(a), int(window), ws_ptr, ws_bytes,
+                                        _stream(stream)), "sinkattn_prefill_backward")
+    return dq, dk, dv, ds
+
+
+def sinkattn_set_wait_limit_ns(ns: int) -> None:
+    """How long a kernel on the current device waits on an internal barrier before it gives up
+    and records it in the wait-timeout flag (default 10**9 ns; 0 gives up at the first wait that
+    is not already satisfied). Process-wide per device; synchronises the device first."""
+    _raise(lib().sinkattn_set_wait_limit_ns(int(ns)), "sinkattn_set_wait_limit_ns")

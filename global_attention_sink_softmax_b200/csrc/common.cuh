@@ -80,8 +80,11 @@ __device__ uint32_t g_device_error = 0;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // A wait on an mbarrier that takes longer than this is treated as a fault: the kernel records
-// it and leaves. Legitimate waits here last microseconds.
+// it and leaves. Legitimate waits here last microseconds. The limit of the waits that give up
+// is g_wait_limit_ns (set per device by sinkattn_set_wait_limit_ns; 0 gives up at the first wait
+// whose first try fails); a CTA's final waits for its own copies and MMAs keep this one.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+__constant__ uint64_t g_wait_limit_ns = kWaitLimitNs;
 
 SA_DEV uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
@@ -143,21 +146,25 @@ SA_DEV bool mbar_test(uint64_t *bar, uint32_t parity)
 }
 
 // Waits for the phase with the given parity to complete. Gives up (returns false) when
-// *abort is set by another thread, or after kWaitLimitNs, in which case it sets *abort and
-// the device error bit `err_bit`.
+// *abort is set by another thread, or after g_wait_limit_ns, in which case it sets *abort and
+// the device error bit `err_bit`. The limit is only read once the first try has failed, so a
+// wait that finds its phase complete costs one instruction; a limit of 0 gives up at that point.
 SA_DEV bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t err_bit)
 {
     if (mbar_try_wait(bar, parity))
         return true;
+    const uint64_t limit = g_wait_limit_ns;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
+        if (limit != 0) {
 #pragma unroll 1
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity))
-                return true;
+            for (int i = 0; i < 32; ++i)
+                if (mbar_try_wait(bar, parity))
+                    return true;
+        }
         if (*abort)
             return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 >= limit) {
             *abort = 1;
             atomicOr(&g_device_error, err_bit);
             return false;
@@ -412,6 +419,55 @@ SA_DEV uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Partial rotary embedding and value scale on 8-element bf16 pieces (the RoPE pass and the
+// commit share these, so both give the same bits)
+// ---------------------------------------------------------------------------------------------
+// (cos, sin) of the angle m * w, w = theta^(-2i/rope_dim) given in fp64. The angle is formed in
+// fp64 and reduced to [-pi, pi] by subtracting the nearest multiple of 2 pi, with 2 pi split into
+// a leading and a trailing fp64 part (Cody and Waite's additive range reduction); only then is
+// it rounded to fp32 for sincosf. At position 262143 the fp32 product alone would be off by
+// ~0.016 rad.
+SA_DEV float2 rope_cos_sin(int64_t m, double w)
+{
+    // 2 pi = k2PiHi + k2PiLo: k2PiHi is 2 pi rounded to fp64, k2PiLo what that rounding lost
+    const double k2PiHi = 6.283185307179586232, k2PiLo = 2.4492935982947064e-16;
+    const double kInv2Pi = 0.15915494309189533577;
+    const double angle = (double)m * w;
+    const double n2pi = rint(angle * kInv2Pi);
+    const double red = fma(-n2pi, k2PiLo, fma(-n2pi, k2PiHi, angle));
+    float s, c;
+    sincosf((float)red, &s, &c);
+    return make_float2(c, s);
+}
+
+// Rotates 8 dimension pairs: a holds x_i (i = i0 .. i0 + 7 of the first rotary half), b the
+// partners x_{i + rope_dim/2}; cs[j] = (cos, sin) of pair i0 + j. In fp32, each result rounded
+// once to bf16 (nearest even):
+//     y_i = x_i cos - x_{i+h} sin,   y_{i+h} = x_{i+h} cos + x_i sin.
+SA_DEV void rope_rotate8(uint4 &a, uint4 &b, const float2 *cs)
+{
+    uint32_t *wa = reinterpret_cast<uint32_t *>(&a);
+    uint32_t *wb = reinterpret_cast<uint32_t *>(&b);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 c0 = cs[2 * j], c1 = cs[2 * j + 1];
+        const float x0 = __uint_as_float(wa[j] << 16), x1 = __uint_as_float(wa[j] & 0xffff0000u);
+        const float y0 = __uint_as_float(wb[j] << 16), y1 = __uint_as_float(wb[j] & 0xffff0000u);
+        wa[j] = pack_bf16x2(fmaf(x0, c0.x, -y0 * c0.y), fmaf(x1, c1.x, -y1 * c1.y));
+        wb[j] = pack_bf16x2(fmaf(y0, c0.x, x0 * c0.y), fmaf(y1, c1.x, x1 * c1.y));
+    }
+}
+
+// 8 bf16 values times s, each rounded once to bf16.
+SA_DEV void scale8(uint4 &a, float s)
+{
+    uint32_t *w = reinterpret_cast<uint32_t *>(&a);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        w[j] = pack_bf16x2(__uint_as_float(w[j] << 16) * s, __uint_as_float(w[j] & 0xffff0000u) * s);
 }
 
 // Sum of the two bf16 halves of a packed pair, as fp32 (bf16 -> fp32 is exact).

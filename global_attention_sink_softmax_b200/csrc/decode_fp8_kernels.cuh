@@ -476,75 +476,47 @@ cudaError_t launch_decode_fp8(const DecodeParams &p, cudaStream_t stream)
     return launch_decode_merge(p, stream);
 }
 
-// Commit into an FP8 cache: as kv_commit_kernel, each 8-element piece of a new token's bf16
-// K / V row quantised to 8 codes (the same rule as the decode's load of new tokens).
-__global__ void __launch_bounds__(128) kv_commit_fp8_kernel(const CommitParams p)
+// Commit into an FP8 cache: as kv_commit_kernel (the same pieces, rotated / scaled first when
+// the commit transforms), each 8-value bf16 piece quantised to 8 codes by the decode's rule for
+// new tokens.
+SA_DEV uint2 quant_piece(const uint4 &x, float scale)
+{
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+        c[j] = quant_e4m3x2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u), scale);
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+__global__ void __launch_bounds__(128) kv_commit_fp8_kernel(const __grid_constant__ CommitParams p)
 {
     const int b = blockIdx.x;
-    const int n = max(0, min(p.n_accept[b], p.T));
-    int head = 0, len = 0, ctx = 0;
-    if (p.kind == 0) {
-        head = ((p.ring_head[b] % p.ring_cap) + p.ring_cap) % p.ring_cap;
-        len = max(0, min(p.ring_len[b], p.ring_cap));
-    } else {
-        ctx = max(0, min(p.ctx_len[b], p.max_ctx));
-    }
+    const CommitState cs = commit_state(p, b);
     uint8_t *k8 = reinterpret_cast<uint8_t *>(p.k_cache);
     uint8_t *v8 = reinterpret_cast<uint8_t *>(p.v_cache);
-    const int per_tok = p.Hkv * 40; // 8-element pieces: 24 of K + 16 of V per head
-    for (int i = threadIdx.x; i < n * per_tok; i += blockDim.x) {
+    const int pph = commit_pieces_per_head(p);
+    const int per_tok = p.Hkv * pph;
+    const int64_t pos0 = p.pos ? (int64_t)p.pos[b] : (int64_t)cs.ctx;
+    for (int i = threadIdx.x; i < cs.n * per_tok; i += blockDim.x) {
         const int u = i / per_tok;
         const int rem = i - u * per_tok;
-        const int gh = rem / 40, ch = rem % 40;
+        const int gh = rem / pph;
+        const CommitPiece pc = commit_piece(p, rem - gh * pph);
         int64_t kdst, vdst;
-        if (p.kind == 0) {
-            const int slot = (head + len + u) % p.ring_cap;
-            kdst = (int64_t)b * p.kc_sb + (int64_t)slot * p.kc_ss;
-            vdst = (int64_t)b * p.vc_sb + (int64_t)slot * p.vc_ss;
-        } else if (p.kind == 1) {
-            const int pos = ctx + u;
-            if (pos >= p.max_ctx)
-                continue;
-            kdst = (int64_t)b * p.kc_sb + (int64_t)pos * p.kc_ss;
-            vdst = (int64_t)b * p.vc_sb + (int64_t)pos * p.vc_ss;
-        } else {
-            const int pos = ctx + u;
-            const int pg = pos / p.page_size;
-            if (pos >= p.max_ctx || pg >= p.max_pages)
-                continue;
-            const int pid = p.page_table[(int64_t)b * p.max_pages + pg];
-            if (pid < 0 || pid >= p.num_pages)
-                continue;
-            const int rr = pos - pg * p.page_size;
-            kdst = (int64_t)pid * p.kc_sb + (int64_t)rr * p.kc_ss;
-            vdst = (int64_t)pid * p.vc_sb + (int64_t)rr * p.vc_ss;
-        }
-        const bool is_k = ch < 24;
-        const uint16_t *src =
-            is_k ? p.k_new + (int64_t)b * p.kn_sb + (int64_t)u * p.kn_st + (int64_t)gh * p.kn_sh + ch * 8
-                 : p.v_new + (int64_t)b * p.vn_sb + (int64_t)u * p.vn_st + (int64_t)gh * p.vn_sh +
-                       (ch - 24) * 8;
-        uint8_t *dst = is_k ? k8 + kdst + (int64_t)gh * p.kc_sh + ch * 8
-                            : v8 + vdst + (int64_t)gh * p.vc_sh + (ch - 24) * 8;
-        const float scale = is_k ? p.k_scale : p.v_scale;
-        const uint4 x = *reinterpret_cast<const uint4 *>(src);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t c[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-            c[j] = quant_e4m3x2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xffff0000u), scale);
-        *reinterpret_cast<uint2 *>(dst) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+        if (!commit_dst(p, b, u, cs.head, cs.len, cs.ctx, kdst, vdst))
+            continue;
+        uint4 x0, x1;
+        commit_load(p, pc, b, u, gh, pos0 + u, x0, x1);
+        uint8_t *row = pc.is_k ? k8 + kdst + (int64_t)gh * p.kc_sh : v8 + vdst + (int64_t)gh * p.vc_sh;
+        const float scale = pc.is_k ? p.k_scale : p.v_scale;
+        *reinterpret_cast<uint2 *>(row + pc.c0 * 8) = quant_piece(x0, scale);
+        if (pc.c1 >= 0)
+            *reinterpret_cast<uint2 *>(row + pc.c1 * 8) = quant_piece(x1, scale);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        if (p.kind == 0) {
-            const int over = max(0, len + n - p.ring_cap);
-            p.ring_len[b] = min(p.ring_cap, len + n);
-            p.ring_head[b] = (head + over) % p.ring_cap;
-        } else {
-            p.ctx_len[b] = min(ctx + n, p.max_ctx);
-        }
-    }
+    if (threadIdx.x == 0)
+        commit_advance(p, b, cs);
 }
 
 cudaError_t launch_commit_fp8(const CommitParams &p, cudaStream_t stream)

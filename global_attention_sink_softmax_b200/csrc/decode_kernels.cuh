@@ -507,74 +507,148 @@ cudaError_t launch_decode(const DecodeParams &p, cudaStream_t stream)
 // Cache commit: one CTA per sequence copies its accepted tokens, then thread 0 advances that
 // sequence's ring head / length or context length (only this CTA reads them).
 // ---------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) kv_commit_kernel(const CommitParams p)
+// The work of one thread: one 16-byte piece (8 values) of a new token's K or V head row, or,
+// when the commit rotates K, the two K pieces c and c + rope_half / 8 whose dims are the rotation
+// pairs (i, i + rope_dim / 2).
+struct CommitPiece {
+    int is_k, c0, c1; // c1 < 0: one piece
+};
+
+SA_DEV int commit_pieces_per_head(const CommitParams &p) { return 24 - p.rope_half / 8 + 16; }
+
+SA_DEV CommitPiece commit_piece(const CommitParams &p, int idx)
+{
+    const int nrp = p.rope_half / 8; // rotated piece pairs
+    const int nk = 24 - nrp;         // K work items: the pairs, then the unrotated pieces
+    if (idx < nrp)
+        return CommitPiece{1, idx, idx + nrp};
+    if (idx < nk)
+        return CommitPiece{1, idx + nrp, -1};
+    return CommitPiece{0, idx - nk, -1};
+}
+
+// The piece(s) of new token u, KV head gh, of sequence b as the cache stores them: rotated at
+// position `pos` (a K pair) or multiplied by v_mul (V, when the commit transforms), else as
+// given. The arithmetic is the RoPE pass's, so both give the same bits.
+SA_DEV void commit_load(const CommitParams &p, const CommitPiece &pc, int b, int u, int gh,
+                        int64_t pos, uint4 &x0, uint4 &x1)
+{
+    const uint16_t *row =
+        pc.is_k ? p.k_new + (int64_t)b * p.kn_sb + (int64_t)u * p.kn_st + (int64_t)gh * p.kn_sh
+                : p.v_new + (int64_t)b * p.vn_sb + (int64_t)u * p.vn_st + (int64_t)gh * p.vn_sh;
+    x0 = *reinterpret_cast<const uint4 *>(row + pc.c0 * 8);
+    if (pc.c1 >= 0) {
+        x1 = *reinterpret_cast<const uint4 *>(row + pc.c1 * 8);
+        float2 cs[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            cs[j] = rope_cos_sin(pos, p.inv_freq[pc.c0 * 8 + j]);
+        rope_rotate8(x0, x1, cs);
+    } else if (!pc.is_k && p.rope_half > 0) {
+        scale8(x0, p.v_mul);
+    }
+}
+
+// Where token u of sequence b goes: its K and V row offsets (elements for a bf16 cache, bytes
+// for an FP8 one); false if it falls outside the cache (dropped).
+SA_DEV bool commit_dst(const CommitParams &p, int b, int u, int head, int len, int ctx,
+                       int64_t &kdst, int64_t &vdst)
+{
+    if (p.kind == 0) {
+        const int slot = (head + len + u) % p.ring_cap;
+        kdst = (int64_t)b * p.kc_sb + (int64_t)slot * p.kc_ss;
+        vdst = (int64_t)b * p.vc_sb + (int64_t)slot * p.vc_ss;
+        return true;
+    }
+    const int pos = ctx + u;
+    if (pos >= p.max_ctx)
+        return false;
+    if (p.kind == 1) {
+        kdst = (int64_t)b * p.kc_sb + (int64_t)pos * p.kc_ss;
+        vdst = (int64_t)b * p.vc_sb + (int64_t)pos * p.vc_ss;
+        return true;
+    }
+    const int pg = pos / p.page_size;
+    if (pg >= p.max_pages)
+        return false;
+    const int pid = p.page_table[(int64_t)b * p.max_pages + pg];
+    if (pid < 0 || pid >= p.num_pages)
+        return false;
+    const int rr = pos - pg * p.page_size;
+    kdst = (int64_t)pid * p.kc_sb + (int64_t)rr * p.kc_ss;
+    vdst = (int64_t)pid * p.vc_sb + (int64_t)rr * p.vc_ss;
+    return true;
+}
+
+// The sequence's cache state before the commit, and the advance after it (thread 0, once every
+// thread of the CTA is done).
+struct CommitState {
+    int head, len, ctx, n;
+};
+
+SA_DEV CommitState commit_state(const CommitParams &p, int b)
+{
+    CommitState c{0, 0, 0, max(0, min(p.n_accept[b], p.T))};
+    if (p.kind == 0) {
+        c.head = ((p.ring_head[b] % p.ring_cap) + p.ring_cap) % p.ring_cap;
+        c.len = max(0, min(p.ring_len[b], p.ring_cap));
+    } else {
+        c.ctx = max(0, min(p.ctx_len[b], p.max_ctx));
+    }
+    return c;
+}
+
+SA_DEV void commit_advance(const CommitParams &p, int b, const CommitState &c)
+{
+    if (p.kind == 0) {
+        const int over = max(0, c.len + c.n - p.ring_cap);
+        p.ring_len[b] = min(p.ring_cap, c.len + c.n);
+        p.ring_head[b] = (c.head + over) % p.ring_cap;
+    } else {
+        p.ctx_len[b] = min(c.ctx + c.n, p.max_ctx);
+    }
+}
+
+__global__ void __launch_bounds__(128) kv_commit_kernel(const __grid_constant__ CommitParams p)
 {
     const int b = blockIdx.x;
-    const int n = max(0, min(p.n_accept[b], p.T));
-    int head = 0, len = 0, ctx = 0;
-    if (p.kind == 0) {
-        head = ((p.ring_head[b] % p.ring_cap) + p.ring_cap) % p.ring_cap;
-        len = max(0, min(p.ring_len[b], p.ring_cap));
-    } else {
-        ctx = max(0, min(p.ctx_len[b], p.max_ctx));
-    }
-    // 16-byte chunks per token: Hkv heads x (24 K chunks + 16 V chunks)
-    const int per_tok = p.Hkv * 40;
-    for (int i = threadIdx.x; i < n * per_tok; i += blockDim.x) {
+    const CommitState cs = commit_state(p, b);
+    const int pph = commit_pieces_per_head(p);
+    const int per_tok = p.Hkv * pph;
+    const int64_t pos0 = p.pos ? (int64_t)p.pos[b] : (int64_t)cs.ctx;
+    for (int i = threadIdx.x; i < cs.n * per_tok; i += blockDim.x) {
         const int u = i / per_tok;
         const int rem = i - u * per_tok;
-        const int gh = rem / 40, ch = rem % 40;
+        const int gh = rem / pph;
+        const CommitPiece pc = commit_piece(p, rem - gh * pph);
         int64_t kdst, vdst;
-        if (p.kind == 0) {
-            const int slot = (head + len + u) % p.ring_cap;
-            kdst = (int64_t)b * p.kc_sb + (int64_t)slot * p.kc_ss;
-            vdst = (int64_t)b * p.vc_sb + (int64_t)slot * p.vc_ss;
-        } else if (p.kind == 1) {
-            const int pos = ctx + u;
-            if (pos >= p.max_ctx)
-                continue;
-            kdst = (int64_t)b * p.kc_sb + (int64_t)pos * p.kc_ss;
-            vdst = (int64_t)b * p.vc_sb + (int64_t)pos * p.vc_ss;
-        } else {
-            const int pos = ctx + u;
-            const int pg = pos / p.page_size;
-            if (pos >= p.max_ctx || pg >= p.max_pages)
-                continue;
-            const int pid = p.page_table[(int64_t)b * p.max_pages + pg];
-            if (pid < 0 || pid >= p.num_pages)
-                continue;
-            const int rr = pos - pg * p.page_size;
-            kdst = (int64_t)pid * p.kc_sb + (int64_t)rr * p.kc_ss;
-            vdst = (int64_t)pid * p.vc_sb + (int64_t)rr * p.vc_ss;
-        }
-        if (ch < 24) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.k_new + (int64_t)b * p.kn_sb + (int64_t)u * p.kn_st + (int64_t)gh * p.kn_sh);
-            uint4 *dst = reinterpret_cast<uint4 *>(p.k_cache + kdst + (int64_t)gh * p.kc_sh);
-            dst[ch] = src[ch];
-        } else {
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                p.v_new + (int64_t)b * p.vn_sb + (int64_t)u * p.vn_st + (int64_t)gh * p.vn_sh);
-            uint4 *dst = reinterpret_cast<uint4 *>(p.v_cache + vdst + (int64_t)gh * p.vc_sh);
-            dst[ch - 24] = src[ch - 24];
-        }
+        if (!commit_dst(p, b, u, cs.head, cs.len, cs.ctx, kdst, vdst))
+            continue;
+        uint4 x0, x1;
+        commit_load(p, pc, b, u, gh, pos0 + u, x0, x1);
+        uint16_t *row = pc.is_k ? p.k_cache + kdst + (int64_t)gh * p.kc_sh
+                                : p.v_cache + vdst + (int64_t)gh * p.vc_sh;
+        *reinterpret_cast<uint4 *>(row + pc.c0 * 8) = x0;
+        if (pc.c1 >= 0)
+            *reinterpret_cast<uint4 *>(row + pc.c1 * 8) = x1;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        if (p.kind == 0) {
-            const int over = max(0, len + n - p.ring_cap);
-            p.ring_len[b] = min(p.ring_cap, len + n);
-            p.ring_head[b] = (head + over) % p.ring_cap;
-        } else {
-            p.ctx_len[b] = min(ctx + n, p.max_ctx);
-        }
-    }
+    if (threadIdx.x == 0)
+        commit_advance(p, b, cs);
 }
 
 cudaError_t launch_commit(const CommitParams &p, cudaStream_t stream)
 {
     kv_commit_kernel<<<p.B, 128, 0, stream>>>(p);
     return cudaGetLastError();
+}
+
+cudaError_t set_wait_limit(uint64_t ns)
+{
+    cudaError_t e = cudaDeviceSynchronize(); // no kernel of ours runs while the limit changes
+    if (e != cudaSuccess)
+        return e;
+    return cudaMemcpyToSymbol(g_wait_limit_ns, &ns, sizeof(ns));
 }
 
 cudaError_t read_and_clear_device_error(uint32_t *flag)

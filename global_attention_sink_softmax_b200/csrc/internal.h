@@ -98,6 +98,9 @@ cudaError_t launch_decode_ring(const CUtensorMap &kc, const CUtensorMap &vc, con
 cudaError_t launch_decode_merge(const DecodeParams &p, cudaStream_t stream);
 int decode_stages(const DecodeParams &p);
 
+// Fused partial RoPE + value scale: rope_dim <= 2 * kRopeMaxHalf.
+constexpr int kRopeMaxHalf = 64; // rope_dim <= 128
+
 struct CommitParams {
     int kind, B, T, Hkv;
     const uint16_t *k_new, *v_new;
@@ -113,14 +116,24 @@ struct CommitParams {
     const int32_t *n_accept;
     int fp8;               // quantise into an E4M3 cache (strides count bytes)
     float k_scale, v_scale;
+    // RoPE + value scale as the tokens are stored (rope_half = 0: store as given): pair i of the
+    // first rope_half dims turns at inv_freq[i] with position pos[b] + u (pos null: the cache's
+    // own count), V is multiplied by v_mul; an FP8 cache stores the codes of the results
+    int rope_half;
+    float v_mul;
+    const int32_t *pos;
+    double inv_freq[kRopeMaxHalf];
 };
 
 cudaError_t launch_commit(const CommitParams &p, cudaStream_t stream);
 cudaError_t launch_decode_fp8(const DecodeParams &p, cudaStream_t stream);
+// FP8-cache decode fed by TMA: code maps {d, Hkv, rows, blocks} over uint8, box {64, 1, 64, 1},
+// 64-byte swizzle.
+cudaError_t launch_decode_fp8_tma(const CUtensorMap &kc, const CUtensorMap &vc,
+                                  const DecodeParams &p, cudaStream_t stream);
 cudaError_t launch_commit_fp8(const CommitParams &p, cudaStream_t stream);
 
 // Fused partial RoPE + value scale, in place (rope_kernels.cuh).
-constexpr int kRopeMaxHalf = 64; // rope_dim <= 128
 struct RopeParams {
     uint16_t *q, *k, *v; // any may be null (skipped)
     const int32_t *pos_base;
@@ -133,6 +146,28 @@ struct RopeParams {
 
 cudaError_t launch_rope_qkv(const RopeParams &p, cudaStream_t stream);
 
+// ---- prefill backward ------------------------------------------------------------------------
+struct BwdParams {
+    int B, L, Hq, Hkv, G, window;
+    float scale, scale_log2;
+    const uint16_t *o, *dout;
+    int64_t o_sb, o_sl, o_sh, do_sb, do_sl, do_sh;
+    const float *lse, *sink;
+    float *delta; // [B, Hq, L]
+    float *dq, *dk, *dv, *dsink;
+    int64_t dq_sb, dq_sl, dq_sh, dk_sb, dk_sl, dk_sh, dv_sb, dv_sl, dv_sh;
+};
+
+// delta and dsink (dsink, when given, must hold zeros on entry)
+cudaError_t launch_bwd_delta(const BwdParams &p, cudaStream_t stream);
+// q / do maps {d, Hq, L, B}, k / v maps {d, Hkv, L, B}; boxes of 64 rows (dK/dV: q, do) or
+// 128 rows (dK/dV: k, v; dQ: all four)
+cudaError_t launch_bwd_dkdv(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
+                            const CUtensorMap &dout, const BwdParams &p, cudaStream_t stream);
+cudaError_t launch_bwd_dq(const CUtensorMap &q, const CUtensorMap &k, const CUtensorMap &v,
+                          const CUtensorMap &dout, const BwdParams &p, cudaStream_t stream);
+
 cudaError_t read_and_clear_device_error(uint32_t *flag);
+cudaError_t set_wait_limit(uint64_t ns);
 
 } // namespace sinkattn

@@ -11,11 +11,9 @@
 //     y_{i+rope_dim/2} = x_{i+rope_dim/2} cos + x_i sin
 // Dims rope_dim .. d-1 are not touched (not even read). V is multiplied by v_scale.
 //
-// Precision. The angle m * w_i is formed in fp64 (w_i from the host in fp64) and reduced to
-// [-pi, pi] by subtracting the nearest multiple of 2 pi, with 2 pi split into a leading and a
-// trailing fp64 part (Cody and Waite's additive range reduction); only then is it rounded to
-// fp32 for sincosf. At position 262143 the fp32 product alone would be off by ~0.016 rad.
-// The rotation runs in fp32 and each result is rounded once to bf16 (nearest even).
+// Precision (rope_cos_sin, rope_rotate8 in common.cuh): the angle m * w_i is formed in fp64 (w_i
+// from the host in fp64) and range-reduced in fp64 before sincosf; the rotation runs in fp32 and
+// each result is rounded once to bf16 (nearest even).
 //
 // Work split: a CTA takes TOK tokens. Its threads first compute (cos, sin) for every
 // (token, pair) into shared memory (the angle depends on the token only, so one value serves
@@ -32,14 +30,6 @@ namespace rp {
 constexpr int THREADS = 256;
 constexpr int TOK = 8; // tokens per CTA
 } // namespace rp
-
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-__device__ __forceinline__ uint32_t pack_rn(float lo, float hi)
-{
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t *>(&v);
-}
 
 // One unit of work: where its two 16-byte pieces live and what to do with them.
 struct RopeUnit {
@@ -95,23 +85,11 @@ __device__ __forceinline__ void rope_apply(const RopeUnit &r, uint4 a, uint4 b,
 {
     if (r.pair0 == -2)
         return;
-    uint32_t *wa = reinterpret_cast<uint32_t *>(&a);
-    uint32_t *wb = reinterpret_cast<uint32_t *>(&b);
     if (r.pair0 >= 0) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float2 c0 = cs[r.pair0 + 2 * j], c1 = cs[r.pair0 + 2 * j + 1];
-            const float x0 = bf16_lo(wa[j]), x1 = bf16_hi(wa[j]); // pairs 2j, 2j+1: first half
-            const float y0 = bf16_lo(wb[j]), y1 = bf16_hi(wb[j]); //                  second half
-            wa[j] = pack_rn(fmaf(x0, c0.x, -y0 * c0.y), fmaf(x1, c1.x, -y1 * c1.y));
-            wb[j] = pack_rn(fmaf(y0, c0.x, x0 * c0.y), fmaf(y1, c1.x, x1 * c1.y));
-        }
+        rope_rotate8(a, b, cs + r.pair0); // pairs pair0 .. pair0 + 7: first half in a
     } else {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            wa[j] = pack_rn(bf16_lo(wa[j]) * v_scale, bf16_hi(wa[j]) * v_scale);
-            wb[j] = pack_rn(bf16_lo(wb[j]) * v_scale, bf16_hi(wb[j]) * v_scale);
-        }
+        scale8(a, v_scale);
+        scale8(b, v_scale);
     }
     *r.p0 = a;
     *r.p1 = b;
@@ -131,21 +109,13 @@ __global__ void __launch_bounds__(rp::THREADS) rope_qkv_kernel(const __grid_cons
     const int ntk = (int)min((int64_t)TOK, ntok - t0);
 
     if (q_units + k_units > 0) {
-        // 2 pi = k2PiHi + k2PiLo: k2PiHi is 2 pi rounded to fp64, k2PiLo what that rounding lost
-        const double k2PiHi = 6.283185307179586232, k2PiLo = 2.4492935982947064e-16;
-        const double kInv2Pi = 0.15915494309189533577;
         for (int e = threadIdx.x; e < ntk * p.half; e += THREADS) {
             const int tt = e / p.half, i = e - tt * p.half;
             const int64_t t = t0 + tt;
             const int b = (int)(t / p.L);
             const int l = (int)(t - (int64_t)b * p.L);
             const int64_t m = p.pos0 + (p.pos_base ? (int64_t)p.pos_base[b] : 0) + l;
-            const double angle = (double)m * p.inv_freq[i];
-            const double n2pi = rint(angle * kInv2Pi);
-            const double red = fma(-n2pi, k2PiLo, fma(-n2pi, k2PiHi, angle));
-            float s, c;
-            sincosf((float)red, &s, &c);
-            cs[e] = make_float2(c, s);
+            cs[e] = rope_cos_sin(m, p.inv_freq[i]);
         }
         __syncthreads();
     }

@@ -10,9 +10,11 @@
 #include "common.cuh"
 #include "decode_kernels.cuh"
 #include "decode_fp8_kernels.cuh"
+#include "decode_fp8_tma_kernels.cuh"
 #include "decode_tma_kernels.cuh"
 #include "decode_umma_kernels.cuh"
 #include "decode_ring_kernels.cuh"
+#include "backward_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
 #include "rope_kernels.cuh"
@@ -69,6 +71,27 @@ int make_map(CUtensorMap *map, const void *base, int d, int heads, int tokens, i
     const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? SINKATTN_OK : SINKATTN_ERR_INVALID_ARG;
+}
+
+// 4-D map over one-byte codes [blocks, tokens, heads, d] given as dims {d, heads, tokens,
+// blocks}, strides in bytes; box {64, 1, box_tokens, 1} (64-byte rows), 64-byte swizzle, zero
+// fill outside the tensor.
+int make_map_u8(CUtensorMap *map, const void *base, int d, int heads, int tokens, int blocks,
+                int64_t s_head, int64_t s_tok, int64_t s_blk, int box_tokens)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn)
+        return SINKATTN_ERR_CUDA;
+    const cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)tokens,
+                                (cuuint64_t)blocks};
+    const cuuint64_t strides[3] = {(cuuint64_t)s_head, (cuuint64_t)s_tok, (cuuint64_t)s_blk};
+    const cuuint32_t box[4] = {64, 1, (cuuint32_t)box_tokens, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void *>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? SINKATTN_OK : SINKATTN_ERR_INVALID_ARG;
 }
@@ -229,6 +252,55 @@ int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *st
     p.lse = a->lse;
     const cudaError_t e = launch_prefill_band(tq, tk, tv, p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+// ---- prefill backward --------------------------------------------------------------------------
+int validate_backward(const sinkattn_backward_args *a)
+{
+    if (!a)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->B < 0 || a->L < 0 || a->Hq <= 0 || a->Hkv <= 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->d_qk != kDQ || a->d_v != kDV || a->Hq % a->Hkv != 0)
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (!isfinite(a->scale) || !(a->scale > 0.f))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->B == 0 || a->L == 0)
+        return SINKATTN_OK;
+    const void *ptrs[9] = {a->q, a->k, a->v, a->o, a->dout, a->lse, a->dq, a->dk, a->dv};
+    for (int i = 0; i < 9; ++i) {
+        if (!ptrs[i])
+            return SINKATTN_ERR_INVALID_ARG;
+        if (!aligned16(ptrs[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    const int64_t sb[15] = {a->q_sb, a->q_sl, a->q_sh, a->k_sb, a->k_sl, a->k_sh, a->v_sb, a->v_sl,
+                            a->v_sh, a->o_sb, a->o_sl, a->o_sh, a->do_sb, a->do_sl, a->do_sh};
+    for (int i = 0; i < 15; ++i) {
+        if (sb[i] <= 0)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (!stride_ok(sb[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    // fp32 gradients: element strides, positive multiples of 4 (16 bytes)
+    const int64_t sf[9] = {a->dq_sb, a->dq_sl, a->dq_sh, a->dk_sb, a->dk_sl, a->dk_sh,
+                           a->dv_sb, a->dv_sl, a->dv_sh};
+    for (int i = 0; i < 9; ++i) {
+        if (sf[i] <= 0)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (sf[i] % 4 != 0)
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    if (a->dsink && !aligned16(a->dsink))
+        return SINKATTN_ERR_ALIGNMENT;
+    if ((int64_t)a->B * a->Hq * a->L > ((int64_t)1 << 40))
+        return SINKATTN_ERR_UNSUPPORTED;
+    return SINKATTN_OK;
+}
+
+size_t backward_workspace_bytes(const sinkattn_backward_args *a)
+{
+    return (size_t)a->B * a->Hq * a->L * sizeof(float); // delta
 }
 
 // ---- decode sizing ----------------------------------------------------------------------------
@@ -473,10 +545,11 @@ cudaError_t noalloc_workspace_ptr(void **out)
     return cudaSuccess;
 }
 
-// The TMA-fed decode kernels take whole 64-key tiles: contiguous caches, and paged caches whose
-// pages hold a multiple of 64 tokens (without a window, so tiles stay page-aligned). Rings and
-// other page sizes use the cp.async kernel: on a 128-slot ring each (sequence, KV head) item is
-// only 80 KB, and there the cp.async kernel, two CTAs per SM, is the faster of the two.
+// The split-KV TMA-fed decode kernels take whole 64-key tiles: contiguous caches, and paged
+// caches whose pages hold a multiple of 64 tokens (without a window, so tiles stay page-aligned).
+// Rings of up to 16 query rows per item go to the ring kernel; other rings (a 4-token verify's
+// 32 rows measured faster on the cp.async kernel, whose CTA serves all rows) and other page
+// sizes use the cp.async kernel.
 bool decode_tma_ok(const sinkattn_decode_args *a, const DecodeParams &)
 {
     if (a->kind == SINKATTN_KV_CONTIG)
@@ -490,7 +563,23 @@ int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *strea
 {
     cudaError_t e;
     if (p.fp8) {
-        e = launch_decode_fp8(p, (cudaStream_t)stream);
+        // whole 64-key tiles of codes by TMA: contiguous caches, pages of a multiple of 64
+        // tokens without a window, rings of a multiple of 64 slots in one span; the rest (and a
+        // cache the encoder rejects, e.g. an empty one) take the cp.async kernel
+        const bool tiles = a->kind == SINKATTN_KV_CONTIG ||
+                           (a->kind == SINKATTN_KV_PAGED && a->window == 0 && a->page_size % 64 == 0) ||
+                           (a->kind == SINKATTN_KV_RING && a->ring_cap % 64 == 0 && p.splits == 1);
+        const int rows = a->kind == SINKATTN_KV_RING ? a->ring_cap
+                         : a->kind == SINKATTN_KV_CONTIG ? a->max_ctx
+                                                         : a->page_size;
+        const int blocks = a->kind == SINKATTN_KV_PAGED ? a->num_pages : a->B;
+        CUtensorMap kc, vc;
+        if (tiles && rows > 0 &&
+            !make_map_u8(&kc, a->k_cache, kDQ, a->Hkv, rows, blocks, a->kc_sh, a->kc_ss, a->kc_sb, 64) &&
+            !make_map_u8(&vc, a->v_cache, kDV, a->Hkv, rows, blocks, a->vc_sh, a->vc_ss, a->vc_sb, 64))
+            e = launch_decode_fp8_tma(kc, vc, p, (cudaStream_t)stream);
+        else
+            e = launch_decode_fp8(p, (cudaStream_t)stream);
         return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
     }
     if (a->kind == SINKATTN_KV_RING && p.R <= 16 && a->ring_cap % 32 == 0 && p.splits == 1) {
@@ -510,14 +599,11 @@ int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *strea
         }
     }
     if (decode_tma_ok(a, p)) {
-        const int rows = a->kind == SINKATTN_KV_RING ? a->ring_cap
-                         : a->kind == SINKATTN_KV_CONTIG ? a->max_ctx
-                                                         : a->page_size;
+        const int rows = a->kind == SINKATTN_KV_CONTIG ? a->max_ctx : a->page_size;
         const int blocks = a->kind == SINKATTN_KV_PAGED ? a->num_pages : a->B;
         // tcgen05 kernel: blocks of more than 16 query rows over 128-key tiles (pages of a
         // multiple of 128 tokens); the mma.sync TMA kernel: the rest, over 64-key tiles
-        const bool umma = (p.R > 16 && (a->kind != SINKATTN_KV_PAGED || a->page_size % 128 == 0)) ||
-                          a->kind == SINKATTN_KV_RING;
+        const bool umma = p.R > 16 && (a->kind != SINKATTN_KV_PAGED || a->page_size % 128 == 0);
         const int new_rows = umma ? 16 : 64;
         const int box = umma ? 128 : 64;
         CUtensorMap kc, vc, kn, vn, q;
@@ -531,13 +617,8 @@ int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *strea
                 e = launch_decode_tma(kc, vc, kn, vn, p, (cudaStream_t)stream);
                 return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
             }
-            DeviceInfo di;
-            const int st = device_info(&di);
-            if (st != SINKATTN_OK)
-                return st;
             if (!make_map(&q, a->q, kDQ, a->Hq, a->T, a->B, a->q_sh, a->q_st, a->q_sb, p.G, a->T)) {
-                e = launch_decode_umma(q, kc, vc, kn, vn, p,
-                                       a->kind == SINKATTN_KV_RING ? di.sms : 0, (cudaStream_t)stream);
+                e = launch_decode_umma(q, kc, vc, kn, vn, p, 0, (cudaStream_t)stream);
                 return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
             }
         }
@@ -652,6 +733,17 @@ int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, v
         return SINKATTN_ERR_UNSUPPORTED;
     if (kv_dtype_check(a) != SINKATTN_OK)
         return SINKATTN_ERR_INVALID_ARG;
+    if (a->commit_rope != 0 && a->commit_rope != 1)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (a->commit_rope) {
+        if (!(a->rope_theta > 0.0) || !isfinite(a->rope_theta) || !isfinite(a->commit_v_scale))
+            return SINKATTN_ERR_INVALID_ARG;
+        if (a->kind == SINKATTN_KV_RING && !a->commit_pos)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (a->rope_dim < 16 || a->rope_dim > 2 * kRopeMaxHalf || a->rope_dim % 16 != 0 ||
+            a->rope_dim > kDQ)
+            return SINKATTN_ERR_UNSUPPORTED;
+    }
     if (a->B == 0 || a->T == 0)
         return SINKATTN_OK;
     if (!n_accept || !a->k_new || !a->v_new || !a->k_cache || !a->v_cache)
@@ -710,6 +802,12 @@ int sinkattn_kv_commit(const sinkattn_decode_args *a, const int32_t *n_accept, v
     p.max_pages = a->max_pages;
     p.num_pages = a->num_pages;
     p.n_accept = n_accept;
+    p.rope_half = a->commit_rope ? a->rope_dim / 2 : 0;
+    p.v_mul = a->commit_rope ? a->commit_v_scale : 1.f;
+    p.pos = a->commit_rope ? a->commit_pos : nullptr;
+    // the same fp64 frequencies as sinkattn_rope_qkv, so both give the same bits
+    for (int i = 0; i < kRopeMaxHalf; ++i)
+        p.inv_freq[i] = i < p.rope_half ? pow(a->rope_theta, -2.0 * i / (2.0 * p.rope_half)) : 0.0;
     const cudaError_t e = fp8 ? launch_commit_fp8(p, (cudaStream_t)stream)
                               : launch_commit(p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
@@ -780,6 +878,85 @@ int sinkattn_rope_qkv(const sinkattn_rope_args *a, void *stream)
         p.inv_freq[i] = i < p.half ? pow(a->theta, -2.0 * i / (2.0 * p.half)) : 0.0;
     const cudaError_t e = launch_rope_qkv(p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+size_t sinkattn_prefill_backward_workspace_size(const sinkattn_backward_args *args)
+{
+    if (validate_backward(args) != SINKATTN_OK || args->B == 0 || args->L == 0)
+        return 0;
+    return backward_workspace_bytes(args);
+}
+
+int sinkattn_prefill_backward(const sinkattn_backward_args *a, int32_t window, void *workspace,
+                              size_t ws_bytes, void *stream)
+{
+    if (window < 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    int st = validate_backward(a);
+    if (st != SINKATTN_OK || a->B == 0 || a->L == 0)
+        return st;
+    const size_t need = backward_workspace_bytes(a);
+    if (!workspace || ws_bytes < need)
+        return SINKATTN_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(workspace))
+        return SINKATTN_ERR_ALIGNMENT;
+    CUtensorMap q64, do64, q128, do128, k128, v128;
+    if ((st = make_map(&q64, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, 1, 64)) ||
+        (st = make_map(&do64, a->dout, kDV, a->Hq, a->L, a->B, a->do_sh, a->do_sl, a->do_sb, 1, 64)) ||
+        (st = make_map(&q128, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, 1, 128)) ||
+        (st = make_map(&do128, a->dout, kDV, a->Hq, a->L, a->B, a->do_sh, a->do_sl, a->do_sb, 1, 128)) ||
+        (st = make_map(&k128, a->k, kDQ, a->Hkv, a->L, a->B, a->k_sh, a->k_sl, a->k_sb, 1, 128)) ||
+        (st = make_map(&v128, a->v, kDV, a->Hkv, a->L, a->B, a->v_sh, a->v_sl, a->v_sb, 1, 128)))
+        return st;
+    BwdParams p;
+    p.B = a->B;
+    p.L = a->L;
+    p.Hq = a->Hq;
+    p.Hkv = a->Hkv;
+    p.G = a->Hq / a->Hkv;
+    p.window = window;
+    p.scale = a->scale;
+    p.scale_log2 = a->scale * kLog2e;
+    p.o = static_cast<const uint16_t *>(a->o);
+    p.dout = static_cast<const uint16_t *>(a->dout);
+    p.o_sb = a->o_sb;
+    p.o_sl = a->o_sl;
+    p.o_sh = a->o_sh;
+    p.do_sb = a->do_sb;
+    p.do_sl = a->do_sl;
+    p.do_sh = a->do_sh;
+    p.lse = a->lse;
+    p.sink = a->sink;
+    p.delta = static_cast<float *>(workspace);
+    p.dq = a->dq;
+    p.dk = a->dk;
+    p.dv = a->dv;
+    p.dsink = a->dsink;
+    p.dq_sb = a->dq_sb;
+    p.dq_sl = a->dq_sl;
+    p.dq_sh = a->dq_sh;
+    p.dk_sb = a->dk_sb;
+    p.dk_sl = a->dk_sl;
+    p.dk_sh = a->dk_sh;
+    p.dv_sb = a->dv_sb;
+    p.dv_sl = a->dv_sl;
+    p.dv_sh = a->dv_sh;
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = cudaSuccess;
+    if (a->dsink)
+        e = cudaMemsetAsync(a->dsink, 0, sizeof(float) * a->Hq, s);
+    if (e == cudaSuccess)
+        e = launch_bwd_delta(p, s);
+    if (e == cudaSuccess)
+        e = launch_bwd_dkdv(q64, k128, v128, do64, p, s);
+    if (e == cudaSuccess)
+        e = launch_bwd_dq(q128, k128, v128, do128, p, s);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+int sinkattn_set_wait_limit_ns(uint64_t ns)
+{
+    return set_wait_limit(ns) == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 
 int sinkattn_take_device_error(uint32_t *flag_out)

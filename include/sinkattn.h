@@ -199,6 +199,20 @@ typedef struct sinkattn_decode_args {
      * |q| must stay below 65504 on this path. */
     int32_t kv_dtype;
     float k_scale, v_scale;
+    /* sinkattn_kv_commit only (decode ignores them). With commit_rope = 1 the commit applies the
+     * two steps that precede attention ("MiMo-V2-Flash 模型架构深度拆解" CH10.3) as it stores each
+     * accepted token, exactly as sinkattn_rope_qkv would: K's first rope_dim dims get the partial
+     * rotary embedding with rope_theta at the token's absolute position, and V is multiplied by
+     * commit_v_scale (0.707 for the pages' model). Accepted token u of sequence b sits at
+     * position commit_pos[b] + u; commit_pos may be NULL for CONTIG and PAGED caches, where it
+     * defaults to ctx_len[b] before the commit, and must be given for a RING (whose length stops
+     * at ring_cap). An FP8 cache stores the codes of the rotated / scaled bf16 values.
+     * commit_rope = 0 (a zero-initialised struct) stores k_new / v_new as given. */
+    int32_t commit_rope;
+    int32_t rope_dim;          /* a multiple of 16 in 16..128 (64 for the pages' model) */
+    double rope_theta;         /* > 0 and finite: 5e6 on GA layers, 1e4 on SWA layers */
+    float commit_v_scale;      /* finite */
+    const int32_t *commit_pos; /* device int32 [B] or NULL */
 } sinkattn_decode_args;
 
 /* Bytes of device workspace sinkattn_decode needs for these arguments. The pages give no
@@ -256,8 +270,12 @@ int sinkattn_decode_noalloc(const sinkattn_decode_args *args, void *stream);
  *   CONTIG: row ctx_len[b] + u (tokens beyond max_ctx are dropped); ctx_len grows.
  *   PAGED:  position ctx_len[b] + u through the page table (positions beyond
  *           max_pages * page_size are dropped); ctx_len grows.
- * Uses the cache, metadata and *_new fields of `args` (q, o, lse, sink are ignored). Updates
- * k_cache, v_cache, ring_head / ring_len or ctx_len in place, in stream order.
+ * Uses the cache, metadata, *_new and commit_* fields of `args` (q, o, lse, sink are ignored).
+ * Updates k_cache, v_cache, ring_head / ring_len or ctx_len in place, in stream order. With
+ * commit_rope = 1 the stored K / V are rotated and scaled first (see sinkattn_decode_args); the
+ * caller's k_new / v_new are not modified. Errors: INVALID_ARG also for commit_rope not 0 / 1,
+ * rope_theta <= 0 or not finite, commit_v_scale not finite, a RING without commit_pos;
+ * UNSUPPORTED for rope_dim out of range.
  * ------------------------------------------------------------------------------------------- */
 int sinkattn_kv_commit(const sinkattn_decode_args *args, const int32_t *n_accept, void *stream);
 
@@ -302,6 +320,60 @@ typedef struct sinkattn_rope_args {
 
 int sinkattn_rope_qkv(const sinkattn_rope_args *args, void *stream);
 
+/* ---------------------------------------------------------------------------------------------
+ * Backward of the whole-sequence prefill: the training variant. The gradients of a loss through
+ * O = attention(q, k, v, sink) given dO = dLoss/dO. The sink enters the softmax the way
+ * "MiMo-V2-Flash 模型架构深度拆解" CH10.1 builds it (a column of per-head logits concatenated
+ * after the scaled, masked scores, softmax, then that column dropped), so its gradient is that
+ * column's softmax gradient with zero value (CH10.1 creates it with requires_grad=False; it is
+ * given here for a caller that does train it). With P_ij = exp(a_ij - LSE_i) and
+ * p_s,i = exp(sink_h - LSE_i) (LSE of the forward, sink included), for every row i:
+ *     delta_i  = <dO_i, O_i>
+ *     dS_ij    = P_ij (<dO_i, v_j> - delta_i)
+ *     dq_i     = scale sum_j dS_ij k_j,   dk_j = scale sum_{i, heads of the group} dS_ij q_i,
+ *     dv_j     = sum_{i, heads of the group} P_ij dO_i,   dsink_h = - sum_{b, i} p_s,i delta_i.
+ *
+ *   q, k, v, o, dout: bf16 as in prefill (o [B, L, Hq, 128] the forward's output, dout its
+ *       gradient, strides o_*, do_*); lse: fp32 [B, Hq, L] contiguous, the forward's LSE.
+ *   dq [B, L, Hq, 192], dk [B, L, Hkv, 192], dv [B, L, Hkv, 128]: fp32, written (element
+ *       strides dq_*, dk_*, dv_*, multiples of 4, the last dim contiguous).
+ *   dsink: fp32 [Hq], written (NULL: not computed); sink NULL means no sink (dsink = 0).
+ *   window = 0: full causal (GA); window >= 1: sliding window (SWA).
+ *   workspace: device memory of sinkattn_prefill_backward_workspace_size bytes, 16-byte aligned
+ *       (delta, B * Hq * L floats); its contents on entry do not matter.
+ * Errors: as for prefill (dims 192 / 128 only), plus NULL o / dout / lse / gradient pointers,
+ * SINKATTN_ERR_WORKSPACE_TOO_SMALL. The gradients do not depend on the order of any atomic sum
+ * except dsink (a float sum over the batch's rows).
+ * ------------------------------------------------------------------------------------------- */
+typedef struct sinkattn_backward_args {
+    const void *q;
+    const void *k;
+    const void *v;
+    const void *o;
+    const void *dout;
+    const float *lse;
+    const float *sink;
+    float *dq;
+    float *dk;
+    float *dv;
+    float *dsink;
+    int32_t B, L, Hq, Hkv, d_qk, d_v;
+    float scale;
+    int64_t q_sb, q_sl, q_sh;
+    int64_t k_sb, k_sl, k_sh;
+    int64_t v_sb, v_sl, v_sh;
+    int64_t o_sb, o_sl, o_sh;
+    int64_t do_sb, do_sl, do_sh;
+    int64_t dq_sb, dq_sl, dq_sh;
+    int64_t dk_sb, dk_sl, dk_sh;
+    int64_t dv_sb, dv_sl, dv_sh;
+} sinkattn_backward_args;
+
+size_t sinkattn_prefill_backward_workspace_size(const sinkattn_backward_args *args);
+
+int sinkattn_prefill_backward(const sinkattn_backward_args *args, int32_t window,
+                              void *workspace, size_t workspace_bytes, void *stream);
+
 /* Human-readable name of a status code (static storage). */
 const char *sinkattn_status_string(int status);
 
@@ -312,6 +384,17 @@ int sinkattn_version(void);
  * prefill, bit 1: decode). Synchronises the current device. Returns SINKATTN_OK and writes the
  * flag to *flag_out, or SINKATTN_ERR_CUDA. */
 int sinkattn_take_device_error(uint32_t *flag_out);
+
+/* Sets how long a kernel on the current device waits on an internal barrier before it gives
+ * up, records bit 0 (prefill) or 1 (decode) in the device flag above and returns (its output
+ * is then unspecified). Failure detection: a stuck copy or MMA ends the call instead of hanging
+ * the GPU. Default 1 s (1e9 ns); legitimate waits last microseconds. 0 makes every wait that is
+ * not already satisfied when first tested give up, which exercises the failure path on demand
+ * (the library's tests do this). The waits a CTA makes for its own copies and MMAs before it
+ * exits keep the 1 s bound. Process-wide for the current device; synchronises the device first.
+ * Returns SINKATTN_OK or SINKATTN_ERR_CUDA. The pages have no counterpart: this is a service of
+ * the library, not part of the method. */
+int sinkattn_set_wait_limit_ns(uint64_t ns);
 
 #ifdef __cplusplus
 }

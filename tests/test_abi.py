@@ -60,6 +60,7 @@ int main(void) {
   printf("sinkattn_prefill_args %zu\n", sizeof(sinkattn_prefill_args));
   printf("sinkattn_decode_args %zu\n", sizeof(sinkattn_decode_args));
   printf("sinkattn_rope_args %zu\n", sizeof(sinkattn_rope_args));
+  printf("sinkattn_backward_args %zu\n", sizeof(sinkattn_backward_args));
   %FIELDS%
   return 0;
 }
@@ -69,7 +70,7 @@ int main(void) {
 def test_struct_layout_matches_header(tmp_path):
     lines = []
     structs = (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs),
-               ("sinkattn_rope_args", sa.RopeArgs))
+               ("sinkattn_rope_args", sa.RopeArgs), ("sinkattn_backward_args", sa.BackwardArgs))
     for cname, py in structs:
         for f, _ in py._fields_:
             lines.append(f"F({cname}, {f})")
@@ -82,6 +83,7 @@ def test_struct_layout_matches_header(tmp_path):
     assert int(got["sinkattn_prefill_args"]) == ctypes.sizeof(sa.PrefillArgs)
     assert int(got["sinkattn_decode_args"]) == ctypes.sizeof(sa.DecodeArgs)
     assert int(got["sinkattn_rope_args"]) == ctypes.sizeof(sa.RopeArgs)
+    assert int(got["sinkattn_backward_args"]) == ctypes.sizeof(sa.BackwardArgs)
     for cname, py in structs:
         for f, _ in py._fields_:
             assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
@@ -192,6 +194,57 @@ def test_commit_rejects_bad_arguments(L):
     assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(dv=64)), ctypes.c_void_p(0x60000), None) == 2
     assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(kind=0)), ctypes.c_void_p(0x60000), None) == 1
     assert L.sinkattn_kv_commit(ctypes.byref(_decode_args(B=0)), None, None) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(commit_rope=2), 1),                                         # not a flag
+    (dict(commit_rope=1, rope_dim=64, rope_theta=0.0), 1),            # theta must be > 0
+    (dict(commit_rope=1, rope_dim=64, rope_theta=float("nan")), 1),
+    (dict(commit_rope=1, rope_dim=64, rope_theta=1e4, commit_v_scale=float("inf")), 1),
+    (dict(commit_rope=1, rope_dim=24, rope_theta=1e4), 2),            # not a multiple of 16
+    (dict(commit_rope=1, rope_dim=144, rope_theta=1e4), 2),           # wider than 128
+    (dict(commit_rope=1, rope_dim=64, rope_theta=1e4, kind=0, ring_head=0x50000,
+          ring_len=0x50100, ring_cap=128), 1),                        # a ring needs commit_pos
+])
+def test_commit_rope_arguments_are_checked(L, kw, status):
+    """Host-side checks of the commit's fused RoPE + value scale: nothing reaches the GPU."""
+    a = _decode_args(**kw)
+    assert L.sinkattn_kv_commit(ctypes.byref(a), ctypes.c_void_p(0x60000), None) == status
+
+
+def _backward_args(**kw):
+    a = sa.BackwardArgs()
+    a.q = a.k = a.v = a.o = a.dout = a.lse = a.dq = a.dk = a.dv = 0x10000
+    a.B, a.L, a.Hq, a.Hkv, a.d_qk, a.d_v = 1, 64, 8, 1, 192, 128
+    a.scale = 0.07
+    for t, d, h in (("q", 192, 8), ("k", 192, 1), ("v", 128, 1), ("o", 128, 8), ("do", 128, 8),
+                    ("dq", 192, 8), ("dk", 192, 1), ("dv", 128, 1)):
+        setattr(a, t + "_sh", d)
+        setattr(a, t + "_sl", d * h)
+        setattr(a, t + "_sb", d * h * 64)
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(d_qk=128), 2), (dict(Hkv=3), 2), (dict(B=-1), 1), (dict(scale=0.0), 1),
+    (dict(o=None), 1), (dict(lse=None), 1), (dict(dk=None), 1), (dict(dout=0x10008), 3),
+    (dict(q_sl=100), 3), (dict(dq_sl=6), 3), (dict(dv_sh=0), 1),
+])
+def test_backward_rejects_bad_arguments(L, kw, status):
+    """Host-side checks of the prefill backward: nothing reaches the GPU."""
+    a = _backward_args(**kw)
+    assert L.sinkattn_prefill_backward(ctypes.byref(a), 0, None, 0, None) == status
+
+
+def test_backward_workspace_and_window(L):
+    a = _backward_args()
+    need = L.sinkattn_prefill_backward_workspace_size(ctypes.byref(a))
+    assert need == 1 * 8 * 64 * 4   # delta: one float per (sequence, head, row)
+    assert L.sinkattn_prefill_backward(ctypes.byref(a), 0, None, 0, None) == 4
+    assert L.sinkattn_prefill_backward(ctypes.byref(a), -1, None, 0, None) == 1
+    assert L.sinkattn_prefill_backward(ctypes.byref(_backward_args(L=0)), 0, None, 0, None) == 0
 
 
 def _rope_args(**kw):
