@@ -179,7 +179,12 @@ class DecodeRunner:
             self.kw.update(k_scale=d["k_scale"], v_scale=d["v_scale"])
         rows = w.T * (w.Hq // w.Hkv)
         if fp8:
-            self.kernel = "decode_fp8_kernel"
+            # whole 64-key tiles of codes by TMA (contiguous, pages of a multiple of 64 tokens
+            # without a window, one-span rings of a multiple of 64 slots), else cp.async
+            tma = (w.kind == W.KV_CONTIG or (w.kind == W.KV_PAGED and w.window == 0 and
+                                             w.page_size % 64 == 0) or
+                   (w.kind == W.KV_RING and w.ring_cap % 64 == 0))
+            self.kernel = "decode_fp8_tma_kernel" if tma else "decode_fp8_kernel"
         elif w.kind == W.KV_RING:
             self.kernel = ("decode_ring_kernel" if rows <= 16 and w.ring_cap % 32 == 0
                            else "decode_split_kernel")
@@ -236,6 +241,54 @@ class RopeRunner:
     def release(self):
         if hasattr(self, "d"):
             del self.d
+
+
+class BackwardRunner:
+    """The prefill backward (the training variant) on a prefill workload: the forward runs once
+    to give O and LSE, then each step computes dq, dk, dv and dsink from dout. Algorithmic FLOPs
+    per visible (row, head, key) pair: 2 (d_qk + d_qk + d_qk + d_v + d_v) = 1664 (S recomputed
+    once, dP, dV, dK, dQ); bytes: q, k, v, o, dout and LSE read once, the fp32 gradients written
+    once."""
+
+    FLOP_PER_PAIR = 2 * (3 * W.DQ + 2 * W.DV)
+
+    def __init__(self, w, dev):
+        import global_attention_sink_softmax_b200 as sa
+        self.sa, self.w = sa, w
+        d = W.prefill_inputs(w, device=dev)
+        self.q, self.k, self.v, self.sink = d["q"], d["k"], d["v"], d["sink"]
+        if w.window:
+            self.o, self.lse = sa.sinkattn_prefill_swa(self.q, self.k, self.v, self.sink, w.window)
+        else:
+            self.o, self.lse = sa.sinkattn_prefill_ga(self.q, self.k, self.v, self.sink)
+        g = torch.Generator(device=dev).manual_seed(w.seed + 7)
+        self.dout = torch.randn(self.o.shape, generator=g, device=dev).to(torch.bfloat16)
+        f32 = dict(dtype=torch.float32, device=dev)
+        self.dq = torch.empty(w.B, w.L, w.Hq, w.dq, **f32)
+        self.dk = torch.empty(w.B, w.L, w.Hkv, w.dq, **f32)
+        self.dv = torch.empty(w.B, w.L, w.Hkv, w.dv, **f32)
+        self.dsink = torch.empty(w.Hq, **f32)
+        self.ws = torch.empty(w.B * w.Hq * w.L * 4, dtype=torch.uint8, device=dev)
+        pairs = w.B * w.Hq * visible_pairs_prefill(w.L, w.window)
+        self.flops = pairs * self.FLOP_PER_PAIR
+        bf16 = 2 * w.B * w.L * (w.Hq * w.dq + w.Hkv * (w.dq + w.dv) + 2 * w.Hq * w.dv)
+        self.bytes = bf16 + 4 * w.B * w.Hq * w.L + 4 * w.B * w.L * (w.Hq * w.dq + w.Hkv * (w.dq + w.dv))
+        self.launches = 4  # dsink clear, delta, dK / dV, dQ
+        self.kernel = None
+        self.workload = w.name + "_backward"
+        self.config = dict(B=w.B, L=w.L, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
+                           window=w.window, kind=("SWA" if w.window else "GA") + " backward",
+                           grads="fp32")
+
+    def step(self):
+        self.sa.sinkattn_prefill_backward(self.q, self.k, self.v, self.o, self.lse, self.dout,
+                                          self.sink, window=self.w.window, dq=self.dq, dk=self.dk,
+                                          dv=self.dv, dsink=self.dsink, workspace=self.ws)
+
+    def release(self):
+        for k in ("q", "k", "v", "o", "lse", "dout", "dq", "dk", "dv", "ws", "sink", "dsink"):
+            if hasattr(self, k):
+                delattr(self, k)
 
 
 class HybridRunner:
@@ -416,7 +469,12 @@ def measured_traffic(kernel):
                                     "decode_ring_kernels.cuh"],
              "rope_qkv_kernel": ["common.cuh", "rope_kernels.cuh"],
              "decode_fp8_kernel": ["common.cuh", "decode_kernels.cuh",
-                                   "decode_fp8_kernels.cuh"]}[kernel]
+                                   "decode_fp8_kernels.cuh"],
+             "decode_fp8_tma_kernel": ["common.cuh", "decode_kernels.cuh",
+                                       "decode_tma_kernels.cuh", "decode_fp8_kernels.cuh",
+                                       "decode_fp8_tma_kernels.cuh"]}.get(kernel)
+    if files is None:
+        return None
     m = hashlib.sha256()
     for f in files:
         m.update(open(os.path.join(csrc, f), "rb").read())
@@ -652,7 +710,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default=None,
                     help="run one workload only: swa_prefill, ga_prefill, ga_chunk_prefill, "
-                         "ga_decode, ga_decode_fp8, swa_decode, hybrid, rope")
+                         "ga_backward, ga_decode, ga_decode_fp8, swa_decode, hybrid, rope")
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--ref-L", type=int, default=0, help="reference arm: shorter sequences (tests)")
     ap.add_argument("--small", action="store_true",
@@ -741,6 +799,8 @@ def main():
             jobs.append(("ga_chunk_prefill", lambda: PrefillRunner(gac_w, dev), None))
         if only in (None, "rope"):
             jobs.append(("rope_qkv", lambda: RopeRunner(swa_w, dev, 1e4), None))
+        if only in (None, "ga_backward"):
+            jobs.append(("ga_prefill_backward", lambda: BackwardRunner(ga_w, dev), None))
         if only in (None, "ga_decode"):
             jobs.append(("ga_decode", lambda: DecodeRunner(gad_w, dev), None))
         if only in (None, "ga_decode_fp8"):
@@ -767,7 +827,8 @@ def main():
                 ms = measure(r, steps, max(3, args.warmup), flush, world)
             ms_step = ms / steps
             rl = roofline(r, ms_step, peaks, peak_src,
-                          bound="hbm" if isinstance(r, RopeRunner) else None)
+                          bound="hbm" if isinstance(r, RopeRunner) else
+                          ("tensor" if isinstance(r, BackwardRunner) else None))
             entry = {"workload": r.workload, "config": r.config, "ms_per_step": round(ms_step, 4),
                      "tflops": round(r.flops / (ms_step * 1e-3) / 1e12, 3),
                      "gbs": round(r.bytes / (ms_step * 1e-3) / 1e9, 2), "roofline": rl,

@@ -28,7 +28,7 @@ __all__ = [
     "sinkattn_status_string", "sinkattn_version", "EXPORTED_SYMBOLS",
     "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES", "sinkattn_rope_qkv",
     "ROPE_THETA_GA", "ROPE_THETA_SWA", "V_SCALE", "KV_BF16", "KV_FP8_E4M3",
-    "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward",
+    "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward", "sinkattn_prefill_chunk_paged",
 ]
 
 KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
@@ -43,7 +43,7 @@ EXPORTED_SYMBOLS = [
     "sinkattn_decode_workspace_size", "sinkattn_decode", "sinkattn_kv_commit", "sinkattn_status_string", "sinkattn_version",
     "sinkattn_take_device_error", "sinkattn_decode_noalloc", "sinkattn_rope_qkv",
     "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward_workspace_size",
-    "sinkattn_prefill_backward",
+    "sinkattn_prefill_backward", "sinkattn_prefill_chunk_paged",
 ]
 # Size of the library's own split-KV workspace used by sinkattn_decode_noalloc.
 NOALLOC_WORKSPACE_BYTES = 16 << 20
@@ -125,6 +125,9 @@ def lib() -> ctypes.CDLL:
             L.sinkattn_prefill_ga.argtypes = [ctypes.POINTER(PrefillArgs), _P]
             L.sinkattn_prefill_chunk.restype = ctypes.c_int
             L.sinkattn_prefill_chunk.argtypes = [ctypes.POINTER(PrefillArgs), _I32, _I32, _P]
+            L.sinkattn_prefill_chunk_paged.restype = ctypes.c_int
+            L.sinkattn_prefill_chunk_paged.argtypes = [ctypes.POINTER(PrefillArgs),
+                                                       ctypes.POINTER(PagedKV), _I32, _I32, _P]
             L.sinkattn_prefill_ga.restype = ctypes.c_int
             L.sinkattn_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeArgs)]
             L.sinkattn_decode_workspace_size.restype = _SZ
@@ -219,7 +222,14 @@ def _prefill_args(q, k, v, sink, o, lse, scale):
     return a
 
 
-def _prefill(fn, q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix=0):
+class PagedKV(ctypes.Structure):
+    _fields_ = [("k_pages", _P), ("v_pages", _P),
+                ("kp_sb", _I64), ("kp_ss", _I64), ("kp_sh", _I64),
+                ("vp_sb", _I64), ("vp_ss", _I64), ("vp_sh", _I64),
+                ("page_table", _P), ("page_size", _I32), ("max_pages", _I32), ("num_pages", _I32)]
+
+
+def _prefill(fn, q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix=0, paged=None):
     B, L, Hq, dq = q.shape
     if scale is None:
         scale = 1.0 / math.sqrt(dq)
@@ -233,6 +243,9 @@ def _prefill(fn, q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix=
         st = L_.sinkattn_prefill_swa(ctypes.byref(a), int(window), _stream(stream))
     elif fn == "chunk":
         st = L_.sinkattn_prefill_chunk(ctypes.byref(a), int(prefix), int(window), _stream(stream))
+    elif fn == "chunk_paged":
+        st = L_.sinkattn_prefill_chunk_paged(ctypes.byref(a), ctypes.byref(paged), int(prefix),
+                                             int(window), _stream(stream))
     else:
         st = L_.sinkattn_prefill_ga(ctypes.byref(a), _stream(stream))
     _raise(st, f"sinkattn_prefill_{fn}")
@@ -264,6 +277,28 @@ def sinkattn_prefill_chunk(q, k, v, sink=None, *, prefix, window=0, o=None, lse=
     if k.shape[1] != prefix + q.shape[1] or v.shape[1] != prefix + q.shape[1]:
         raise ValueError("k and v must hold prefix + L positions")
     return _prefill("chunk", q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix)
+
+
+def sinkattn_prefill_chunk_paged(q, k, v, k_pages, v_pages, page_table, sink=None, *, prefix,
+                                 window=0, num_pages=None, o=None, lse=None, scale=None,
+                                 stream=None, want_lse=True):
+    """Chunked prefill against a paged prefix: q, k, v [B, L, ...] are the chunk's own tokens
+    (positions prefix .. prefix+L-1); positions 0 .. prefix-1 are row c % page_size of page
+    page_table[b, c // page_size] of k_pages [pages, page_size, Hkv, 192] / v_pages [.., 128].
+    prefix and page_size must be multiples of 128. Returns (o, lse) as sinkattn_prefill_chunk."""
+    _check_bf16("k_pages", k_pages)
+    _check_bf16("v_pages", v_pages)
+    if page_table.dtype != torch.int32 or not page_table.is_cuda or not page_table.is_contiguous() \
+            or page_table.dim() != 2:
+        raise ValueError("page_table must be a contiguous 2-D CUDA int32 tensor")
+    pk = PagedKV()
+    pk.k_pages, pk.v_pages, pk.page_table = _ptr(k_pages), _ptr(v_pages), _ptr(page_table)
+    pk.kp_sb, pk.kp_ss, pk.kp_sh = k_pages.stride(0), k_pages.stride(1), k_pages.stride(2)
+    pk.vp_sb, pk.vp_ss, pk.vp_sh = v_pages.stride(0), v_pages.stride(1), v_pages.stride(2)
+    pk.page_size, pk.max_pages = k_pages.shape[1], page_table.shape[1]
+    pk.num_pages = k_pages.shape[0] if num_pages is None else int(num_pages)
+    return _prefill("chunk_paged", q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix,
+                    pk)
 
 
 # ----------------------------------------------------------------------------------------------
@@ -509,6 +544,6 @@ def sinkattn_prefill_backward(q, k, v, o, lse, dout, sink=None, *, window=0, sca
 
 def sinkattn_set_wait_limit_ns(ns: int) -> None:
     """How long a kernel on the current device waits on an internal barrier before it gives up
-    and records it in the wait-timeout flag (default 10**9 ns; 0 gives up at the first wait that
-    is not already satisfied). Process-wide per device; synchronises the device first."""
+    and records it in the wait-timeout flag (default 10**9 ns; 0 gives up as soon as a wait's
+    first, briefly suspending try fails). Process-wide per device; synchronises the device."""
     _raise(lib().sinkattn_set_wait_limit_ns(int(ns)), "sinkattn_set_wait_limit_ns")

@@ -46,6 +46,7 @@ constexpr int CONSUMERS = 4;
 constexpr int THREADS = 32 * (CONSUMERS + 1);
 constexpr int RED_STRIDE = 70;
 constexpr int SMEM_BYTES = NSTAGE * STAGE + 256 + 1024;
+constexpr float TAU = 8.0f;               // lazy-rescale threshold (log2 units)
 static_assert(CONSUMERS * 32 * RED_STRIDE * 4 <= NSTAGE * STAGE, "combine scratch fits the ring");
 } // namespace d8t
 
@@ -267,11 +268,15 @@ __global__ void __launch_bounds__(d8t::THREADS, 2)
         const uint32_t sK = smem_u32(stage), sV = smem_u32(stage + STAGE_K);
         const int key0 = ks * KW; // first key of this warp inside the tile
         const bool tile_ok = decode_tile_ok(p, d, b, t);
+        // a cached tile whose 64 keys every row sees (no window, a contiguous or paged cache,
+        // inside the span's cached keys): no mask and no V rows to zero
+        const bool whole = p.kind != 0 && p.window <= 0 && tile_ok && t < d.cache_tiles &&
+                           d.kb + (t + 1) * KT <= min(d.ke, d.n_used);
         // zero the V codes of this warp's keys that the span must not see (a NaN code times a
         // zero weight would still be NaN), 32 keys at a time
         bool zeroed = false;
 #pragma unroll
-        for (int k32 = 0; k32 < KW; k32 += 32) {
+        for (int k32 = 0; k32 < KW && !whole; k32 += 32) {
             bool valid;
             int pos;
             decode_key(p, d, t, key0 + k32 + (lane % KW), tile_ok, valid, pos);
@@ -307,34 +312,65 @@ __global__ void __launch_bounds__(d8t::THREADS, 2)
             }
         }
 
-        // ---- mask, online softmax (sink-free partial)
+        // ---- mask, online softmax (sink-free partial) with a lazily raised max
         float mxa = -INFINITY, mxb = -INFINITY;
+        if (whole) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
+            for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int kc = nt * 8 + 2 * (lane & 3) + e;
-                bool valid;
-                int pos;
-                decode_key(p, d, t, key0 + kc, tile_ok, valid, pos);
-                const bool vis_a = valid && pos <= ta && (p.window <= 0 || pos > ta - p.window);
-                const bool vis_b = valid && pos <= tb && (p.window <= 0 || pos > tb - p.window);
-                sacc[nt][e] = vis_a ? sacc[nt][e] * p.scale_log2 : -INFINITY;
-                sacc[nt][2 + e] = vis_b ? sacc[nt][2 + e] * p.scale_log2 : -INFINITY;
-                mxa = fmaxf(mxa, sacc[nt][e]);
-                mxb = fmaxf(mxb, sacc[nt][2 + e]);
+                for (int e = 0; e < 2; ++e) {
+                    sacc[nt][e] *= p.scale_log2;
+                    sacc[nt][2 + e] *= p.scale_log2;
+                    mxa = fmaxf(mxa, sacc[nt][e]);
+                    mxb = fmaxf(mxb, sacc[nt][2 + e]);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int kc = nt * 8 + 2 * (lane & 3) + e;
+                    bool valid;
+                    int pos;
+                    decode_key(p, d, t, key0 + kc, tile_ok, valid, pos);
+                    const bool vis_a = valid && pos <= ta && (p.window <= 0 || pos > ta - p.window);
+                    const bool vis_b = valid && pos <= tb && (p.window <= 0 || pos > tb - p.window);
+                    sacc[nt][e] = vis_a ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+                    sacc[nt][2 + e] = vis_b ? sacc[nt][2 + e] * p.scale_log2 : -INFINITY;
+                    mxa = fmaxf(mxa, sacc[nt][e]);
+                    mxb = fmaxf(mxb, sacc[nt][2 + e]);
+                }
             }
         }
         mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 1));
         mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, 2));
         mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 1));
         mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, 2));
-        const float mna = fmaxf(m_a, mxa), mnb = fmaxf(m_b, mxb);
-        const float alpha_a = (mna == -INFINITY) ? 1.f : fast_exp2(m_a - mna);
-        const float alpha_b = (mnb == -INFINITY) ? 1.f : fast_exp2(m_b - mnb);
-        const float ua = (mna == -INFINITY) ? 0.f : mna, ub = (mnb == -INFINITY) ? 0.f : mnb;
-        m_a = mna;
-        m_b = mnb;
+        // a row's reference max rises only when the tile's exceeds it by more than TAU (always
+        // for the first visible score: m is -inf), so most tiles skip the rescale of O; P stays
+        // <= 2^TAU, well inside fp16
+        const bool up_a = mxa > m_a + TAU, up_b = mxb > m_b + TAU;
+        if (__any_sync(0xffffffffu, up_a || up_b)) {
+            const float alpha_a = up_a ? fast_exp2(m_a - mxa) : 1.f; // 0 while m is -inf
+            const float alpha_b = up_b ? fast_exp2(m_b - mxb) : 1.f;
+            if (up_a)
+                m_a = mxa;
+            if (up_b)
+                m_b = mxb;
+            l_a *= alpha_a;
+            l_b *= alpha_b;
+            e_a *= alpha_a;
+            e_b *= alpha_b;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                o[i][0] *= alpha_a;
+                o[i][1] *= alpha_a;
+                o[i][2] *= alpha_b;
+                o[i][3] *= alpha_b;
+            }
+        }
+        const float ua = (m_a == -INFINITY) ? 0.f : m_a, ub = (m_b == -INFINITY) ? 0.f : m_b;
         uint32_t pp[NT][2];
         float sa = 0.f, sb = 0.f, xa = 0.f, xb = 0.f;
 #pragma unroll
@@ -348,17 +384,10 @@ __global__ void __launch_bounds__(d8t::THREADS, 2)
             sa += sum_f16x2(pp[nt][0]);
             sb += sum_f16x2(pp[nt][1]);
         }
-        l_a = l_a * alpha_a + sa;
-        l_b = l_b * alpha_b + sb;
-        e_a = e_a * alpha_a + xa;
-        e_b = e_b * alpha_b + xb;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            o[i][0] *= alpha_a;
-            o[i][1] *= alpha_a;
-            o[i][2] *= alpha_b;
-            o[i][3] *= alpha_b;
-        }
+        l_a += sa;
+        l_b += sb;
+        e_a += xa;
+        e_b += xb;
 
         // ---- O += P V: per 16 keys and 32 dims one ldmatrix.x4.trans; prmt splits each
         // register's byte pairs into the "even" (dim 2g) and "odd" (dim 2g + 1) n-tiles

@@ -18,12 +18,27 @@ struct PrefillParams {
     void *o;              // bf16
     int64_t o_sb, o_sl, o_sh;
     float *lse;           // [B, Hq, L] or nullptr
+    // paged prefix (paged != 0): keys at positions < q_off come from a page pool through
+    // page_table [B, max_pages] (q_off and page_size multiples of 128); the K / V maps then hold
+    // only the L positions of the chunk
+    int paged;
+    const int32_t *page_table;
+    int page_size, max_pages, num_pages;
 };
 
-// Q map: dims {192, Hq, L, B}; K map: {192, Hkv, q_off + L, B}; V map: {128, Hkv, q_off + L, B}; 128-byte
-// swizzle, 64-element inner box.
+// Q map: dims {192, Hq, L, B}; K map: {192, Hkv, q_off + L, B}; V map: {128, Hkv, q_off + L, B}
+// (paged: {.., L, B}); page maps {d, Hkv, page_size, num_pages} (the K / V maps again when not
+// paged); 128-byte swizzle, 64-element inner box, 128-row boxes.
 cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
-                                const CUtensorMap &tmV, const PrefillParams &p,
+                                const CUtensorMap &tmV, const CUtensorMap &tmKp,
+                                const CUtensorMap &tmVp, const PrefillParams &p,
+                                cudaStream_t stream);
+
+// Full-causal prefill with two query heads of one GQA group per CTA (window 0, even G); maps as
+// for launch_prefill_band.
+cudaError_t launch_prefill_pair(const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                                const CUtensorMap &tmV, const CUtensorMap &tmKp,
+                                const CUtensorMap &tmVp, const PrefillParams &p,
                                 cudaStream_t stream);
 
 // SWA prefill, GQA-packed persistent kernel: item = (b, kv head, block of P = 128 / G positions)

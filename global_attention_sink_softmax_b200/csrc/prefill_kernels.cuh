@@ -76,10 +76,32 @@ enum Bar {
 };
 } // namespace pf
 
+// Where key tile j (positions 128 j .. 128 j + 127) of sequence b comes from: the K / V tensors
+// at (row, block) = (position, sequence), or, for a paged prefix, a page of the pool below the
+// prefix (a page id outside the pool reads zeros) and the chunk's own tensors above it.
+struct PrefillTile {
+    bool pool;
+    int row, blk;
+};
+
+SA_DEV PrefillTile prefill_tile(const PrefillParams &p, int b, int j)
+{
+    const int pos = j * pf::BN;
+    if (!p.paged)
+        return PrefillTile{false, pos, b};
+    if (pos >= p.q_off)
+        return PrefillTile{false, pos - p.q_off, b};
+    const int pg = pos / p.page_size;
+    const int pid = p.page_table[(int64_t)b * p.max_pages + pg];
+    return PrefillTile{true, pos - pg * p.page_size, (pid >= 0 && pid < p.num_pages) ? pid : p.num_pages};
+}
+
 __global__ void __launch_bounds__(pf::THREADS, 1)
     prefill_band_kernel(const __grid_constant__ CUtensorMap tmQ,
                         const __grid_constant__ CUtensorMap tmK,
-                        const __grid_constant__ CUtensorMap tmV, const PrefillParams p)
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmKp,
+                        const __grid_constant__ CUtensorMap tmVp, const PrefillParams p)
 {
     using namespace pf;
     extern __shared__ uint8_t smem_raw[];
@@ -147,10 +169,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 if (idx >= 2 && !mbar_wait(&bars[B_KEMPTY + s], ((idx >> 1) - 1) & 1, abort, 1u))
                     break;
                 const int j = j_lo + idx;
+                const PrefillTile tl = prefill_tile(p, b, j);
                 mbar_arrive_expect_tx(&bars[B_KFULL + s], K_BYTES);
                 for (int c = 0; c < 3; ++c)
-                    tma_load_4d(smem + OFF_K + s * K_BYTES + c * K_REGION, &tmK,
-                                &bars[B_KFULL + s], c * 64, g, j * BN, b);
+                    tma_load_4d(smem + OFF_K + s * K_BYTES + c * K_REGION, tl.pool ? &tmKp : &tmK,
+                                &bars[B_KFULL + s], c * 64, g, tl.row, tl.blk);
                 issued = idx + 1;
             }
             // make sure no copy of ours is still landing in shared memory when the CTA ends
@@ -168,10 +191,11 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 if (idx >= 2 && !mbar_wait(&bars[B_VEMPTY + vs], ((idx >> 1) - 1) & 1, abort, 1u))
                     break;
                 const int j = j_lo + idx;
+                const PrefillTile tl = prefill_tile(p, b, j);
                 mbar_arrive_expect_tx(&bars[B_VFULL + vs], V_BYTES);
                 for (int c = 0; c < 2; ++c)
-                    tma_load_4d(smem + OFF_V + vs * V_BYTES + c * K_REGION, &tmV,
-                                &bars[B_VFULL + vs], c * 64, g, j * BN, b);
+                    tma_load_4d(smem + OFF_V + vs * V_BYTES + c * K_REGION, tl.pool ? &tmVp : &tmV,
+                                &bars[B_VFULL + vs], c * 64, g, tl.row, tl.blk);
                 issued = idx + 1;
             }
             for (int idx = max(0, issued - 2); idx < issued; ++idx)
@@ -383,7 +407,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
 }
 
 cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
-                                const CUtensorMap &tmV, const PrefillParams &p,
+                                const CUtensorMap &tmV, const CUtensorMap &tmKp,
+                                const CUtensorMap &tmVp, const PrefillParams &p,
                                 cudaStream_t stream)
 {
     static PerContextOnce configured; // shared-memory opt-in, once per context
@@ -398,7 +423,8 @@ cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
         return cudaSuccess;
     if (blocks > 0x7fffffff)
         return cudaErrorInvalidConfiguration;
-    prefill_band_kernel<<<(unsigned)blocks, pf::THREADS, pf::SMEM_BYTES, stream>>>(tmQ, tmK, tmV, p);
+    prefill_band_kernel<<<(unsigned)blocks, pf::THREADS, pf::SMEM_BYTES, stream>>>(tmQ, tmK, tmV,
+                                                                                    tmKp, tmVp, p);
     return cudaGetLastError();
 }
 

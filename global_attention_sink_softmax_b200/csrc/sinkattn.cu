@@ -17,6 +17,7 @@
 #include "backward_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
+#include "prefill_pair_kernels.cuh"
 #include "rope_kernels.cuh"
 #include "swa_kernels.cuh"
 
@@ -211,13 +212,42 @@ int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *str
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 
+// Checks of a paged prefix (sinkattn_prefill_chunk_paged).
+int validate_paged_prefix(const sinkattn_paged_kv *kv, int prefix)
+{
+    if (!kv || !kv->k_pages || !kv->v_pages || !kv->page_table)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (kv->page_size <= 0 || kv->max_pages <= 0 || kv->num_pages <= 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (prefix % 128 != 0 || kv->page_size % 128 != 0)
+        return SINKATTN_ERR_UNSUPPORTED;
+    if ((int64_t)prefix > (int64_t)kv->max_pages * kv->page_size)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (!aligned16(kv->k_pages) || !aligned16(kv->v_pages))
+        return SINKATTN_ERR_ALIGNMENT;
+    const int64_t s[6] = {kv->kp_sb, kv->kp_ss, kv->kp_sh, kv->vp_sb, kv->vp_ss, kv->vp_sh};
+    for (int i = 0; i < 6; ++i) {
+        if (s[i] <= 0)
+            return SINKATTN_ERR_INVALID_ARG;
+        if (!stride_ok(s[i]))
+            return SINKATTN_ERR_ALIGNMENT;
+    }
+    return SINKATTN_OK;
+}
+
 // Prefill of the L query rows at positions prefix .. prefix + L - 1 against keys 0 .. prefix +
-// L - 1 (prefix = 0: whole sequences).
-int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *stream)
+// L - 1 (prefix = 0: whole sequences). With `paged`, keys below the prefix come from its pool
+// and args->k / v hold the chunk's L positions only.
+int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *stream,
+                const sinkattn_paged_kv *paged = nullptr)
 {
     int st = validate_prefill(a);
-    if (st != SINKATTN_OK || a->B == 0 || a->L == 0)
+    if (st != SINKATTN_OK)
         return st;
+    if (paged && (st = validate_paged_prefix(paged, prefix)) != SINKATTN_OK)
+        return st;
+    if (a->B == 0 || a->L == 0)
+        return SINKATTN_OK;
     if (prefix < 0 || (int64_t)prefix + a->L > 0x7fffffff)
         return SINKATTN_ERR_INVALID_ARG;
     if (window > 0 && prefix == 0) {
@@ -226,14 +256,25 @@ int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *st
         if (st != SINKATTN_OK || done)
             return st;
     }
-    const int n_kv = prefix + a->L;
-    CUtensorMap tq, tk, tv;
+    const int n_kv = paged ? a->L : prefix + a->L;
+    CUtensorMap tq, tk, tv, tkp, tvp;
     if ((st = make_map(&tq, a->q, kDQ, a->Hq, a->L, a->B, a->q_sh, a->q_sl, a->q_sb, 1, 128)))
         return st;
     if ((st = make_map(&tk, a->k, kDQ, a->Hkv, n_kv, a->B, a->k_sh, a->k_sl, a->k_sb, 1, 128)))
         return st;
     if ((st = make_map(&tv, a->v, kDV, a->Hkv, n_kv, a->B, a->v_sh, a->v_sl, a->v_sb, 1, 128)))
         return st;
+    if (paged) {
+        if ((st = make_map(&tkp, paged->k_pages, kDQ, a->Hkv, paged->page_size, paged->num_pages,
+                           paged->kp_sh, paged->kp_ss, paged->kp_sb, 1, 128)))
+            return st;
+        if ((st = make_map(&tvp, paged->v_pages, kDV, a->Hkv, paged->page_size, paged->num_pages,
+                           paged->vp_sh, paged->vp_ss, paged->vp_sb, 1, 128)))
+            return st;
+    } else {
+        tkp = tk;
+        tvp = tv;
+    }
     PrefillParams p;
     p.B = a->B;
     p.L = a->L;
@@ -250,7 +291,17 @@ int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *st
     p.o_sl = a->o_sl;
     p.o_sh = a->o_sh;
     p.lse = a->lse;
-    const cudaError_t e = launch_prefill_band(tq, tk, tv, p, (cudaStream_t)stream);
+    p.paged = paged ? 1 : 0;
+    p.page_table = paged ? paged->page_table : nullptr;
+    p.page_size = paged ? paged->page_size : 0;
+    p.max_pages = paged ? paged->max_pages : 0;
+    p.num_pages = paged ? paged->num_pages : 0;
+    // full causal with an even group: two heads per CTA share each K / V tile and take turns
+    // with the tensor cores; otherwise one head per CTA
+    const cudaError_t e =
+        (window == 0 && p.G % 2 == 0)
+            ? launch_prefill_pair(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream)
+            : launch_prefill_band(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 
@@ -675,6 +726,15 @@ int sinkattn_prefill_chunk(const sinkattn_prefill_args *args, int32_t prefix, in
     if (window < 0)
         return SINKATTN_ERR_INVALID_ARG;
     return run_prefill(args, window, prefix, stream);
+}
+
+int sinkattn_prefill_chunk_paged(const sinkattn_prefill_args *args,
+                                 const sinkattn_paged_kv *prefix_kv, int32_t prefix,
+                                 int32_t window, void *stream)
+{
+    if (window < 0 || !prefix_kv)
+        return SINKATTN_ERR_INVALID_ARG;
+    return run_prefill(args, window, prefix, stream, prefix_kv);
 }
 
 size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args)

@@ -139,6 +139,32 @@ int sinkattn_prefill_ga(const sinkattn_prefill_args *args, void *stream);
 int sinkattn_prefill_chunk(const sinkattn_prefill_args *args, int32_t prefix, int32_t window,
                            void *stream);
 
+/* The cached prefix of a chunked prefill in a paged KV pool (the serving stack of the
+ * "MiMo-V2-Flash" model card pages its KV cache): position c < prefix of sequence b is row
+ * c mod page_size of page page_table[b * max_pages + c / page_size].
+ *   k_pages [num_pages, page_size, Hkv, 192], v_pages [num_pages, page_size, Hkv, 128]: bf16,
+ *       strides kp_sb / vp_sb (between pages), kp_ss / vp_ss (rows), kp_sh / vp_sh (heads);
+ *   page_table: device int32 [B, max_pages]; every page the prefix uses must be mapped (an id
+ *       outside [0, num_pages) reads as zero keys and values). */
+typedef struct sinkattn_paged_kv {
+    const void *k_pages;
+    const void *v_pages;
+    int64_t kp_sb, kp_ss, kp_sh;
+    int64_t vp_sb, vp_ss, vp_sh;
+    const int32_t *page_table;
+    int32_t page_size, max_pages, num_pages;
+} sinkattn_paged_kv;
+
+/* Chunked prefill against a paged prefix: as sinkattn_prefill_chunk, but args->k / v hold only
+ * the chunk's own L positions ([B, L, Hkv, ...]) and positions 0 .. prefix - 1 come from
+ * `prefix_kv`. prefix and page_size must be multiples of 128 (whole 128-key tiles come from one
+ * page, or from the chunk), and prefix <= max_pages * page_size.
+ * Errors: as sinkattn_prefill_chunk; UNSUPPORTED for prefix or page_size not multiples of 128;
+ * INVALID_ARG for a NULL prefix_kv or page table, non-positive page geometry or strides. */
+int sinkattn_prefill_chunk_paged(const sinkattn_prefill_args *args,
+                                 const sinkattn_paged_kv *prefix_kv, int32_t prefix,
+                                 int32_t window, void *stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Decode / speculative verify: T (1..4) new query tokens per sequence attend to that sequence's
  * cached tokens plus new tokens 0..t. The new tokens' K/V are passed separately and are NOT yet
@@ -388,9 +414,10 @@ int sinkattn_take_device_error(uint32_t *flag_out);
 /* Sets how long a kernel on the current device waits on an internal barrier before it gives
  * up, records bit 0 (prefill) or 1 (decode) in the device flag above and returns (its output
  * is then unspecified). Failure detection: a stuck copy or MMA ends the call instead of hanging
- * the GPU. Default 1 s (1e9 ns); legitimate waits last microseconds. 0 makes every wait that is
- * not already satisfied when first tested give up, which exercises the failure path on demand
- * (the library's tests do this). The waits a CTA makes for its own copies and MMAs before it
+ * the GPU. Default 1 s (1e9 ns); legitimate waits last microseconds. 0 makes a wait give up as
+ * soon as its first try (which suspends the thread only briefly) fails, as it does for waits
+ * that span a load and an MMA step: this exercises the failure path on demand (the library's
+ * tests do this). The waits a CTA makes for its own copies and MMAs before it
  * exits keep the 1 s bound. Process-wide for the current device; synchronises the device first.
  * Returns SINKATTN_OK or SINKATTN_ERR_CUDA. The pages have no counterpart: this is a service of
  * the library, not part of the method. */

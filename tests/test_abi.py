@@ -61,6 +61,7 @@ int main(void) {
   printf("sinkattn_decode_args %zu\n", sizeof(sinkattn_decode_args));
   printf("sinkattn_rope_args %zu\n", sizeof(sinkattn_rope_args));
   printf("sinkattn_backward_args %zu\n", sizeof(sinkattn_backward_args));
+  printf("sinkattn_paged_kv %zu\n", sizeof(sinkattn_paged_kv));
   %FIELDS%
   return 0;
 }
@@ -70,7 +71,8 @@ int main(void) {
 def test_struct_layout_matches_header(tmp_path):
     lines = []
     structs = (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs),
-               ("sinkattn_rope_args", sa.RopeArgs), ("sinkattn_backward_args", sa.BackwardArgs))
+               ("sinkattn_rope_args", sa.RopeArgs), ("sinkattn_backward_args", sa.BackwardArgs),
+               ("sinkattn_paged_kv", sa.PagedKV))
     for cname, py in structs:
         for f, _ in py._fields_:
             lines.append(f"F({cname}, {f})")
@@ -84,6 +86,7 @@ def test_struct_layout_matches_header(tmp_path):
     assert int(got["sinkattn_decode_args"]) == ctypes.sizeof(sa.DecodeArgs)
     assert int(got["sinkattn_rope_args"]) == ctypes.sizeof(sa.RopeArgs)
     assert int(got["sinkattn_backward_args"]) == ctypes.sizeof(sa.BackwardArgs)
+    assert int(got["sinkattn_paged_kv"]) == ctypes.sizeof(sa.PagedKV)
     for cname, py in structs:
         for f, _ in py._fields_:
             assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
@@ -210,6 +213,31 @@ def test_commit_rope_arguments_are_checked(L, kw, status):
     """Host-side checks of the commit's fused RoPE + value scale: nothing reaches the GPU."""
     a = _decode_args(**kw)
     assert L.sinkattn_kv_commit(ctypes.byref(a), ctypes.c_void_p(0x60000), None) == status
+
+
+def _paged_kv(**kw):
+    pk = sa.PagedKV()
+    pk.k_pages, pk.v_pages, pk.page_table = 0x40000, 0x50000, 0x60000
+    pk.page_size, pk.max_pages, pk.num_pages = 128, 4, 8
+    pk.kp_sh, pk.kp_ss, pk.kp_sb = 192, 192, 192 * 128
+    pk.vp_sh, pk.vp_ss, pk.vp_sb = 128, 128, 128 * 128
+    for k, v in kw.items():
+        setattr(pk, k, v)
+    return pk
+
+
+@pytest.mark.parametrize("prefix,kw,status", [
+    (128, dict(page_table=None), 1), (128, dict(page_size=0), 1), (100, {}, 2),
+    (128, dict(page_size=64), 2), (640, {}, 1),           # beyond max_pages * page_size
+    (128, dict(k_pages=0x40008), 3), (128, dict(vp_ss=12), 3), (128, dict(kp_sb=0), 1),
+])
+def test_chunk_paged_checks_its_prefix(L, prefix, kw, status):
+    """Host-side checks of the paged prefix: nothing reaches the GPU."""
+    a = _prefill_args()
+    pk = _paged_kv(**kw)
+    assert L.sinkattn_prefill_chunk_paged(ctypes.byref(a), ctypes.byref(pk), prefix, 0, None) == status
+    assert L.sinkattn_prefill_chunk_paged(ctypes.byref(a), None, 128, 0, None) == 1
+    assert L.sinkattn_prefill_chunk_paged(ctypes.byref(a), ctypes.byref(_paged_kv()), 128, -1, None) == 1
 
 
 def _backward_args(**kw):

@@ -193,3 +193,46 @@ def test_chunked_prefill_full_size_sampled():
     idx = torch.tensor(sample)
     assert_close(o[0, idx].cpu(), ro, lse[0][:, idx].permute(1, 0).cpu(), rl, w.name)
     assert sa.sinkattn_take_device_error() == 0
+
+
+def paged_prefix(k, v, P, page, seed):
+    """The first P positions of k / v in a page pool: each sequence's pages handed out in a
+    seeded random order, plus two spare pages no sequence owns. Returns (k_pages, v_pages,
+    page_table [B, max_pages])."""
+    B, _, Hkv, _ = k.shape
+    max_pages = max(1, (P + page - 1) // page)
+    g = torch.Generator().manual_seed(seed)
+    n = B * max_pages + 2
+    perm = torch.randperm(n, generator=g).to(torch.int32)
+    table = perm[:B * max_pages].reshape(B, max_pages).contiguous()
+    kp = torch.randn(n, page, Hkv, 192, generator=g).to(torch.bfloat16)
+    vp = torch.randn(n, page, Hkv, 128, generator=g).to(torch.bfloat16)
+    for b in range(B):
+        for c in range(P):
+            kp[table[b, c // page], c % page] = k[b, c]
+            vp[table[b, c // page], c % page] = v[b, c]
+    return kp, vp, table
+
+
+@pytest.mark.parametrize("B,P,L,Hq,Hkv,window,page", [
+    (1, 128, 77, 8, 1, 0, 128),     # one prefix page, a ragged chunk
+    (2, 256, 300, 16, 1, 0, 256),   # GA group of 16, 256-token pages
+    (1, 384, 129, 8, 1, 128, 128),  # the SWA window reaching back into the pages
+    (2, 1024, 200, 8, 2, 200, 128), # a window wider than a tile, two KV heads
+    (1, 0, 64, 4, 1, 0, 128),       # no prefix at all
+])
+def test_chunked_prefill_paged_prefix(B, P, L, Hq, Hkv, window, page):
+    """The same chunked prefill with the prefix in a paged pool (the serving stack's paged KV
+    cache) instead of one contiguous tensor: rows P .. P+L-1 of the whole-sequence prefill."""
+    q, k, v, s = rand_inputs(B, P + L, Hq, Hkv, 7 * P + L + window, "mixed")
+    kp, vp, table = paged_prefix(k, v, P, page, seed=P + L)
+    dev = "cuda"
+    o, lse = sa.sinkattn_prefill_chunk_paged(q[:, P:].to(dev), k[:, P:].to(dev), v[:, P:].to(dev),
+                                             kp.to(dev), vp.to(dev), table.to(dev), s.to(dev),
+                                             prefix=P, window=window)
+    torch.cuda.synchronize()
+    rows = [[b, P + i] for b in range(B) for i in range(L)]
+    ro, rl, _ = oracle.prefill(q, k, v, s, 1 / math.sqrt(192), window, rows=rows)
+    assert_close(o.reshape(B * L, Hq, 128), ro, lse.permute(0, 2, 1).reshape(B * L, Hq), rl,
+                 f"paged chunk P{P} L{L} W{window} page{page}")
+    assert sa.sinkattn_take_device_error() == 0
