@@ -127,29 +127,26 @@ class PrefillRunner:
         else:
             self.sa.sinkattn_prefill_ga(d["q"], d["k"], d["v"], d["sink"], o=self.o, lse=self.lse)
 
-    # end to end: pinned host inputs -> device, the call, device -> host outputs
+    # end to end through the host-resident call: pinned host Q / K / V in, O / LSE back to
+    # pinned host memory, copies in both directions overlapping the kernels chunk by chunk
     def e2e_setup(self):
-        self.h_in = {k: v.cpu().pin_memory() for k, v in self.d.items()}
-        self.d_in = {k: torch.empty_like(v) for k, v in self.d.items()}
+        self.h_in = {k: self.d[k].cpu().pin_memory() for k in ("q", "k", "v")}
         self.h_o = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
         self.h_lse = torch.empty(self.lse.shape, dtype=self.lse.dtype).pin_memory()
+        h = self.h_in
+        need = self.sa.sinkattn_prefill_host_workspace_size(h["q"], h["k"], h["v"])
+        self.ws = torch.empty(need, dtype=torch.uint8, device=self.dev)
         self.h2d = sum(v.numel() * v.element_size() for v in self.h_in.values())
         self.d2h = self.h_o.numel() * 2 + self.h_lse.numel() * 4
+        self.e2e_api = "sinkattn_prefill_host"
 
     def e2e_step(self):
-        for k, v in self.h_in.items():
-            self.d_in[k].copy_(v, non_blocking=True)
-        d, w = self.d_in, self.w
-        if w.window:
-            self.sa.sinkattn_prefill_swa(d["q"], d["k"], d["v"], d["sink"], w.window, o=self.o,
-                                         lse=self.lse)
-        else:
-            self.sa.sinkattn_prefill_ga(d["q"], d["k"], d["v"], d["sink"], o=self.o, lse=self.lse)
-        self.h_o.copy_(self.o, non_blocking=True)
-        self.h_lse.copy_(self.lse, non_blocking=True)
+        h = self.h_in
+        self.sa.sinkattn_prefill_host(h["q"], h["k"], h["v"], self.d["sink"], window=self.w.window,
+                                      o=self.h_o, lse=self.h_lse, workspace=self.ws)
 
     def release(self):
-        for k in ("d", "o", "lse", "h_in", "d_in", "h_o", "h_lse"):
+        for k in ("d", "o", "lse", "h_in", "ws", "h_o", "h_lse"):
             if hasattr(self, k):
                 delattr(self, k)
 
@@ -186,8 +183,10 @@ class DecodeRunner:
                    (w.kind == W.KV_RING and w.ring_cap % 64 == 0))
             self.kernel = "decode_fp8_tma_kernel" if tma else "decode_fp8_kernel"
         elif w.kind == W.KV_RING:
-            self.kernel = ("decode_ring_kernel" if rows <= 16 and w.ring_cap % 32 == 0
-                           else "decode_split_kernel")
+            if rows <= 16 and w.ring_cap % 32 == 0:
+                self.kernel = "decode_ring_kernel"
+            else:
+                self.kernel = "decode_split_kernel"
         elif w.kind == W.KV_PAGED and w.page_size % 64 != 0:
             self.kernel = "decode_split_kernel"
         else:
@@ -780,7 +779,7 @@ def main():
             ms_e = max_over_ranks(ms_e) / max(1, min(args.steps, 5))
             result["e2e"] = {"value": round(units / (ms_e * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
                              "h2d_bytes_per_step": r.h2d, "d2h_bytes_per_step": r.d2h,
-                             "ms_per_step": round(ms_e, 3)}
+                             "ms_per_step": round(ms_e, 3), "api": r.e2e_api}
         if rank == 0 and not args.no_cpu_baseline:
             d_cpu = {k: v.cpu() for k, v in r.d.items()}
             r.release()

@@ -29,6 +29,7 @@ __all__ = [
     "sinkattn_decode_noalloc", "NOALLOC_WORKSPACE_BYTES", "sinkattn_rope_qkv",
     "ROPE_THETA_GA", "ROPE_THETA_SWA", "V_SCALE", "KV_BF16", "KV_FP8_E4M3",
     "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward", "sinkattn_prefill_chunk_paged",
+    "sinkattn_prefill_host", "sinkattn_prefill_host_workspace_size", "HOST_CHUNK",
 ]
 
 KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
@@ -44,7 +45,10 @@ EXPORTED_SYMBOLS = [
     "sinkattn_take_device_error", "sinkattn_decode_noalloc", "sinkattn_rope_qkv",
     "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward_workspace_size",
     "sinkattn_prefill_backward", "sinkattn_prefill_chunk_paged",
+    "sinkattn_prefill_host_workspace_size", "sinkattn_prefill_host",
 ]
+# Positions per chunk of the host-resident prefill (its copies in and out overlap chunk by chunk).
+HOST_CHUNK = 4096
 # Size of the library's own split-KV workspace used by sinkattn_decode_noalloc.
 NOALLOC_WORKSPACE_BYTES = 16 << 20
 
@@ -149,6 +153,10 @@ def lib() -> ctypes.CDLL:
             L.sinkattn_prefill_backward_workspace_size.restype = _SZ
             L.sinkattn_prefill_backward.argtypes = [ctypes.POINTER(BackwardArgs), _I32, _P, _SZ, _P]
             L.sinkattn_prefill_backward.restype = ctypes.c_int
+            L.sinkattn_prefill_host_workspace_size.argtypes = [ctypes.POINTER(PrefillArgs), _I32]
+            L.sinkattn_prefill_host_workspace_size.restype = _SZ
+            L.sinkattn_prefill_host.argtypes = [ctypes.POINTER(PrefillArgs), _I32, _I32, _P, _SZ, _P]
+            L.sinkattn_prefill_host.restype = ctypes.c_int
             L.sinkattn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
             L.sinkattn_set_wait_limit_ns.restype = ctypes.c_int
             _lib = L
@@ -299,6 +307,64 @@ def sinkattn_prefill_chunk_paged(q, k, v, k_pages, v_pages, page_table, sink=Non
     pk.num_pages = k_pages.shape[0] if num_pages is None else int(num_pages)
     return _prefill("chunk_paged", q, k, v, sink, window, o, lse, scale, stream, want_lse, prefix,
                     pk)
+
+
+def _host_prefill_args(q, k, v, sink, o, lse, scale):
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.is_cuda:
+            raise ValueError(f"{n} must be a bfloat16 host tensor")
+        if t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous 4-D tensor")
+    if lse is not None and (lse.dtype != torch.float32 or lse.is_cuda or not lse.is_contiguous()):
+        raise ValueError("lse must be a contiguous float32 host tensor")
+    _check_vec("sink", sink, torch.float32)
+    B, L, Hq, dq = q.shape
+    a = PrefillArgs()
+    a.q, a.k, a.v, a.sink, a.o = q.data_ptr(), k.data_ptr(), v.data_ptr(), _ptr(sink), o.data_ptr()
+    a.lse = lse.data_ptr() if lse is not None else None
+    a.B, a.L, a.Hq, a.Hkv, a.dq, a.dv = B, L, Hq, k.shape[2], dq, v.shape[3]
+    a.scale = scale
+    a.q_sb, a.q_sl, a.q_sh = q.stride(0), q.stride(1), q.stride(2)
+    a.k_sb, a.k_sl, a.k_sh = k.stride(0), k.stride(1), k.stride(2)
+    a.v_sb, a.v_sl, a.v_sh = v.stride(0), v.stride(1), v.stride(2)
+    a.o_sb, a.o_sl, a.o_sh = o.stride(0), o.stride(1), o.stride(2)
+    return a
+
+
+def sinkattn_prefill_host_workspace_size(q, k, v, *, chunk=HOST_CHUNK):
+    """Device workspace bytes of sinkattn_prefill_host for these (host) tensor shapes."""
+    B, L, Hq, dq = q.shape
+    a = PrefillArgs()
+    a.B, a.L, a.Hq, a.Hkv, a.dq, a.dv = B, L, Hq, k.shape[2], dq, v.shape[3]
+    return int(lib().sinkattn_prefill_host_workspace_size(ctypes.byref(a), int(chunk)))
+
+
+def sinkattn_prefill_host(q, k, v, sink=None, *, window=0, o=None, lse=None, workspace=None,
+                          chunk=HOST_CHUNK, scale=None, stream=None, want_lse=True):
+    """Prefill with q, k, v and the results in host memory (pinned for the copies to overlap):
+    the sequences pass through the device in chunks of `chunk` positions, copies in, kernels and
+    copies out overlapping on their own streams. window = 0 full causal (GA), >= 1 sliding
+    window (SWA); sink is a CUDA fp32 [Hq] tensor or None; workspace a CUDA uint8 tensor of at
+    least sinkattn_prefill_host_workspace_size bytes (allocated if None). Returns (o, lse) host
+    tensors, complete once `stream` (default: the current stream) has finished."""
+    B, L, Hq, dq = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dq)
+    if o is None:
+        o = torch.empty(B, L, Hq, v.shape[3], dtype=torch.bfloat16, pin_memory=True)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, L, dtype=torch.float32, pin_memory=True)
+    a = _host_prefill_args(q, k, v, sink, o, lse, scale)
+    need = lib().sinkattn_prefill_host_workspace_size(ctypes.byref(a), int(chunk))
+    if workspace is None:
+        dev = sink.device if sink is not None else torch.device("cuda", torch.cuda.current_device())
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if workspace.dtype != torch.uint8 or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA uint8 tensor")
+    st = lib().sinkattn_prefill_host(ctypes.byref(a), int(window), int(chunk), _ptr(workspace),
+                                     workspace.numel(), _stream(stream))
+    _raise(st, "sinkattn_prefill_host")
+    return o, lse
 
 
 # ----------------------------------------------------------------------------------------------

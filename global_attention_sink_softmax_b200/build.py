@@ -17,8 +17,7 @@ SOURCES = ["sinkattn.cu"]
 DEPS = SOURCES + ["common.cuh", "internal.h", "prefill_kernels.cuh", "swa_kernels.cuh",
                   "decode_kernels.cuh", "decode_tma_kernels.cuh", "decode_umma_kernels.cuh",
                   "decode_ring_kernels.cuh", "rope_kernels.cuh", "decode_fp8_kernels.cuh",
-                  "decode_fp8_tma_kernels.cuh", "backward_kernels.cuh",
-                  "prefill_pair_kernels.cuh"]
+                  "decode_fp8_tma_kernels.cuh", "backward_kernels.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",

@@ -135,7 +135,9 @@ __global__ void __launch_bounds__(d8t::THREADS, 2)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    // the KV heads of a span are neighbours in the grid: a head's 192-byte K rows share 128-byte
+    // lines with the next head's, which then meet in L2 instead of being fetched twice
+    const int g = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int MT = p.MT;
     const int mt = warp % MT, ks = warp / MT;
@@ -504,7 +506,7 @@ cudaError_t launch_decode_fp8_tma(const CUtensorMap &kc, const CUtensorMap &vc,
     });
     if (e != cudaSuccess)
         return e;
-    dim3 grid(p.splits, p.Hkv, p.B);
+    dim3 grid(p.Hkv, p.splits, p.B);
     if (p.MT == 1)
         decode_fp8_tma_kernel<4><<<grid, d8t::THREADS, d8t::SMEM_BYTES, stream>>>(kc, vc, p);
     else if (p.MT == 2)

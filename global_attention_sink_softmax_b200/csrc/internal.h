@@ -34,13 +34,6 @@ cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                 const CUtensorMap &tmVp, const PrefillParams &p,
                                 cudaStream_t stream);
 
-// Full-causal prefill with two query heads of one GQA group per CTA (window 0, even G); maps as
-// for launch_prefill_band.
-cudaError_t launch_prefill_pair(const CUtensorMap &tmQ, const CUtensorMap &tmK,
-                                const CUtensorMap &tmV, const CUtensorMap &tmKp,
-                                const CUtensorMap &tmVp, const PrefillParams &p,
-                                cudaStream_t stream);
-
 // SWA prefill, GQA-packed persistent kernel: item = (b, kv head, block of P = 128 / G positions)
 struct SwaParams {
     int B, L, Hq, Hkv, G;

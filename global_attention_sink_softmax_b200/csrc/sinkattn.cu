@@ -2,6 +2,7 @@
 // sizing and kernel launches. Everything is enqueued on the caller's stream; the library
 // allocates no device memory. The kernels live in prefill_kernels.cuh / decode_kernels.cuh;
 // the whole library is this one translation unit.
+#include <algorithm>
 #include <math.h>
 #include <mutex>
 
@@ -17,7 +18,6 @@
 #include "backward_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
-#include "prefill_pair_kernels.cuh"
 #include "rope_kernels.cuh"
 #include "swa_kernels.cuh"
 
@@ -296,12 +296,183 @@ int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *st
     p.page_size = paged ? paged->page_size : 0;
     p.max_pages = paged ? paged->max_pages : 0;
     p.num_pages = paged ? paged->num_pages : 0;
-    // full causal with an even group: two heads per CTA share each K / V tile and take turns
-    // with the tensor cores; otherwise one head per CTA
-    const cudaError_t e =
-        (window == 0 && p.G % 2 == 0)
-            ? launch_prefill_pair(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream)
-            : launch_prefill_band(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream);
+    const cudaError_t e = launch_prefill_band(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream);
+    return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+}
+
+// ---- prefill with host-resident inputs and outputs ---------------------------------------------
+// The sequences stream through the device in chunks of `chunk` positions. Copies in (Q, K, V of
+// a chunk), the chunk's prefill and copies out (its O and LSE) run on three streams ordered by
+// events, with two Q / O / LSE buffers, so while chunk c computes, chunk c + 1 comes in and
+// chunk c - 1 goes out: the two PCIe directions run at the same time. K and V stay on the device
+// for the whole call (later chunks read earlier keys).
+struct HostLayout {
+    int64_t chunk, n_chunks;
+    int64_t qrow, krow, vrow, orow;       // bytes per position
+    size_t off_k, off_v, off_q[2], off_o[2], off_lse[2], total;
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+HostLayout host_layout(const sinkattn_prefill_args *a, int chunk)
+{
+    HostLayout h;
+    h.chunk = chunk;
+    h.n_chunks = (a->L + (int64_t)chunk - 1) / chunk;
+    h.qrow = (int64_t)a->Hq * kDQ * 2;
+    h.krow = (int64_t)a->Hkv * kDQ * 2;
+    h.vrow = (int64_t)a->Hkv * kDV * 2;
+    h.orow = (int64_t)a->Hq * kDV * 2;
+    size_t off = 0;
+    h.off_k = off;
+    off += align256((size_t)a->B * a->L * h.krow);
+    h.off_v = off;
+    off += align256((size_t)a->B * a->L * h.vrow);
+    for (int x = 0; x < 2; ++x) {
+        h.off_q[x] = off;
+        off += align256((size_t)a->B * chunk * h.qrow);
+        h.off_o[x] = off;
+        off += align256((size_t)a->B * chunk * h.orow);
+        h.off_lse[x] = off;
+        off += align256((size_t)a->B * a->Hq * chunk * 4);
+    }
+    h.total = off;
+    return h;
+}
+
+// Dense [B, L, H, d] layouts only (the host buffers are copied in whole rows).
+int validate_host_prefill(const sinkattn_prefill_args *a, int window, int chunk)
+{
+    int st = validate_prefill(a);
+    if (st != SINKATTN_OK)
+        return st;
+    if (window < 0 || chunk <= 0)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (chunk % 128 != 0)
+        return SINKATTN_ERR_UNSUPPORTED;
+    if (a->B == 0 || a->L == 0)
+        return SINKATTN_OK;
+    const int64_t qh = kDQ, ql = (int64_t)a->Hq * kDQ, kl = (int64_t)a->Hkv * kDQ;
+    const int64_t vl = (int64_t)a->Hkv * kDV, ol = (int64_t)a->Hq * kDV;
+    const bool dense = a->q_sh == qh && a->q_sl == ql && a->q_sb == ql * a->L && a->k_sh == kDQ &&
+                       a->k_sl == kl && a->k_sb == kl * a->L && a->v_sh == kDV && a->v_sl == vl &&
+                       a->v_sb == vl * a->L && a->o_sh == kDV && a->o_sl == ol &&
+                       a->o_sb == ol * a->L;
+    return dense ? SINKATTN_OK : SINKATTN_ERR_UNSUPPORTED;
+}
+
+int run_prefill_host(const sinkattn_prefill_args *a, int window, int chunk, void *ws,
+                     size_t ws_bytes, void *stream)
+{
+    int st = validate_host_prefill(a, window, chunk);
+    if (st != SINKATTN_OK)
+        return st;
+    if (a->B == 0 || a->L == 0)
+        return SINKATTN_OK;
+    const HostLayout h = host_layout(a, chunk);
+    if (!ws || ws_bytes < h.total)
+        return !ws ? SINKATTN_ERR_INVALID_ARG : SINKATTN_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned16(ws))
+        return SINKATTN_ERR_ALIGNMENT;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const cudaStream_t s_comp = (cudaStream_t)stream;
+    cudaStream_t s_in = nullptr, s_out = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_in[2] = {}, ev_comp[2] = {}, ev_out[2] = {};
+    cudaError_t e = cudaStreamCreateWithFlags(&s_in, cudaStreamNonBlocking);
+    if (e == cudaSuccess)
+        e = cudaStreamCreateWithFlags(&s_out, cudaStreamNonBlocking);
+    if (e == cudaSuccess)
+        e = cudaEventCreateWithFlags(&ev_start, cudaEventDisableTiming);
+    for (int x = 0; x < 2 && e == cudaSuccess; ++x) {
+        e = cudaEventCreateWithFlags(&ev_in[x], cudaEventDisableTiming);
+        if (e == cudaSuccess)
+            e = cudaEventCreateWithFlags(&ev_comp[x], cudaEventDisableTiming);
+        if (e == cudaSuccess)
+            e = cudaEventCreateWithFlags(&ev_out[x], cudaEventDisableTiming);
+    }
+    // the copies start after the caller's earlier work on `stream`
+    if (e == cudaSuccess)
+        e = cudaEventRecord(ev_start, s_comp);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(s_in, ev_start, 0);
+    if (e == cudaSuccess)
+        e = cudaStreamWaitEvent(s_out, ev_start, 0);
+    const uint8_t *hq = static_cast<const uint8_t *>(a->q), *hk = static_cast<const uint8_t *>(a->k);
+    const uint8_t *hv = static_cast<const uint8_t *>(a->v);
+    uint8_t *ho = static_cast<uint8_t *>(a->o);
+    uint8_t *hl = reinterpret_cast<uint8_t *>(a->lse);
+    for (int64_t c = 0; c < h.n_chunks && e == cudaSuccess && st == SINKATTN_OK; ++c) {
+        const int x = (int)(c & 1);
+        const int64_t c0 = c * h.chunk, lc = std::min<int64_t>(h.chunk, a->L - c0);
+        // in: Q of the chunk into buffer x (free once chunk c - 2 has computed), K and V rows
+        if (c >= 2)
+            e = cudaStreamWaitEvent(s_in, ev_comp[x], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(w + h.off_q[x], h.chunk * h.qrow, hq + c0 * h.qrow, a->L * h.qrow,
+                                  lc * h.qrow, a->B, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(w + h.off_k + c0 * h.krow, a->L * h.krow, hk + c0 * h.krow,
+                                  a->L * h.krow, lc * h.krow, a->B, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(w + h.off_v + c0 * h.vrow, a->L * h.vrow, hv + c0 * h.vrow,
+                                  a->L * h.vrow, lc * h.vrow, a->B, cudaMemcpyHostToDevice, s_in);
+        if (e == cudaSuccess)
+            e = cudaEventRecord(ev_in[x], s_in);
+        // compute: the chunk's rows against keys 0 .. c0 + lc - 1, into O / LSE buffer x (free
+        // once chunk c - 2 has gone out)
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(s_comp, ev_in[x], 0);
+        if (e == cudaSuccess && c >= 2)
+            e = cudaStreamWaitEvent(s_comp, ev_out[x], 0);
+        if (e != cudaSuccess)
+            break;
+        sinkattn_prefill_args ac = *a;
+        ac.q = w + h.off_q[x];
+        ac.k = w + h.off_k;
+        ac.v = w + h.off_v;
+        ac.o = w + h.off_o[x];
+        ac.lse = a->lse ? reinterpret_cast<float *>(w + h.off_lse[x]) : nullptr;
+        ac.L = (int32_t)lc;
+        ac.q_sb = h.chunk * (h.qrow / 2);
+        ac.o_sb = h.chunk * (h.orow / 2);
+        st = run_prefill(&ac, window, (int)c0, s_comp);
+        if (st != SINKATTN_OK)
+            break;
+        e = cudaEventRecord(ev_comp[x], s_comp);
+        // out: O rows and the LSE runs of every (sequence, head)
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(s_out, ev_comp[x], 0);
+        if (e == cudaSuccess)
+            e = cudaMemcpy2DAsync(ho + c0 * h.orow, a->L * h.orow, w + h.off_o[x], h.chunk * h.orow,
+                                  lc * h.orow, a->B, cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess && a->lse)
+            e = cudaMemcpy2DAsync(hl + c0 * 4, (size_t)a->L * 4, w + h.off_lse[x], (size_t)lc * 4,
+                                  lc * 4, (size_t)a->B * a->Hq, cudaMemcpyDeviceToHost, s_out);
+        if (e == cudaSuccess)
+            e = cudaEventRecord(ev_out[x], s_out);
+    }
+    // the caller's stream completes only after the last copy out
+    if (e == cudaSuccess && st == SINKATTN_OK)
+        e = cudaStreamWaitEvent(s_comp, ev_out[(h.n_chunks - 1) & 1], 0);
+    if (e == cudaSuccess && st == SINKATTN_OK && h.n_chunks >= 2)
+        e = cudaStreamWaitEvent(s_comp, ev_out[h.n_chunks & 1], 0);
+    // streams and events are released once their pending work is done
+    for (int x = 0; x < 2; ++x) {
+        if (ev_in[x])
+            cudaEventDestroy(ev_in[x]);
+        if (ev_comp[x])
+            cudaEventDestroy(ev_comp[x]);
+        if (ev_out[x])
+            cudaEventDestroy(ev_out[x]);
+    }
+    if (ev_start)
+        cudaEventDestroy(ev_start);
+    if (s_in)
+        cudaStreamDestroy(s_in);
+    if (s_out)
+        cudaStreamDestroy(s_out);
+    if (st != SINKATTN_OK)
+        return st;
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 
@@ -735,6 +906,20 @@ int sinkattn_prefill_chunk_paged(const sinkattn_prefill_args *args,
     if (window < 0 || !prefix_kv)
         return SINKATTN_ERR_INVALID_ARG;
     return run_prefill(args, window, prefix, stream, prefix_kv);
+}
+
+size_t sinkattn_prefill_host_workspace_size(const sinkattn_prefill_args *args, int32_t chunk)
+{
+    if (!args || chunk <= 0 || chunk % 128 != 0 || args->B <= 0 || args->L <= 0 ||
+        args->Hq <= 0 || args->Hkv <= 0)
+        return 0;
+    return host_layout(args, chunk).total;
+}
+
+int sinkattn_prefill_host(const sinkattn_prefill_args *args, int32_t window, int32_t chunk,
+                          void *workspace, size_t ws_bytes, void *stream)
+{
+    return run_prefill_host(args, window, chunk, workspace, ws_bytes, stream);
 }
 
 size_t sinkattn_decode_workspace_size(const sinkattn_decode_args *args)

@@ -165,6 +165,31 @@ int sinkattn_prefill_chunk_paged(const sinkattn_prefill_args *args,
                                  const sinkattn_paged_kv *prefix_kv, int32_t prefix,
                                  int32_t window, void *stream);
 
+/* Prefill with the inputs and outputs in HOST memory (a prompt that arrives from the host and
+ * whose O and LSE go back to it; the "MiMo-V2-Flash" model card's serving command prefills
+ * prompts in chunks, --chunked-prefill-size 16384). The sequences pass through the device in
+ * chunks of `chunk` positions: while chunk c is computed, chunk c + 1 is copied in and chunk
+ * c - 1 copied out, on two internal streams, so both PCIe directions and the kernels overlap.
+ * Each chunk is the chunked prefill of its rows against every earlier key (window = 0: full
+ * causal, GA; window >= 1: sliding window, SWA), so the result equals sinkattn_prefill_swa / _ga
+ * on the whole sequences.
+ *   args->q, k, v:   HOST, dense [B, L, H, d] (the strides in args must say so), read;
+ *   args->o, lse:    HOST, dense o [B, L, Hq, 128] and lse [B, Hq, L] (lse may be NULL), written;
+ *   args->sink:      DEVICE fp32 [Hq] or NULL, as for the device calls;
+ *   chunk:           positions per chunk, a multiple of 128;
+ *   workspace:       DEVICE memory of sinkattn_prefill_host_workspace_size(args, chunk) bytes
+ *                    (K and V of all positions, two chunks of Q, O and LSE), owned by the caller.
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister): pageable memory works
+ * but its copies do not overlap. The call returns once the work is queued; the outputs are
+ * complete when `stream` reaches the end of this call's work (e.g. after cudaStreamSynchronize).
+ * The two copy streams and their events are created and released by each call.
+ * Errors: as sinkattn_prefill_swa; UNSUPPORTED for non-dense strides or a chunk that is not a
+ * multiple of 128; INVALID_ARG for a NULL workspace, chunk <= 0 or window < 0;
+ * WORKSPACE_TOO_SMALL below the size query. The size query returns 0 for invalid arguments. */
+size_t sinkattn_prefill_host_workspace_size(const sinkattn_prefill_args *args, int32_t chunk);
+int sinkattn_prefill_host(const sinkattn_prefill_args *args, int32_t window, int32_t chunk,
+                          void *workspace, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Decode / speculative verify: T (1..4) new query tokens per sequence attend to that sequence's
  * cached tokens plus new tokens 0..t. The new tokens' K/V are passed separately and are NOT yet

@@ -131,6 +131,31 @@ def test_chunk_checks_prefix_and_window(L):
     assert L.sinkattn_prefill_chunk(None, 0, 0, None) == 1
 
 
+def test_host_prefill_sizes_and_checks(L):
+    """The host-resident prefill: the workspace size follows from the shapes alone (K and V of
+    every position, two chunks of Q, O and LSE); arguments are checked before any device work."""
+    a = _prefill_args()  # B 1, L 64, 8 / 1 heads, dense strides
+    L.sinkattn_prefill_host_workspace_size.restype = ctypes.c_size_t
+    size = L.sinkattn_prefill_host_workspace_size(ctypes.byref(a), 128)
+    al = lambda x: (x + 255) // 256 * 256
+    want = al(64 * 1 * 384) + al(64 * 1 * 256) + 2 * (al(128 * 8 * 384) + al(128 * 8 * 256) + al(8 * 128 * 4))
+    assert size == want
+    assert L.sinkattn_prefill_host_workspace_size(ctypes.byref(a), 100) == 0
+    assert L.sinkattn_prefill_host_workspace_size(ctypes.byref(a), 0) == 0
+    assert L.sinkattn_prefill_host_workspace_size(None, 128) == 0
+    ws = ctypes.c_void_p(0x20000)
+    host = L.sinkattn_prefill_host
+    host.argtypes = [ctypes.POINTER(sa.PrefillArgs), ctypes.c_int32, ctypes.c_int32,
+                     ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    assert host(ctypes.byref(a), 128, 100, ws, size, None) == 2          # chunk not 128-aligned
+    assert host(ctypes.byref(a), 128, 0, ws, size, None) == 1            # chunk <= 0
+    assert host(ctypes.byref(a), -1, 128, ws, size, None) == 1           # negative window
+    assert host(ctypes.byref(_prefill_args(k_sl=384)), 128, 128, ws, size, None) == 2  # not dense
+    assert host(ctypes.byref(a), 128, 128, None, size, None) == 1        # no workspace
+    assert host(ctypes.byref(a), 128, 128, ws, size - 1, None) == 4      # workspace too small
+    assert host(ctypes.byref(_prefill_args(L=0)), 128, 128, None, 0, None) == 0
+
+
 def test_prefill_empty_is_ok_and_window_checked(L):
     assert L.sinkattn_prefill_ga(ctypes.byref(_prefill_args(L=0)), None) == 0
     assert L.sinkattn_prefill_ga(ctypes.byref(_prefill_args(B=0, q=None)), None) == 0
