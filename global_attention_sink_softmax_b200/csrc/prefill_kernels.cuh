@@ -24,8 +24,9 @@
 //              one of three S buffers in TMEM, O += P V (M128 N128 K16 x 8, A = P from TMEM)
 //              into O in TMEM (3 x 128 S columns + 128 O columns fill the 512). S_{j+3}
 //              reuses the buffer of P_j once P_j V_j is done, long after it was issued.
-// The issue order S_0, {S_{j+1}, PV_j} lets the tensor cores compute S_{j+1} while the softmax
-// warps work on S_j; the softmax waits for PV_{j-1} only when it has to rescale O.
+// The issue order S_0, S_1, {PV_j, S_{j+2}} keeps S two tiles ahead: the tensor cores compute
+// S_{j+2} while the softmax warps work on S_j, and S_{j+1} is ready when they finish; the
+// softmax waits for PV_{j-1} only when it has to rescale O.
 //
 // Two row sums: O is normalised by the sum of the bf16-rounded P values (the ones the P.V MMA
 // multiplies), so numerator and denominator use identical weights; LSE uses the fp32 sum.
@@ -231,11 +232,15 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 umma_commit(&bars[B_KEMPTY + ks]);
                 return true;
             };
+            // S runs two tiles ahead of P.V: S_0, S_1, then {P.V_idx, S_{idx+2}}. S_{idx+2} goes
+            // into the buffer of P_{idx-1}, whose P.V was issued a whole group earlier, so the
+            // tensor pipe always has work that does not wait for the softmax, and the softmax
+            // warps find S_{idx+1} done when they finish P_idx.
             if (ok)
                 ok = issue_s(0);
+            if (ok && n_tiles > 1)
+                ok = issue_s(1);
             for (int idx = 0; ok && idx < n_tiles; ++idx) {
-                if (idx + 1 < n_tiles && !issue_s(idx + 1))
-                    break;
                 const int sb = idx % S_BUFS, vs = idx & 1;
                 if (!mbar_wait(&bars[B_PFULL + sb], (idx / S_BUFS) & 1, abort, 1u))
                     break;
@@ -254,6 +259,8 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 }
                 umma_commit(&bars[B_PVDONE + sb]);
                 umma_commit(&bars[B_VEMPTY + vs]);
+                if (idx + 2 < n_tiles && !issue_s(idx + 2))
+                    break;
             }
             // every MMA of ours has finished before TMEM is released
             umma_commit(&bars[B_DRAIN]);
