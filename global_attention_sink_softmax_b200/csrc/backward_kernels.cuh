@@ -112,9 +112,11 @@ SA_DEV void tmem_st16(uint32_t taddr, const uint32_t (&w)[16])
 // dQ: one CTA per (128-row query tile, sequence, head)
 // ---------------------------------------------------------------------------------------------
 // Per key tile j of the band: S = Q K_j^T and dP = dO V_j^T into tensor memory; the row warps
-// (thread = query row) turn them into dS = P (dP - delta) as bf16 pairs over S's first 64
-// columns; dQ += dS K_j with K_j as the MN-major B operand. K is double-buffered (it serves S
-// and dQ), V single-buffered (it serves dP only). S_{j+1} is issued once dQ_j has read dS_j.
+// (thread = query row) turn them into dS = P (dP - delta) as bf16 pairs in 64 columns of their
+// own; dQ += dS K_j with K_j as the MN-major B operand. K is double-buffered (it serves S and
+// dQ), V single-buffered (it serves dP only). S_{j+1} is issued as soon as the row warps have
+// read S_j and dP_j (SDP_FREE), so it runs while they compute dS_j; dP_{j+1} follows dQ_j
+// (V_{j+1} lands after dP_j has read V_j); the row warps store dS_{j+1} once dQ_j has read dS_j.
 namespace bq {
 using namespace bw;
 constexpr int OFF_Q = 0;                  // 3 x 16 KB
@@ -123,9 +125,9 @@ constexpr int OFF_K = OFF_DO + 2 * R128;  // 2 stages x 48 KB
 constexpr int OFF_V = OFF_K + 6 * R128;   // 32 KB
 constexpr int OFF_BAR = OFF_V + 2 * R128;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
-constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256; // tensor-memory columns
+constexpr uint32_t T_S = 0, T_DP = 128, T_DQ = 256, T_DS = 448; // tensor-memory columns
 enum Bar { QD_FULL = 0, K_FULL = 1, K_EMPTY = 3, V_FULL = 5, V_EMPTY = 6, S_FULL = 7, DS_FULL = 8,
-           DQ_DONE = 9, DRAIN = 10, NUM_BARS = 11 };
+           DQ_DONE = 9, DRAIN = 10, SDP_FREE = 11, NUM_BARS = 12 };
 } // namespace bq
 
 __global__ void __launch_bounds__(bw::THREADS, 1)
@@ -157,7 +159,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NUM_BARS; ++i)
-            mbar_init(&bars[i], i == DS_FULL ? 128 : 1);
+            mbar_init(&bars[i], (i == DS_FULL || i == SDP_FREE) ? 128 : 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -213,15 +215,12 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
             const uint32_t sQ = smem_u32(smem + OFF_Q), sDO = smem_u32(smem + OFF_DO);
             const uint32_t sK = smem_u32(smem + OFF_K), sV = smem_u32(smem + OFF_V);
             bool ok = mbar_wait(&bars[QD_FULL], 0, abort, 1u);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int ks = j & 1;
-                const uint32_t kb = sK + ks * 3 * R128;
-                if (!mbar_wait(&bars[K_FULL + ks], (j >> 1) & 1, abort, 1u) ||
-                    !mbar_wait(&bars[V_FULL], j & 1, abort, 1u))
-                    break;
-                // S is rewritten only after dQ_{j-1} has read the dS that lies over it
-                if (j >= 1 && !mbar_wait(&bars[DQ_DONE], (j - 1) & 1, abort, 1u))
-                    break;
+            // S_j = Q K_j^T (its K stage landed) and dP_j = dO V_j^T (V landed); both into
+            // columns the row warps have finished reading for tile j - 1
+            auto issue_s = [&](int j) -> bool {
+                const uint32_t kb = sK + (j & 1) * 3 * R128;
+                if (!mbar_wait(&bars[K_FULL + (j & 1)], (j >> 1) & 1, abort, 1u))
+                    return false;
                 tc_fence_after();
 #pragma unroll 1
                 for (int kk = 0; kk < 12; ++kk) {
@@ -229,6 +228,12 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
                     umma_ss(tmem + T_S, smem_desc_sw128(sQ + off, 16, 1024),
                             smem_desc_sw128(kb + off, 16, 1024), idesc_s, kk > 0);
                 }
+                return true;
+            };
+            auto issue_dp = [&](int j) -> bool {
+                if (!mbar_wait(&bars[V_FULL], j & 1, abort, 1u))
+                    return false;
+                tc_fence_after();
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint32_t off = (kk >> 2) * R128 + (kk & 3) * 32;
@@ -237,6 +242,18 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
                 }
                 umma_commit(&bars[S_FULL]);
                 umma_commit(&bars[V_EMPTY]);
+                return true;
+            };
+            if (ok && n_tiles > 0)
+                ok = issue_s(0) && issue_dp(0);
+            // tile j + 1's S runs while the row warps turn tile j into dS, and its dP after
+            // dQ_j (V_{j+1} is loaded only once dP_j has read V_j)
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int ks = j & 1;
+                const uint32_t kb = sK + ks * 3 * R128;
+                const bool more = j + 1 < n_tiles;
+                if (more && (!mbar_wait(&bars[SDP_FREE], j & 1, abort, 1u) || !issue_s(j + 1)))
+                    break;
                 if (!mbar_wait(&bars[DS_FULL], j & 1, abort, 1u))
                     break;
                 tc_fence_after();
@@ -244,11 +261,13 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
                 // B = K_j (16 keys x 192 dims, dims contiguous: MN-major, 64-dim regions 16 KB apart)
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)
-                    umma_ts(tmem + T_DQ, tmem + T_S + kk * 8,
+                    umma_ts(tmem + T_DQ, tmem + T_DS + kk * 8,
                             smem_desc_sw128(kb + kk * 16 * ROW, R128, 1024), idesc_q,
                             (j > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&bars[DQ_DONE]);
                 umma_commit(&bars[K_EMPTY + ks]);
+                if (more && !issue_dp(j + 1))
+                    break;
             }
             // every MMA of ours has finished before TMEM is released
             umma_commit(&bars[DRAIN]);
@@ -279,6 +298,11 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
             for (int c = 0; c < 4; ++c) {
                 uint32_t s[32], dp[32];
                 tmem_ld32x2_sync(tmem + lane_addr + T_S + c * 32, s, tmem + lane_addr + T_DP + c * 32, dp);
+                if (c == 3) {
+                    // tile j's S and dP are all read: the issuer may compute tile j + 1's
+                    tc_fence_before();
+                    mbar_arrive(&bars[SDP_FREE]);
+                }
                 uint32_t w[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -292,9 +316,17 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
                     }
                     w[e] = pack_bf16x2(d2[0], d2[1]);
                 }
-                // dS (bf16 pairs) over columns 16c .. 16c + 15 of S: S chunks <= c are read
-                tmem_st16(tmem + lane_addr + T_S + c * 16, w);
+                // dS (bf16 pairs) into its own 64 columns, once dQ_{j-1} has read tile j - 1's
+                if (c == 0 && j > 0) {
+                    ok = warp_wait(&bars[DQ_DONE], (j - 1) & 1, abort);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                }
+                tmem_st16(tmem + lane_addr + T_DS + c * 16, w);
             }
+            if (!ok)
+                break;
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars[DS_FULL]);
@@ -339,7 +371,10 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
 // rows) into tensor memory; the row warps (thread = key row) form P^T = exp(S^T c - LSE) and
 // dS^T = P^T (dP^T - delta) for the 64 rows, as bf16 pairs in their own columns; then
 // dV += P^T dO and dK += dS^T Q, with dO and Q as MN-major B operands. A step's Q, dO, LSE and
-// delta come in a 3-stage ring.
+// delta come in a 3-stage ring. The two halves of a step overlap with the neighbouring steps:
+// S^T and dP^T of step s + 1 are computed as soon as the row warps have read those of step s
+// (SDP_FREE), while the row warps work, and the row warps store P^T / dS^T of step s + 1 once the
+// dV / dK MMAs of step s have read theirs (DKV_DONE).
 namespace bk {
 using namespace bw;
 constexpr int QB = 64;                         // query rows per step
@@ -355,7 +390,7 @@ constexpr int OFF_BAR = OFF_ST + NST * STAGE;
 constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
 constexpr uint32_t T_S = 0, T_DP = 64, T_P = 128, T_DS = 160, T_DV = 192, T_DK = 320;
 enum Bar { KV_FULL = 0, ST_FULL = 1, ST_EMPTY = 4, S_FULL = 7, P_FULL = 8, DONE = 9,
-           NUM_BARS = 10 };
+           SDP_FREE = 10, DKV_DONE = 11, NUM_BARS = 12 };
 } // namespace bk
 
 __global__ void __launch_bounds__(bw::THREADS, 1)
@@ -388,7 +423,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NUM_BARS; ++i)
-            mbar_init(&bars[i], i == P_FULL ? 128 : 1);
+            mbar_init(&bars[i], (i == P_FULL || i == SDP_FREE) ? 128 : 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -457,21 +492,23 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
             const uint32_t idesc_k = umma_idesc_bf16(128, 192, 1);
             const uint32_t sK = smem_u32(smem + OFF_K), sV = smem_u32(smem + OFF_V);
             bool ok = mbar_wait(&bars[KV_FULL], 0, abort, 1u);
-            for (int s = 0; ok && s < n_steps; ++s) {
+            // S^T = K Q^T and dP^T = V dO^T of step s into their columns (the row warps have read
+            // those of step s - 1)
+            auto issue_sdp = [&](int s) -> bool {
                 const int st = s % NST;
                 const uint32_t sQ = smem_u32(smem + OFF_ST + st * STAGE + ST_Q);
                 const uint32_t sDO = smem_u32(smem + OFF_ST + st * STAGE + ST_DO);
                 if (!mbar_wait(&bars[ST_FULL + st], (s / NST) & 1, abort, 1u))
-                    break;
+                    return false;
                 tc_fence_after();
-                // S^T = K Q^T (A: 128 keys, K-major; B: 64 rows, K-major), 12 k-steps of 16 dims
+                // S^T: A = 128 keys (K-major), B = 64 rows (K-major), 12 k-steps of 16 dims
 #pragma unroll 1
                 for (int kk = 0; kk < 12; ++kk)
                     umma_ss(tmem + T_S,
                             smem_desc_sw128(sK + (kk >> 2) * R128 + (kk & 3) * 32, 16, 1024),
                             smem_desc_sw128(sQ + (kk >> 2) * R64 + (kk & 3) * 32, 16, 1024),
                             idesc_s, kk > 0);
-                // dP^T = V dO^T, 8 k-steps of 16 dims
+                // dP^T, 8 k-steps of 16 dims
 #pragma unroll 1
                 for (int kk = 0; kk < 8; ++kk)
                     umma_ss(tmem + T_DP,
@@ -479,6 +516,19 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
                             smem_desc_sw128(sDO + (kk >> 2) * R64 + (kk & 3) * 32, 16, 1024),
                             idesc_s, kk > 0);
                 umma_commit(&bars[S_FULL]);
+                return true;
+            };
+            if (ok && n_steps > 0)
+                ok = issue_sdp(0);
+            for (int s = 0; ok && s < n_steps; ++s) {
+                const int st = s % NST;
+                const uint32_t sQ = smem_u32(smem + OFF_ST + st * STAGE + ST_Q);
+                const uint32_t sDO = smem_u32(smem + OFF_ST + st * STAGE + ST_DO);
+                // step s + 1's S^T / dP^T, once the row warps hold step s's
+                if (s + 1 < n_steps) {
+                    if (!mbar_wait(&bars[SDP_FREE], s & 1, abort, 1u) || !issue_sdp(s + 1))
+                        break;
+                }
                 if (!mbar_wait(&bars[P_FULL], s & 1, abort, 1u))
                     break;
                 tc_fence_after();
@@ -495,6 +545,7 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
                             (s > 0 || kk > 0) ? 1u : 0u);
                 }
                 umma_commit(&bars[ST_EMPTY + st]);
+                umma_commit(&bars[DKV_DONE]);
             }
             // every MMA of ours has finished before the row warps read dK / dV and TMEM is freed
             umma_commit(&bars[DONE]);
@@ -525,6 +576,11 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
             for (int c = 0; c < 2; ++c) {
                 uint32_t sv[32], dp[32];
                 tmem_ld32x2_sync(tmem + lane_addr + T_S + c * 32, sv, tmem + lane_addr + T_DP + c * 32, dp);
+                if (c == 1) {
+                    // step s's S^T / dP^T are all read: the issuer may compute step s + 1's
+                    tc_fence_before();
+                    mbar_arrive(&bars[SDP_FREE]);
+                }
                 uint32_t wp[16], wd[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
@@ -539,9 +595,18 @@ __global__ void __launch_bounds__(bw::THREADS, 1)
                     wp[e] = pack_bf16x2(pr[0], pr[1]);
                     wd[e] = pack_bf16x2(ds[0], ds[1]);
                 }
+                // P^T / dS^T of step s - 1 must have been read by its dV / dK MMAs
+                if (c == 0 && s > 0) {
+                    ok = warp_wait(&bars[DKV_DONE], (s - 1) & 1, abort);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                }
                 tmem_st16(tmem + lane_addr + T_P + c * 16, wp);
                 tmem_st16(tmem + lane_addr + T_DS + c * 16, wd);
             }
+            if (!ok)
+                break;
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars[P_FULL]);
