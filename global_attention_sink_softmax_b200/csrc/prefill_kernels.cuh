@@ -289,31 +289,34 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             if (!ok)
                 break;
             tc_fence_after();
-            uint32_t raw[128];
-            tmem_ld128(tmem + lane_addr + sb * BN, raw);
-            float x[128]; // raw scores q.k; masked keys -inf
+            // Two passes over the row's 128 scores, 32 columns per TMEM load: the row maximum,
+            // then P. The loops over the four chunks stay rolled, which keeps the code of this
+            // warp small: it shares each SMSP's instruction cache with the producer and UMMA
+            // issuer warps, whose issue gaps on a miss idle the tensor pipe.
+            const uint32_t saddr = tmem + lane_addr + sb * BN;
             // mask only on tiles that cross the diagonal or the window's lower edge
             const bool need_mask = (kbase + BN - 1 > a0) ||
                                    (p.window > 0 && kbase < a0 + BM - p.window);
+            const int hi = ap - kbase;                                       // keep c <= hi
+            const int lo = (p.window > 0) ? ap - p.window + 1 - kbase : -BN; // keep c >= lo
             // eight independent running maxima: short dependency chains
             float mx8[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
                 mx8[i] = -INFINITY;
-            if (need_mask) {
-                const int hi = ap - kbase;                                   // keep c <= hi
-                const int lo = (p.window > 0) ? ap - p.window + 1 - kbase : -BN; // keep c >= lo
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32_sync(saddr + c0, r);
+                if (need_mask) {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    x[c] = (c <= hi && c >= lo) ? __uint_as_float(raw[c]) : -INFINITY;
-                    mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
+                    for (int e = 0; e < 32; ++e)
+                        if (c0 + e > hi || c0 + e < lo)
+                            r[e] = __float_as_uint(-INFINITY);
                 }
-            } else {
 #pragma unroll
-                for (int c = 0; c < 128; ++c) {
-                    x[c] = __uint_as_float(raw[c]);
-                    mx8[c & 7] = fmaxf(mx8[c & 7], x[c]);
-                }
+                for (int e = 0; e < 32; ++e)
+                    mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(r[e]));
             }
             float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 if (!ok)
                     break;
                 tc_fence_after();
-#pragma unroll
+#pragma unroll 1
                 for (int c = 0; c < 4; ++c) {
                     uint32_t o[32];
                     tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * 32, o);
@@ -350,20 +353,30 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             }
             const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
             float pe[4] = {0.f, 0.f, 0.f, 0.f}, pr[4] = {0.f, 0.f, 0.f, 0.f};
-            // P (bf16 pairs: keys 2c, 2c + 1 in column c) over this row's S in TMEM
-            const uint32_t paddr = tmem + lane_addr + sb * BN;
+            // P (bf16 pairs: keys 2c, 2c + 1 in column c) over this row's S in TMEM: chunk c0's
+            // 16 columns of P land on scores already read (columns < c0 + 32)
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32_sync(saddr + c0, r);
+                if (need_mask) {
 #pragma unroll
-            for (int c16 = 0; c16 < 8; ++c16) {
-                uint32_t pk[8];
+                    for (int e = 0; e < 32; ++e)
+                        if (c0 + e > hi || c0 + e < lo)
+                            r[e] = __float_as_uint(-INFINITY);
+                }
+                uint32_t pk[16];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const float e0 = fast_exp2(fmaf(x[c16 * 16 + 2 * u], c_l2, neg_m));
-                    const float e1 = fast_exp2(fmaf(x[c16 * 16 + 2 * u + 1], c_l2, neg_m));
+                for (int u = 0; u < 16; ++u) {
+                    const float e0 = fast_exp2(fmaf(__uint_as_float(r[2 * u]), c_l2, neg_m));
+                    const float e1 = fast_exp2(fmaf(__uint_as_float(r[2 * u + 1]), c_l2, neg_m));
                     pk[u] = pack_bf16x2(e0, e1);
                     pe[u & 3] += e0 + e1;
                     pr[u & 3] += sum_bf16x2(pk[u]);
                 }
-                tmem_st8(paddr + c16 * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+                tmem_st8(saddr + c0 / 2, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
+                tmem_st8(saddr + c0 / 2 + 8, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14],
+                         pk[15]);
             }
             l_exact += (pe[0] + pe[1]) + (pe[2] + pe[3]);
             l_round += (pr[0] + pr[1]) + (pr[2] + pr[3]);
