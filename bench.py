@@ -96,9 +96,10 @@ def decode_counts(w, d):
 # ----------------------------------------------------------------------------------------------
 
 class PrefillRunner:
-    def __init__(self, w, dev):
+    def __init__(self, w, dev, fused_rope=False):
         import global_attention_sink_softmax_b200 as sa
         self.sa, self.w, self.dev = sa, w, dev
+        self.fused_rope = fused_rope
         self.d = W.prefill_inputs(w, device=dev, L=w.prefix + w.L)
         if w.prefix:
             self.d["q"] = self.d["q"][:, w.prefix:]  # the chunk's queries (a strided view)
@@ -114,11 +115,18 @@ class PrefillRunner:
                            window=w.window, kind="SWA" if w.window else "GA")
         if w.prefix:
             self.config["prefix"] = w.prefix
+        if fused_rope:
+            # the SWA layers' partial RoPE (64 dims, theta 1e4) and value scale, in the loads
+            self.workload = w.name + "_fused_rope"
+            self.config.update(rope_dim=sa.ROPE_DIM, theta=sa.ROPE_THETA_SWA, v_scale=sa.V_SCALE)
         self.in_bytes = sum(self.d[k].numel() * self.d[k].element_size() for k in self.d)
 
     def step(self):
         d, w = self.d, self.w
-        if w.prefix:
+        if self.fused_rope:
+            self.sa.sinkattn_prefill_swa_rope(d["q"], d["k"], d["v"], d["sink"], w.window,
+                                              theta=self.sa.ROPE_THETA_SWA, o=self.o, lse=self.lse)
+        elif w.prefix:
             self.sa.sinkattn_prefill_chunk(d["q"], d["k"], d["v"], d["sink"], prefix=w.prefix,
                                            window=w.window, o=self.o, lse=self.lse)
         elif w.window:
@@ -709,7 +717,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--only", default=None,
                     help="run one workload only: swa_prefill, ga_prefill, ga_chunk_prefill, "
-                         "ga_backward, ga_decode, ga_decode_fp8, swa_decode, hybrid, rope")
+                         "ga_backward, ga_decode, ga_decode_fp8, swa_decode, hybrid, rope, "
+                         "swa_prefill_rope")
     ap.add_argument("--ref-rows", type=int, default=128)
     ap.add_argument("--ref-L", type=int, default=0, help="reference arm: shorter sequences (tests)")
     ap.add_argument("--small", action="store_true",
@@ -798,6 +807,9 @@ def main():
             jobs.append(("ga_chunk_prefill", lambda: PrefillRunner(gac_w, dev), None))
         if only in (None, "rope"):
             jobs.append(("rope_qkv", lambda: RopeRunner(swa_w, dev, 1e4), None))
+        if only in (None, "swa_prefill_rope"):
+            # the headline workload with the RoPE pass fused into the prefill's loads
+            jobs.append(("swa_prefill_fused_rope", lambda: PrefillRunner(swa_w, dev, True), None))
         if only in (None, "ga_backward"):
             jobs.append(("ga_prefill_backward", lambda: BackwardRunner(ga_w, dev), None))
         if only in (None, "ga_decode"):

@@ -30,6 +30,7 @@ __all__ = [
     "ROPE_THETA_GA", "ROPE_THETA_SWA", "V_SCALE", "KV_BF16", "KV_FP8_E4M3",
     "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward", "sinkattn_prefill_chunk_paged",
     "sinkattn_prefill_host", "sinkattn_prefill_host_workspace_size", "HOST_CHUNK",
+    "sinkattn_prefill_swa_rope",
 ]
 
 KV_RING, KV_CONTIG, KV_PAGED = 0, 1, 2
@@ -45,7 +46,7 @@ EXPORTED_SYMBOLS = [
     "sinkattn_take_device_error", "sinkattn_decode_noalloc", "sinkattn_rope_qkv",
     "sinkattn_set_wait_limit_ns", "sinkattn_prefill_backward_workspace_size",
     "sinkattn_prefill_backward", "sinkattn_prefill_chunk_paged",
-    "sinkattn_prefill_host_workspace_size", "sinkattn_prefill_host",
+    "sinkattn_prefill_host_workspace_size", "sinkattn_prefill_host", "sinkattn_prefill_swa_rope",
 ]
 # Positions per chunk of the host-resident prefill (its copies in and out overlap chunk by chunk).
 HOST_CHUNK = 4096
@@ -71,6 +72,11 @@ class PrefillArgs(ctypes.Structure):
                 ("k_sb", _I64), ("k_sl", _I64), ("k_sh", _I64),
                 ("v_sb", _I64), ("v_sl", _I64), ("v_sh", _I64),
                 ("o_sb", _I64), ("o_sl", _I64), ("o_sh", _I64)]
+
+
+class RopeSpec(ctypes.Structure):
+    _fields_ = [("pos_base", _P), ("pos0", _I64), ("rope_dim", _I32), ("theta", ctypes.c_double),
+                ("v_scale", _F32)]
 
 
 class RopeArgs(ctypes.Structure):
@@ -157,6 +163,9 @@ def lib() -> ctypes.CDLL:
             L.sinkattn_prefill_host_workspace_size.restype = _SZ
             L.sinkattn_prefill_host.argtypes = [ctypes.POINTER(PrefillArgs), _I32, _I32, _P, _SZ, _P]
             L.sinkattn_prefill_host.restype = ctypes.c_int
+            L.sinkattn_prefill_swa_rope.argtypes = [ctypes.POINTER(PrefillArgs), _I32,
+                                                    ctypes.POINTER(RopeSpec), _P]
+            L.sinkattn_prefill_swa_rope.restype = ctypes.c_int
             L.sinkattn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
             L.sinkattn_set_wait_limit_ns.restype = ctypes.c_int
             _lib = L
@@ -268,6 +277,32 @@ def sinkattn_prefill_swa(q, k, v, sink=None, window=128, *, o=None, lse=None, sc
     strides with a contiguous last dim); sink fp32 [Hq] or None. Returns (o [B,L,Hq,128] bf16,
     lse [B,Hq,L] fp32 or None)."""
     return _prefill("swa", q, k, v, sink, window, o, lse, scale, stream, want_lse)
+
+
+def sinkattn_prefill_swa_rope(q, k, v, sink=None, window=128, *, theta=ROPE_THETA_SWA,
+                              rope_dim=ROPE_DIM, v_scale=V_SCALE, pos0=0, pos_base=None, o=None,
+                              lse=None, scale=None, stream=None, want_lse=True):
+    """Sliding-window prefill with the partial RoPE and the value scale applied as Q, K and V
+    are loaded: the result of sinkattn_rope_qkv(q, k, v, ...) then sinkattn_prefill_swa, without
+    modifying q, k, v. Token l of sequence b sits at position pos0 + pos_base[b] (CUDA int32
+    [B] or None) + l. Takes the GQA-packed path (8 query heads per KV head, window <= 128);
+    other shapes raise SinkAttnError (UNSUPPORTED)."""
+    B, L, Hq, dq = q.shape
+    if scale is None:
+        scale = 1.0 / math.sqrt(dq)
+    if o is None:
+        o = torch.empty(B, L, Hq, v.shape[3], dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, Hq, L, dtype=torch.float32, device=q.device)
+    a = _prefill_args(q, k, v, sink, o, lse, scale)
+    _check_vec("pos_base", pos_base, torch.int32)
+    spec = RopeSpec()
+    spec.pos_base, spec.pos0, spec.rope_dim = _ptr(pos_base), int(pos0), int(rope_dim)
+    spec.theta, spec.v_scale = float(theta), float(v_scale)
+    st = lib().sinkattn_prefill_swa_rope(ctypes.byref(a), int(window), ctypes.byref(spec),
+                                         _stream(stream))
+    _raise(st, "sinkattn_prefill_swa_rope")
+    return o, lse
 
 
 def sinkattn_prefill_ga(q, k, v, sink=None, *, o=None, lse=None, scale=None, stream=None,

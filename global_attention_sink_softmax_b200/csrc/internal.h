@@ -35,6 +35,10 @@ cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                 cudaStream_t stream);
 
 // SWA prefill, GQA-packed persistent kernel: item = (b, kv head, block of P = 128 / G positions)
+// Partial RoPE applied to Q and K as they land in shared memory (rope_dim <= 64: the rotary
+// dims lie in the first 64-dim region of a tile); the value scale multiplies O.
+constexpr int kRopeFusedMaxHalf = 32;
+
 struct SwaParams {
     int B, L, Hq, Hkv, G;
     int P;                // positions per item
@@ -46,6 +50,13 @@ struct SwaParams {
     void *o;
     int64_t o_sb, o_sl, o_sh;
     float *lse;
+    // fused RoPE (rope = 0: Q, K, V taken as given): token l of sequence b at position
+    // pos0 + pos_base[b] + l, pair i turning by position * inv_freq[i]
+    int rope, rope_half;
+    float out_mul; // the value scale (1 without RoPE)
+    const int32_t *pos_base;
+    int64_t pos0;
+    double inv_freq[kRopeFusedMaxHalf];
 };
 
 // Q map box {64, G, P, 1}; K / V map box {64, 1, NS, 1}; K / V chunk map box {64, 1, 16, 1};

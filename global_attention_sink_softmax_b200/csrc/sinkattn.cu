@@ -154,7 +154,8 @@ int device_info(DeviceInfo *out)
 
 // SWA prefill with the GQA group packed into the MMA rows: possible when G divides 128 and the
 // span of P + W - 1 keys (P = 128 / G positions) fits one MMA (<= 256) and shared memory.
-int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *stream, bool *done)
+int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *stream, bool *done,
+                           const sinkattn_rope_spec *rope = nullptr)
 {
     *done = false;
     const int G = a->Hq / a->Hkv;
@@ -205,6 +206,13 @@ int try_prefill_swa_packed(const sinkattn_prefill_args *a, int window, void *str
     p.o_sl = a->o_sl;
     p.o_sh = a->o_sh;
     p.lse = a->lse;
+    p.rope = rope ? 1 : 0;
+    p.rope_half = rope ? rope->rope_dim / 2 : 8;
+    p.out_mul = rope ? rope->v_scale : 1.f;
+    p.pos_base = rope ? rope->pos_base : nullptr;
+    p.pos0 = rope ? rope->pos0 : 0;
+    for (int i = 0; i < kRopeFusedMaxHalf; ++i)
+        p.inv_freq[i] = (rope && i < p.rope_half) ? pow(rope->theta, -2.0 * i / (2.0 * p.rope_half)) : 0.0;
     const int grid = (int)(items < di.sms ? items : di.sms);
     const cudaError_t e =
         launch_prefill_swa_packed(tq, tk, tv, tkc, tvc, p, grid, (cudaStream_t)stream);
@@ -906,6 +914,28 @@ int sinkattn_prefill_chunk_paged(const sinkattn_prefill_args *args,
     if (window < 0 || !prefix_kv)
         return SINKATTN_ERR_INVALID_ARG;
     return run_prefill(args, window, prefix, stream, prefix_kv);
+}
+
+int sinkattn_prefill_swa_rope(const sinkattn_prefill_args *args, int32_t window,
+                              const sinkattn_rope_spec *rope, void *stream)
+{
+    if (window < 1 || !rope)
+        return SINKATTN_ERR_INVALID_ARG;
+    if (!(rope->theta > 0.0) || !isfinite(rope->theta) || !isfinite(rope->v_scale))
+        return SINKATTN_ERR_INVALID_ARG;
+    if (rope->rope_dim < 16 || rope->rope_dim > 2 * kRopeFusedMaxHalf || rope->rope_dim % 16 != 0)
+        return SINKATTN_ERR_UNSUPPORTED;
+    int st = validate_prefill(args);
+    if (st != SINKATTN_OK)
+        return st;
+    if (args->B == 0 || args->L == 0)
+        return SINKATTN_OK;
+    bool done = false;
+    st = try_prefill_swa_packed(args, window, stream, &done, rope);
+    if (st != SINKATTN_OK)
+        return st;
+    // the fused path is the GQA-packed kernel's: other shapes take the separate pass
+    return done ? SINKATTN_OK : SINKATTN_ERR_UNSUPPORTED;
 }
 
 size_t sinkattn_prefill_host_workspace_size(const sinkattn_prefill_args *args, int32_t chunk)

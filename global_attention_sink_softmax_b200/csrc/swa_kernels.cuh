@@ -23,10 +23,12 @@
 //
 // Specialised for the 144-key span of G = 8 query heads per KV head (P = 16) and W <= 128.
 //
-// Roles (384 threads): warps 0-3 and 4-7 softmax + epilogue (even / odd items; thread = row =
+// Roles (480 threads): warps 0-3 and 4-7 softmax + epilogue (even / odd items; thread = row =
 // TMEM lane); warp 8 TMA producer for Q and K, warp 10 for V; warp 9 TMEM allocator +
-// single-thread UMMA issuer, issuing S_0, {S_{n+1}, PV_n}. Waits are bounded as in the band
-// kernel.
+// single-thread UMMA issuer, issuing S_0, {S_{n+1}, PV_n}; warps 11-14 apply the partial RoPE to
+// each Q tile and each new K chunk as they land, when asked to (the rotary dims lie in the first
+// 64-dim region of a tile; the issuer then waits for the rotated tiles instead of the copies),
+// and the value scale multiplies O. Waits are bounded as in the band kernel.
 #pragma once
 #include "common.cuh"
 #include "internal.h"
@@ -34,8 +36,9 @@
 namespace sinkattn {
 
 namespace sw {
-constexpr int THREADS = 384;
+constexpr int THREADS = 480;
 constexpr int WARP_LOAD = 8, WARP_MMA = 9, WARP_VLOAD = 10;
+constexpr int WARP_ROPE = 11, ROPE_WARPS = 4; // warps 11-14 rotate (fused RoPE)
 constexpr int ROW = 128;          // bytes per swizzled row (64 bf16)
 constexpr int Q_REGION = 128 * ROW;
 constexpr int Q_BYTES = 3 * Q_REGION;
@@ -56,12 +59,19 @@ enum Bar {
     P_FULL = 16,  // + warpgroup
     PV_DONE = 18, // + warpgroup
     O_FREE = 20,
-    DRAIN = 21, NUM_BARS
+    DRAIN = 21,
+    Q_ROT = 22,   // + Q buffer: Q rotated (fused RoPE)
+    K_ROT = 24,   // + item parity: the item's new K chunks rotated
+    NUM_BARS = 26
 };
 
 __host__ __device__ constexpr bool counted_by_rows(int i)
 {
     return i == P_FULL || i == P_FULL + 1 || i == O_FREE;
+}
+__host__ __device__ constexpr bool counted_by_rope_warps(int i)
+{
+    return i == Q_ROT || i == Q_ROT + 1 || i == K_ROT || i == K_ROT + 1;
 }
 
 // K and V rings: R = NSC / 16 + P / 16 chunks of 16 keys per 64-dim region (the span plus the
@@ -72,7 +82,15 @@ __host__ __device__ constexpr int v_bytes(int p) { return 2 * ring_chunks(p) * C
 __host__ __device__ constexpr int off_k() { return 2 * Q_BYTES; }
 __host__ __device__ constexpr int off_v(int p) { return off_k() + k_bytes(p); }
 __host__ __device__ constexpr int off_bar(int p) { return off_v(p) + v_bytes(p); }
-__host__ __device__ constexpr int smem_bytes(int p) { return off_bar(p) + 256 + 1024; }
+// Fused RoPE tables: the pair frequencies, then (cos, sin) of the item's P query positions and
+// of its A * 16 new keys, per rotary pair
+__host__ __device__ constexpr int off_rope(int p) { return off_bar(p) + 256; }
+__host__ __device__ constexpr int rope_bytes(int p)
+{
+    return ROPE_WARPS * kRopeFusedMaxHalf * 8 + p * kRopeFusedMaxHalf * 8; // frequencies, table
+}
+__host__ __device__ constexpr int smem_bytes(int p) { return off_rope(p) + rope_bytes(p) + 1024; }
+static_assert(NUM_BARS * 8 + 8 <= 256, "barriers, TMEM slot and abort flag fit their 256 bytes");
 } // namespace sw
 
 struct SwaItem {
@@ -99,6 +117,40 @@ SA_DEV int swa_next_base(const SwaParams &p, const SwaItem &it, int base)
 {
     const int R = sw::ring_chunks(p.P), A = p.P / 16;
     return it.fresh ? 0 : (base + A) % R;
+}
+
+// Rotates the 8 pairs of 16-byte chunk c (dims 8c .. 8c + 7) of a 128-byte swizzled row with
+// their partners nch chunks further on (dims half + 8c ..), in shared memory; cs: the 8 pairs'
+// (cos, sin). Row `row` of a tile (1 KB-aligned atoms of 8 rows) sits at `rowp`.
+SA_DEV void swa_rotate_chunk(uint8_t *rowp, int row, int c, int nch, const float2 *cs)
+{
+    uint4 *a = reinterpret_cast<uint4 *>(rowp + ((c ^ (row & 7)) << 4));
+    uint4 *b = reinterpret_cast<uint4 *>(rowp + (((c + nch) ^ (row & 7)) << 4));
+    uint4 x = *a, y = *b;
+    rope_rotate8(x, y, cs);
+    *a = x;
+    *b = y;
+}
+
+// Fused RoPE of a whole key span (the first item of a run loads all NSC keys into ring slots
+// 0 .. SC - 1): region 0 of key r sits in slot r / 16, row r % 16. Rotator warp rw takes keys
+// r = rw, rw + 4, ...; lane = (key, chunk c). Angles computed here, key by key. Out of line: it
+// runs once per run of items, and its code stays out of the rotators' loop.
+__device__ __noinline__ void swa_rope_span(uint8_t *kring, int ks, int L, int64_t mb, const double *wf,
+                                           int nch, int rw, int lane)
+{
+    const int c = lane & 3;
+    for (int rr = lane >> 2; rr < sw::NSC / sw::ROPE_WARPS; rr += 8) {
+        const int r = rr * sw::ROPE_WARPS + rw;
+        const int key = ks + r;
+        if (c >= nch || key < 0 || key >= L)
+            continue; // a row outside the sequence: zeros from the copy, masked
+        float2 csk[8];
+#pragma unroll 1
+        for (int j = 0; j < 8; ++j)
+            csk[j] = rope_cos_sin(mb + key, wf[c * 8 + j]);
+        swa_rotate_chunk(kring + (r >> 4) * sw::CHUNK + (r & 15) * sw::ROW, r & 15, c, nch, csk);
+    }
 }
 
 // Loads 3 chunks of 16 columns of a row (one TMEM round trip).
@@ -150,7 +202,7 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NUM_BARS; ++i)
-            mbar_init(&bars[i], counted_by_rows(i) ? 128 : 1);
+            mbar_init(&bars[i], counted_by_rows(i) ? 128 : counted_by_rope_warps(i) ? ROPE_WARPS : 1);
         *abort = 0;
         fence_mbar_init();
     }
@@ -269,8 +321,9 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                 else
                     base_even = base_s;
                 const int sb = n & 1;
-                if (!mbar_wait(&bars[Q_FULL + sb], (n >> 1) & 1, abort, 1u) ||
-                    !mbar_wait(&bars[K_FULL + (n & 1)], (n >> 1) & 1, abort, 1u))
+                // the tiles as loaded, or once rotated (fused RoPE)
+                if (!mbar_wait(&bars[(p.rope ? Q_ROT : Q_FULL) + sb], (n >> 1) & 1, abort, 1u) ||
+                    !mbar_wait(&bars[(p.rope ? K_ROT : K_FULL) + (n & 1)], (n >> 1) & 1, abort, 1u))
                     return false;
                 // S buffer sb held S and P of item n - 2: free once that P.V is done
                 if (n >= 2 && !mbar_wait(&bars[S_FREE + sb], ((n >> 1) - 1) & 1, abort, 1u))
@@ -323,6 +376,95 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             }
             umma_commit(&bars[DRAIN]);
             mbar_wait_drain(&bars[DRAIN], 0);
+        }
+        __syncwarp();
+    } else if (warp >= WARP_ROPE && warp < WARP_ROPE + ROPE_WARPS) {
+        // ------- fused partial RoPE: Q tiles and the new K chunks, rotated in shared memory by
+        // four warps. Warp rw owns query positions rw * 4 .. rw * 4 + 3 of each item (P = 16:
+        // their 32 Q rows, and the new keys at those positions, since the span ends at the item's
+        // last position) and its own rows of the (cos, sin) table, so the warps never wait for
+        // one another; each releases its share of an item with one arrival on each of Q_ROT and
+        // K_ROT. Lane = (position, chunk c of 8 rotary pairs, half of the heads): it holds its 8
+        // pairs' (cos, sin) in registers and applies them to 4 Q rows (heads hb * 4 .. + 3) and,
+        // in head half 0, to the new key at its position; the 8 lanes of a quarter warp touch 8
+        // distinct bank groups. The loop is kept small and rolled: its code shares the SM's
+        // instruction caches with the softmax warps' loops, and more code here slows those.
+        if (p.rope && cnt > 0) {
+            const int rw = warp - WARP_ROPE;
+            const int half = p.rope_half, nch = half / 8;
+            const int c = lane & 3, hb = (lane >> 2) & 1, pos = lane >> 3;
+            // the frequencies in shared memory (a per-lane index into the kernel's parameters
+            // serialises the warp; done once), this lane's own in a register
+            double *wf = reinterpret_cast<double *>(smem + off_rope(p.P)) + rw * kRopeFusedMaxHalf;
+            float2 *cs = reinterpret_cast<float2 *>(smem + off_rope(p.P) + ROPE_WARPS * kRopeFusedMaxHalf * 8) +
+                         rw * 4 * kRopeFusedMaxHalf; // [4][half], this warp's positions
+            wf[lane] = p.inv_freq[lane];
+            const double w_lane = wf[lane];
+            __syncwarp();
+            // consecutive items: the position block and the sequence advance without division
+            int pblk = it0 % p.n_pblk, bg = it0 / p.n_pblk, base = 0;
+            int64_t mb = p.pos0 + (p.pos_base ? p.pos_base[bg / p.Hkv] : 0);
+            for (int n = 0; n < cnt; ++n) {
+                const bool fresh = n == 0 || pblk == 0;
+                base = fresh ? 0 : (base + 1 == R ? 0 : base + 1);
+                const int p0 = pblk * 16;
+                // (cos, sin) of the warp's 4 positions: lane = rotary pair
+                if (lane < half) {
+#pragma unroll 1
+                    for (int l = 0; l < 4; ++l)
+                        cs[l * half + lane] = rope_cos_sin(mb + p0 + rw * 4 + l, w_lane);
+                }
+                __syncwarp();
+                // the item's Q tile and K chunks (one lane polls)
+                bool ok = true;
+                if (lane == 0)
+                    ok = mbar_wait(&bars[Q_FULL + (n & 1)], (n >> 1) & 1, abort, 1u) &&
+                         mbar_wait(&bars[K_FULL + (n & 1)], (n >> 1) & 1, abort, 1u);
+                if (!__shfl_sync(0xffffffffu, (int)ok, 0))
+                    break;
+                // the first item of a run loaded its whole span: rotate it here (rare)
+                if (fresh)
+                    swa_rope_span(smem + off_k(), p0 + 16 - NSC, p.L, mb, wf, nch, rw, lane);
+                if (c < nch) {
+                    float2 csl[8];
+                    const float4 *src = reinterpret_cast<const float4 *>(cs + pos * half + c * 8);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float4 v = src[j];
+                        csl[2 * j] = make_float2(v.x, v.y);
+                        csl[2 * j + 1] = make_float2(v.z, v.w);
+                    }
+                    // tasks 0-3: the Q rows; task 4: the new key (slot base + SC - 1 of the
+                    // ring, row = its position in the chunk), unless the span was just rotated
+                    const int key = p0 + rw * 4 + pos;
+                    const int ntask = (!fresh && hb == 0 && key < p.L) ? 5 : 4;
+                    uint8_t *q0 = smem + (n & 1) * Q_BYTES;
+#pragma unroll 1
+                    for (int t = 0; t < ntask; ++t) {
+                        int row = rw * 32 + pos * 8 + hb * 4 + t;
+                        uint8_t *rowp = q0 + row * ROW;
+                        if (t == 4) {
+                            const int slot = base + SC - 1 >= R ? base + SC - 1 - R : base + SC - 1;
+                            row = rw * 4 + pos;
+                            rowp = smem + off_k() + slot * CHUNK + row * ROW;
+                        }
+                        swa_rotate_chunk(rowp, row, c, nch, csl);
+                    }
+                }
+                // generic stores before the tensor cores' reads; then release this warp's share
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&bars[Q_ROT + (n & 1)]);
+                    mbar_arrive(&bars[K_ROT + (n & 1)]);
+                }
+                if (++pblk == p.n_pblk) {
+                    pblk = 0;
+                    ++bg;
+                    if (n + 1 < cnt) // the next item's sequence (none past the CTA's last item)
+                        mb = p.pos0 + (p.pos_base ? p.pos_base[bg / p.Hkv] : 0);
+                }
+            }
         }
         __syncwarp();
     } else if (warp < 8) {
@@ -397,7 +539,7 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                 break;
             tc_fence_after();
             const bool valid = l < p.L;
-            const float inv_l = 1.f / l_round;
+            const float inv_l = p.out_mul / l_round; // the value scale (fused RoPE) rides on 1 / l
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (int64_t)it.b * p.o_sb +
                                   (int64_t)l * p.o_sl + (int64_t)h * p.o_sh;
 #pragma unroll 1

@@ -371,6 +371,34 @@ typedef struct sinkattn_rope_args {
 
 int sinkattn_rope_qkv(const sinkattn_rope_args *args, void *stream);
 
+/* Sliding-window prefill with the partial RoPE and the value scale fused into its loads: the
+ * result of sinkattn_rope_qkv (same positions, rope_dim, theta and v_scale) over the sequences'
+ * Q, K and V followed by sinkattn_prefill_swa, without that pass's round trip through HBM and
+ * without modifying q, k, v ("MiMo-V2-Flash 模型架构深度拆解" CH10.3: V times v_scale, then RoPE
+ * on the rotary part of Q and K, then attention). Each Q tile and each new K chunk is rotated in
+ * shared memory as it lands, exactly as the pass rotates it (fp64-reduced angle, fp32 rotation,
+ * one bf16 rounding); the value scale multiplies O instead of V (the same value in exact
+ * arithmetic; bf16 rounding of v_scale * V is not reproduced).
+ *   args, window: as for sinkattn_prefill_swa; token l of sequence b sits at position
+ *       pos0 + pos_base[b] + l;
+ *   rope_dim: a multiple of 16 in 16..64 (the rotary dims lie in the first 64 of the 192);
+ *       theta > 0 and finite; v_scale finite.
+ * The fused path is the GQA-packed kernel's (G = 8 query heads per KV head, window <= 128, the
+ * pages' SWA layers); other shapes return UNSUPPORTED (use sinkattn_rope_qkv, then the prefill).
+ * Errors: as sinkattn_prefill_swa; INVALID_ARG for window < 1, a NULL spec, theta <= 0 or
+ * non-finite values; UNSUPPORTED for rope_dim out of range or a shape the fused path does not
+ * take. */
+typedef struct sinkattn_rope_spec {
+    const int32_t *pos_base; /* device int32 [B] or NULL */
+    int64_t pos0;
+    int32_t rope_dim;
+    double theta;
+    float v_scale;
+} sinkattn_rope_spec;
+
+int sinkattn_prefill_swa_rope(const sinkattn_prefill_args *args, int32_t window,
+                              const sinkattn_rope_spec *rope, void *stream);
+
 /* ---------------------------------------------------------------------------------------------
  * Backward of the whole-sequence prefill: the training variant. The gradients of a loss through
  * O = attention(q, k, v, sink) given dO = dLoss/dO. The sink enters the softmax the way

@@ -62,6 +62,7 @@ int main(void) {
   printf("sinkattn_rope_args %zu\n", sizeof(sinkattn_rope_args));
   printf("sinkattn_backward_args %zu\n", sizeof(sinkattn_backward_args));
   printf("sinkattn_paged_kv %zu\n", sizeof(sinkattn_paged_kv));
+  printf("sinkattn_rope_spec %zu\n", sizeof(sinkattn_rope_spec));
   %FIELDS%
   return 0;
 }
@@ -72,7 +73,7 @@ def test_struct_layout_matches_header(tmp_path):
     lines = []
     structs = (("sinkattn_prefill_args", sa.PrefillArgs), ("sinkattn_decode_args", sa.DecodeArgs),
                ("sinkattn_rope_args", sa.RopeArgs), ("sinkattn_backward_args", sa.BackwardArgs),
-               ("sinkattn_paged_kv", sa.PagedKV))
+               ("sinkattn_paged_kv", sa.PagedKV), ("sinkattn_rope_spec", sa.RopeSpec))
     for cname, py in structs:
         for f, _ in py._fields_:
             lines.append(f"F({cname}, {f})")
@@ -87,6 +88,7 @@ def test_struct_layout_matches_header(tmp_path):
     assert int(got["sinkattn_rope_args"]) == ctypes.sizeof(sa.RopeArgs)
     assert int(got["sinkattn_backward_args"]) == ctypes.sizeof(sa.BackwardArgs)
     assert int(got["sinkattn_paged_kv"]) == ctypes.sizeof(sa.PagedKV)
+    assert int(got["sinkattn_rope_spec"]) == ctypes.sizeof(sa.RopeSpec)
     for cname, py in structs:
         for f, _ in py._fields_:
             assert int(got[f"{cname}.{f}"]) == getattr(py, f).offset, (cname, f)
@@ -154,6 +156,30 @@ def test_host_prefill_sizes_and_checks(L):
     assert host(ctypes.byref(a), 128, 128, None, size, None) == 1        # no workspace
     assert host(ctypes.byref(a), 128, 128, ws, size - 1, None) == 4      # workspace too small
     assert host(ctypes.byref(_prefill_args(L=0)), 128, 128, None, 0, None) == 0
+
+
+def test_fused_rope_prefill_checks(L):
+    """The fused RoPE SWA prefill checks its spec before any device work."""
+    f = L.sinkattn_prefill_swa_rope
+    f.argtypes = [ctypes.POINTER(sa.PrefillArgs), ctypes.c_int32, ctypes.POINTER(sa.RopeSpec),
+                  ctypes.c_void_p]
+
+    def spec(**kw):
+        r = sa.RopeSpec()
+        r.pos_base, r.pos0, r.rope_dim, r.theta, r.v_scale = None, 0, 64, 1e4, 0.707
+        for k, v in kw.items():
+            setattr(r, k, v)
+        return r
+    a = _prefill_args()
+    assert f(ctypes.byref(a), 128, None, None) == 1                          # no spec
+    assert f(ctypes.byref(a), 0, ctypes.byref(spec()), None) == 1            # window < 1
+    assert f(ctypes.byref(a), 128, ctypes.byref(spec(theta=0.0)), None) == 1
+    assert f(ctypes.byref(a), 128, ctypes.byref(spec(theta=float("inf"))), None) == 1
+    assert f(ctypes.byref(a), 128, ctypes.byref(spec(v_scale=float("nan"))), None) == 1
+    for rd in (0, 8, 24, 80, 128):                                           # not 16..64 step 16
+        assert f(ctypes.byref(a), 128, ctypes.byref(spec(rope_dim=rd)), None) == 2
+    assert f(ctypes.byref(_prefill_args(dq=128)), 128, ctypes.byref(spec()), None) == 2
+    assert f(ctypes.byref(_prefill_args(L=0)), 128, ctypes.byref(spec()), None) == 0
 
 
 def test_prefill_empty_is_ok_and_window_checked(L):
