@@ -191,7 +191,9 @@ class DecodeRunner:
                    (w.kind == W.KV_RING and w.ring_cap % 64 == 0))
             self.kernel = "decode_fp8_tma_kernel" if tma else "decode_fp8_kernel"
         elif w.kind == W.KV_RING:
-            if rows <= 16 and w.ring_cap % 32 == 0:
+            if w.ring_cap == 128 and w.Hq // w.Hkv == 8 and w.T <= 4:
+                self.kernel = "decode_ring_umma_kernel"
+            elif rows <= 16 and w.ring_cap % 32 == 0:
                 self.kernel = "decode_ring_kernel"
             else:
                 self.kernel = "decode_split_kernel"
@@ -298,12 +300,33 @@ class BackwardRunner:
                 delattr(self, k)
 
 
+def graph_of(fn):
+    """fn's launches captured once into a CUDA graph (after two plain calls that do the one-time
+    setup: function attributes, device queries). A decode step of many short layer calls issued
+    one by one from Python is bound by the host's call overhead (~25 us a call against ~15 us of
+    GPU time for an SWA layer); a serving loop replays the step as one graph, as here."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        fn()
+        fn()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 class HybridRunner:
-    """One speculative-verify step of the hybrid stack: every layer's decode call in order."""
+    """One speculative-verify step of the hybrid stack: every layer's decode call in order, the
+    49 calls replayed as one CUDA graph."""
 
     def __init__(self, dev):
         self.layers = [DecodeRunner(W.hybrid_layer_workload(i), dev)
                        for i in range(len(W.HYBRID_LAYERS))]
+        self.graph = graph_of(self.eager_step)
         self.flops = sum(r.flops for r in self.layers)
         self.bytes = sum(r.bytes for r in self.layers)
         self.ga_bytes = sum(r.bytes for r in self.layers if r.w.kind != W.KV_RING)
@@ -312,15 +335,25 @@ class HybridRunner:
         self.config = dict(B=W.HYBRID_B, T=W.HYBRID_T, layers=len(W.HYBRID_LAYERS),
                            ga_layers=W.HYBRID_LAYERS.count("GA"),
                            swa_layers=W.HYBRID_LAYERS.count("SWA"),
-                           ctx_range=[W.HYBRID_CTX_LO, W.HYBRID_CTX_HI])
+                           ctx_range=[W.HYBRID_CTX_LO, W.HYBRID_CTX_HI], cuda_graph=True)
 
-    def step(self):
+    def eager_step(self):
         for r in self.layers:
             r.step()
 
+    def step(self):
+        self.graph.replay()
+
     def kind_runner(self, ring):
-        """The GA (ring=False) or SWA (ring=True) layers alone, for a per-kind breakdown."""
+        """The GA (ring=False) or SWA (ring=True) layers alone, for a per-kind breakdown (also
+        one CUDA graph per step)."""
         sel = [r for r in self.layers if (r.w.kind == W.KV_RING) == ring]
+
+        def eager():
+            for r in sel:
+                r.step()
+        graph = graph_of(eager)
+        self.sub_graphs = getattr(self, "sub_graphs", []) + [graph]
 
         class Sub:
             flops = sum(r.flops for r in sel)
@@ -329,11 +362,12 @@ class HybridRunner:
 
             @staticmethod
             def step():
-                for r in sel:
-                    r.step()
+                graph.replay()
         return Sub
 
     def release(self):
+        self.graph = None
+        self.sub_graphs = []
         for r in self.layers:
             r.release()
         self.layers = []
@@ -474,6 +508,7 @@ def measured_traffic(kernel):
                                     "decode_tma_kernels.cuh", "decode_umma_kernels.cuh"],
              "decode_ring_kernel": ["common.cuh", "decode_kernels.cuh",
                                     "decode_ring_kernels.cuh"],
+             "decode_ring_umma_kernel": ["common.cuh", "decode_ring_umma_kernels.cuh"],
              "rope_qkv_kernel": ["common.cuh", "rope_kernels.cuh"],
              "decode_fp8_kernel": ["common.cuh", "decode_kernels.cuh",
                                    "decode_fp8_kernels.cuh"],

@@ -16,7 +16,7 @@ LIB = os.path.join(PKG, "libsinkattn.so")
 SOURCES = ["sinkattn.cu"]
 DEPS = SOURCES + ["common.cuh", "internal.h", "prefill_kernels.cuh", "swa_kernels.cuh",
                   "decode_kernels.cuh", "decode_tma_kernels.cuh", "decode_umma_kernels.cuh",
-                  "decode_ring_kernels.cuh", "rope_kernels.cuh", "decode_fp8_kernels.cuh",
+                  "decode_ring_kernels.cuh", "decode_ring_umma_kernels.cuh", "rope_kernels.cuh", "decode_fp8_kernels.cuh",
                   "decode_fp8_tma_kernels.cuh", "backward_kernels.cuh"]
 
 NVCC_FLAGS = [

@@ -114,6 +114,12 @@ cudaError_t launch_decode_umma(const CUtensorMap &q, const CUtensorMap &kc, cons
 cudaError_t launch_decode_ring(const CUtensorMap &kc, const CUtensorMap &vc, const CUtensorMap &kn,
                                const CUtensorMap &vn, const DecodeParams &p, int sms,
                                cudaStream_t stream);
+// Ring decode / verify on the tensor cores: 128-slot rings, G = 8, T <= 4; q map {192, Hq, T, B}
+// box {64, 8, T, 1}, cache maps {d, Hkv, 128, B} box {64, 1, 128, 1}, new-token maps
+// {d, Hkv, T, B} box {64, 1, 16, 1}. One CTA per SM (at most one per unit).
+cudaError_t launch_decode_ring_umma(const CUtensorMap &q, const CUtensorMap &kc, const CUtensorMap &vc,
+                                    const CUtensorMap &kn, const CUtensorMap &vn, const DecodeParams &p,
+                                    int sms, cudaStream_t stream);
 cudaError_t launch_decode_merge(const DecodeParams &p, cudaStream_t stream);
 int decode_stages(const DecodeParams &p);
 

@@ -15,6 +15,7 @@
 #include "decode_tma_kernels.cuh"
 #include "decode_umma_kernels.cuh"
 #include "decode_ring_kernels.cuh"
+#include "decode_ring_umma_kernels.cuh"
 #include "backward_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
@@ -777,9 +778,9 @@ cudaError_t noalloc_workspace_ptr(void **out)
 
 // The split-KV TMA-fed decode kernels take whole 64-key tiles: contiguous caches, and paged
 // caches whose pages hold a multiple of 64 tokens (without a window, so tiles stay page-aligned).
-// Rings of up to 16 query rows per item go to the ring kernel; other rings (a 4-token verify's
-// 32 rows measured faster on the cp.async kernel, whose CTA serves all rows) and other page
-// sizes use the cp.async kernel.
+// Rings of 128 slots on 8-head groups with up to 4 query tokens (the model's SWA layers, decode
+// and verify) go to the tcgen05 ring kernel; other rings of up to 16 rows per item to the
+// mma.sync ring kernel; the remaining rings and other page sizes use the cp.async kernel.
 bool decode_tma_ok(const sinkattn_decode_args *a, const DecodeParams &)
 {
     if (a->kind == SINKATTN_KV_CONTIG)
@@ -812,9 +813,26 @@ int run_decode(const sinkattn_decode_args *a, const DecodeParams &p, void *strea
             e = launch_decode_fp8(p, (cudaStream_t)stream);
         return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
     }
+    if (a->kind == SINKATTN_KV_RING && a->ring_cap == rv::CAP && p.G == rv::G && a->T <= rv::TMAX &&
+        p.splits == 1) {
+        // a unit (sequence, KV head) per MMA pass: S = Q K^T over the 128 slots and the new
+        // tokens, P V from TMEM
+        CUtensorMap q, kc, vc, kn, vn;
+        DeviceInfo di;
+        int st = device_info(&di);
+        if (st != SINKATTN_OK)
+            return st;
+        if (!make_map(&q, a->q, kDQ, a->Hq, a->T, a->B, a->q_sh, a->q_st, a->q_sb, rv::G, a->T) &&
+            !make_map(&kc, a->k_cache, kDQ, a->Hkv, rv::CAP, a->B, a->kc_sh, a->kc_ss, a->kc_sb, 1, rv::CAP) &&
+            !make_map(&vc, a->v_cache, kDV, a->Hkv, rv::CAP, a->B, a->vc_sh, a->vc_ss, a->vc_sb, 1, rv::CAP) &&
+            !make_map(&kn, a->k_new, kDQ, a->Hkv, a->T, a->B, a->kn_sh, a->kn_st, a->kn_sb, 1, 16) &&
+            !make_map(&vn, a->v_new, kDV, a->Hkv, a->T, a->B, a->vn_sh, a->vn_st, a->vn_sb, 1, 16)) {
+            e = launch_decode_ring_umma(q, kc, vc, kn, vn, p, di.sms, (cudaStream_t)stream);
+            return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
+        }
+    }
     if (a->kind == SINKATTN_KV_RING && p.R <= 16 && a->ring_cap % 32 == 0 && p.splits == 1) {
-        // a ring item per warp, streamed in 32-key chunks (units of more than 16 rows, as in a
-        // 4-token verify, measured faster on the cp.async kernel, whose CTA serves all rows)
+        // a ring item per warp, streamed in 32-key chunks
         CUtensorMap kc, vc, kn, vn;
         DeviceInfo di;
         int st = device_info(&di);

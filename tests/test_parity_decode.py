@@ -95,6 +95,22 @@ def test_ring_decode_other_capacities(cap, window, T):
     check(sa.KV_RING, d, window, f"ring cap {cap} W{window} T{T}")
 
 
+@pytest.mark.parametrize("window", [0, 1, 3, 64, 127, 200])
+@pytest.mark.parametrize("T", [3, 4])
+def test_ring_verify_windows(window, T):
+    """128-slot rings with a 3- or 4-token verify on 8-head groups (the tensor-core ring kernel):
+    windows shorter than the ring (down to one key), equal to it, longer, and none; empty,
+    partial and full rings with wrapped heads; a sink of -inf on some heads."""
+    g = torch.Generator().manual_seed(31 * window + T)
+    B, Hq, Hkv, cap = 7, 16, 2, 128
+    d = dict(q=rnd((B, T, Hq, 192), g), k_new=rnd((B, T, Hkv, 192), g),
+             v_new=rnd((B, T, Hkv, 128), g), k_cache=rnd((B, cap, Hkv, 192), g),
+             v_cache=rnd((B, cap, Hkv, 128), g), sink=make_sink(Hq, g, "mixed"),
+             ring_head=torch.tensor([0, 17, 127, 64, 125, 90, 1], dtype=torch.int32),
+             ring_len=torch.tensor([128, 0, 1, 127, 128, 40, 2], dtype=torch.int32))
+    check(sa.KV_RING, d, window, f"ring verify W{window} T{T}")
+
+
 @pytest.mark.parametrize("T", [1, 4])
 @pytest.mark.parametrize("ctx", [[0, 1, 63, 64], [65, 127, 128, 129], [1000, 5000, 3, 4093]])
 def test_contig_decode(T, ctx):
