@@ -122,20 +122,6 @@ SA_DEV void rv_mask48(uint32_t (&r)[48], uint64_t hidden)
             r[u] = __float_as_uint(-INFINITY);
 }
 
-// 48 columns of this thread's TMEM lane; the empty asm after the wait names the registers, so
-// no use of them is scheduled before the wait.
-SA_DEV void rv_ld48(uint32_t taddr, uint32_t (&r)[48])
-{
-    tmem_ld16(taddr + 0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-    tmem_ld16(taddr + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-    tmem_ld16(taddr + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 48; i += 8)
-        asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]),
-                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
-}
-
 __global__ void __launch_bounds__(rv::THREADS, 1)
     decode_ring_umma_kernel(const __grid_constant__ CUtensorMap tmQ,
                             const __grid_constant__ CUtensorMap tmKc,
@@ -172,6 +158,11 @@ __global__ void __launch_bounds__(rv::THREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    // Programmatic dependent launch: the next kernel in the stream may start its own set-up now;
+    // this one reads no global memory before the kernels ahead of it have completed and their
+    // writes are visible (without a programmatic launch both are no-ops).
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     if (warp == WARP_LOAD || warp == WARP_VLOAD) {
         // Q and K (warp 8) or V (warp 10) of unit n into stage n & 1, once the unit n - 2 that
@@ -289,42 +280,47 @@ __global__ void __launch_bounds__(rv::THREADS, 1)
             if (!warp_wait(&bars[S_FULL + wg], (n >> 1) & 1, abort))
                 break;
             tc_fence_after();
-            // row max, then P, in groups of 48 columns per TMEM round trip
+            // the row's 144 scores in one TMEM round trip (a CTA of five warps leaves each
+            // thread room for them in registers), masked; the row max; then P
             const uint32_t saddr = tmem + lane_addr + wg * NK;
-            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-            for (int c0 = 0; c0 < NK; c0 += 48) {
-                uint32_t r[48];
-                rv_ld48(saddr + c0, r);
-                rv_mask48(r, rv_hidden48(c0, hid_e, hid_k, i_lo, i_hi));
+            uint32_t sv[NK];
+            tmem_ld32(saddr + 0, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+            tmem_ld32(saddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+            tmem_ld32(saddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&sv[64]));
+            tmem_ld32(saddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&sv[96]));
+            tmem_ld16(saddr + 128, *reinterpret_cast<uint32_t(*)[16]>(&sv[128]));
+            tmem_ld_wait();
 #pragma unroll
-                for (int u = 0; u < 48; ++u)
-                    mx4[u & 3] = fmaxf(mx4[u & 3], __uint_as_float(r[u]));
-            }
+            for (int i = 0; i < NK; i += 8)
+                asm volatile("" : "+r"(sv[i]), "+r"(sv[i + 1]), "+r"(sv[i + 2]), "+r"(sv[i + 3]),
+                             "+r"(sv[i + 4]), "+r"(sv[i + 5]), "+r"(sv[i + 6]), "+r"(sv[i + 7])::"memory");
+#pragma unroll
+            for (int c0 = 0; c0 < NK; c0 += 48)
+                rv_mask48(*reinterpret_cast<uint32_t(*)[48]>(&sv[c0]),
+                          rv_hidden48(c0, hid_e, hid_k, i_lo, i_hi));
+            float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int u = 0; u < NK; ++u)
+                mx4[u & 3] = fmaxf(mx4[u & 3], __uint_as_float(sv[u]));
             const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             // m = max(sink, max_j a_j) in log2 units (the max includes the sink)
             const float m = fmaxf(sink_l2, mx * c_l2);
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
+            // P = 2^(s c - m) as bf16 pairs over S's first 72 columns; sums of fp32 and of
+            // rounded P
             float pe[4] = {0.f, 0.f, 0.f, 0.f}, pr[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-            for (int c0 = 0; c0 < NK; c0 += 48) {
-                uint32_t r[48];
-                rv_ld48(saddr + c0, r);
-                rv_mask48(r, rv_hidden48(c0, hid_e, hid_k, i_lo, i_hi));
 #pragma unroll
-                for (int k = 0; k < 3; ++k) {
-                    uint32_t pk[8];
+            for (int k = 0; k < NK / 16; ++k) {
+                uint32_t pk[8];
 #pragma unroll
-                    for (int u = 0; u < 16; u += 2) {
-                        const float e0 = fast_exp2(fmaf(__uint_as_float(r[k * 16 + u]), c_l2, neg_m));
-                        const float e1 = fast_exp2(fmaf(__uint_as_float(r[k * 16 + u + 1]), c_l2, neg_m));
-                        pe[(u >> 1) & 3] += e0 + e1;
-                        pk[u >> 1] = pack_bf16x2(e0, e1);
-                        pr[(u >> 1) & 3] += sum_bf16x2(pk[u >> 1]);
-                    }
-                    tmem_st8(saddr + c0 / 2 + k * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5],
-                             pk[6], pk[7]);
+                for (int u = 0; u < 16; u += 2) {
+                    const float e0 = fast_exp2(fmaf(__uint_as_float(sv[k * 16 + u]), c_l2, neg_m));
+                    const float e1 = fast_exp2(fmaf(__uint_as_float(sv[k * 16 + u + 1]), c_l2, neg_m));
+                    pe[(u >> 1) & 3] += e0 + e1;
+                    pk[u >> 1] = pack_bf16x2(e0, e1);
+                    pr[(u >> 1) & 3] += sum_bf16x2(pk[u >> 1]);
                 }
+                tmem_st8(saddr + k * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
             }
             // V rows of slots that hold no key: zeros (lane = slot mod 32), once V has landed,
             // seen by P V through the async proxy
@@ -367,18 +363,15 @@ __global__ void __launch_bounds__(rv::THREADS, 1)
             tc_fence_after();
             const float inv_l = 1.f / l_round;
             uint16_t *orow = p.o + (int64_t)x.b * p.o_sb + (int64_t)(row_ok ? t : 0) * p.o_st + (int64_t)h * p.o_sh;
-#pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                tmem_ld32_sync(tmem + lane_addr + TMEM_O + c * 32, o);
-                if (c == 3) {
-                    // O is read: the next P V may overwrite it
-                    tc_fence_before();
-                    mbar_arrive(&bars[O_FREE]);
-                }
+            {
+                uint32_t o[128];
+                tmem_ld128(tmem + lane_addr + TMEM_O, o);
+                // O is read: the next P V may overwrite it
+                tc_fence_before();
+                mbar_arrive(&bars[O_FREE]);
                 if (row_ok) {
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
+                    for (int v = 0; v < 16; ++v) {
                         uint4 pk;
                         pk.x = pack_bf16x2(__uint_as_float(o[v * 8 + 0]) * inv_l,
                                            __uint_as_float(o[v * 8 + 1]) * inv_l);
@@ -388,7 +381,7 @@ __global__ void __launch_bounds__(rv::THREADS, 1)
                                            __uint_as_float(o[v * 8 + 5]) * inv_l);
                         pk.w = pack_bf16x2(__uint_as_float(o[v * 8 + 6]) * inv_l,
                                            __uint_as_float(o[v * 8 + 7]) * inv_l);
-                        *reinterpret_cast<uint4 *>(orow + c * 32 + v * 8) = pk;
+                        *reinterpret_cast<uint4 *>(orow + v * 8) = pk;
                     }
                 }
             }
@@ -417,9 +410,19 @@ cudaError_t launch_decode_ring_umma(const CUtensorMap &q, const CUtensorMap &kc,
     if (e != cudaSuccess)
         return e;
     const int units = p.B * p.Hkv;
-    decode_ring_umma_kernel<<<units < sms ? units : sms, rv::THREADS, rv::SMEM_BYTES, stream>>>(
-        q, kc, vc, kn, vn, p);
-    return cudaGetLastError();
+    // launched as a programmatic dependent: its CTAs are placed and set up (barriers, TMEM)
+    // while the kernel before it finishes, and wait for it before reading memory
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(units < sms ? units : sms);
+    cfg.blockDim = dim3(rv::THREADS);
+    cfg.dynamicSmemBytes = rv::SMEM_BYTES;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_ring_umma_kernel, q, kc, vc, kn, vn, p);
 }
 
 } // namespace sinkattn
