@@ -306,9 +306,9 @@ __global__ void __launch_bounds__(rv::THREADS, 1)
             // m = max(sink, max_j a_j) in log2 units (the max includes the sink)
             const float m = fmaxf(sink_l2, mx * c_l2);
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            // P = 2^(s c - m) as bf16 pairs over S's first 72 columns; sums of fp32 and of
-            // rounded P
-            float pe[4] = {0.f, 0.f, 0.f, 0.f}, pr[4] = {0.f, 0.f, 0.f, 0.f};
+            // P = 2^(s c - m) as bf16 pairs over S's first 72 columns; the row sum of the fp32 P
+            // normalises O (the P V MMA multiplies P rounded to bf16) and gives LSE
+            float pe[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int k = 0; k < NK / 16; ++k) {
                 uint32_t pk[8];
@@ -318,7 +318,6 @@ __global__ void __launch_bounds__(rv::THREADS, 1)
                     const float e1 = fast_exp2(fmaf(__uint_as_float(sv[k * 16 + u + 1]), c_l2, neg_m));
                     pe[(u >> 1) & 3] += e0 + e1;
                     pk[u >> 1] = pack_bf16x2(e0, e1);
-                    pr[(u >> 1) & 3] += sum_bf16x2(pk[u >> 1]);
                 }
                 tmem_st8(saddr + k * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
             }
@@ -355,13 +354,12 @@ __global__ void __launch_bounds__(rv::THREADS, 1)
             // the sink seeds both sums: exp(sink - m)
             const float s0 = (sink_l2 == -INFINITY) ? 0.f : fast_exp2(sink_l2 - m);
             const float l_exact = s0 + ((pe[0] + pe[1]) + (pe[2] + pe[3]));
-            const float l_round = s0 + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
 
-            // epilogue: O = (P V) / l_round, LSE = m + log2(l_exact)
+            // epilogue: O = (P V) / l_exact, LSE = m + log2(l_exact)
             if (!warp_wait(&bars[PV_DONE + wg], (n >> 1) & 1, abort))
                 break;
             tc_fence_after();
-            const float inv_l = 1.f / l_round;
+            const float inv_l = 1.f / l_exact;
             uint16_t *orow = p.o + (int64_t)x.b * p.o_sb + (int64_t)(row_ok ? t : 0) * p.o_st + (int64_t)h * p.o_sh;
             {
                 uint32_t o[128];

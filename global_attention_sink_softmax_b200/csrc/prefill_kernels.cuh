@@ -28,8 +28,10 @@
 // S_{j+2} while the softmax warps work on S_j, and S_{j+1} is ready when they finish; the
 // softmax waits for PV_{j-1} only when it has to rescale O.
 //
-// Two row sums: O is normalised by the sum of the bf16-rounded P values (the ones the P.V MMA
-// multiplies), so numerator and denominator use identical weights; LSE uses the fp32 sum.
+// One row sum, of the fp32 P: it normalises O (whose P.V MMA multiplies P rounded to bf16,
+// a relative error of at most 2^-9 per weight) and gives LSE. A second sum of the rounded P, for
+// O alone, cost three instructions per score pair in the softmax, which sets this kernel's pace
+// (5 % of the GA prefill's time).
 //
 // Lazy rescaling: the running max used for the exponent is only raised when a tile's row max
 // exceeds it by more than 8 (log2 units); P values stay <= 2^8 and the final O / l and LSE are
@@ -275,12 +277,10 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
         const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
         const float sink_l2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
         const float c_l2 = p.scale_log2; // > 0, so max(s) * c = max(s * c)
-        // m_run: reference max (log2 units); l_exact: sum of fp32 P (gives LSE); l_round: sum
-        // of the bf16-rounded P the P.V MMA consumes (normalises O). Both start with the sink:
-        // m_0 = sink, l_0 = exp(sink - m_0) = 1.
+        // m_run: reference max (log2 units); l_exact: sum of fp32 P (normalises O, gives LSE),
+        // seeded with the sink: m_0 = sink, l_0 = exp(sink - m_0) = 1.
         float m_run = sink_l2;
         float l_exact = (sink_l2 > -INFINITY) ? 1.f : 0.f;
-        float l_round = l_exact;
         bool ok = true;
         for (int idx = 0; idx < n_tiles; ++idx) {
             const int sb = idx % S_BUFS;
@@ -328,7 +328,6 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
             if (rescale) {
                 alpha = fast_exp2(m_run - mx); // 0 when m_run is -inf
                 l_exact *= alpha;
-                l_round *= alpha;
                 m_run = mx;
             }
             // O is only touched when one of this warp's rows raises its max: then wait for the
@@ -352,7 +351,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                 tmem_st_wait();
             }
             const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-            float pe[4] = {0.f, 0.f, 0.f, 0.f}, pr[4] = {0.f, 0.f, 0.f, 0.f};
+            float pe[4] = {0.f, 0.f, 0.f, 0.f};
             // P (bf16 pairs: keys 2c, 2c + 1 in column c) over this row's S in TMEM: chunk c0's
             // 16 columns of P land on scores already read (columns < c0 + 32)
 #pragma unroll 1
@@ -372,14 +371,12 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                     const float e1 = fast_exp2(fmaf(__uint_as_float(r[2 * u + 1]), c_l2, neg_m));
                     pk[u] = pack_bf16x2(e0, e1);
                     pe[u & 3] += e0 + e1;
-                    pr[u & 3] += sum_bf16x2(pk[u]);
                 }
                 tmem_st8(saddr + c0 / 2, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5], pk[6], pk[7]);
                 tmem_st8(saddr + c0 / 2 + 8, pk[8], pk[9], pk[10], pk[11], pk[12], pk[13], pk[14],
                          pk[15]);
             }
             l_exact += (pe[0] + pe[1]) + (pe[2] + pe[3]);
-            l_round += (pr[0] + pr[1]) + (pr[2] + pr[3]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&bars[B_PFULL + sb]);
@@ -389,7 +386,7 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                            ((n_tiles - 1) / S_BUFS) & 1, abort);
         if (ok) {
             tc_fence_after();
-            const float inv_l = 1.f / l_round;
+            const float inv_l = 1.f / l_exact;
             const bool valid = rp < p.L;
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (int64_t)b * p.o_sb +
                                   (int64_t)rp * p.o_sl + (int64_t)h * p.o_sh;

@@ -503,9 +503,9 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             // m = max(sink, max_j a_j) in log2 units (the max includes the sink)
             const float m = fmaxf(sink_l2, mx * c_l2);
             const float neg_m = (m == -INFINITY) ? 0.f : -m;
-            // P = 2^(s c - m) as bf16 pairs over the consumed scores; sums of fp32 and of
-            // rounded P
-            float pe[4] = {0.f, 0.f, 0.f, 0.f}, pr[4] = {0.f, 0.f, 0.f, 0.f};
+            // P = 2^(s c - m) as bf16 pairs over the consumed scores; the row sum of the fp32 P
+            // normalises O and gives LSE
+            float pe[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
             for (int c0 = 0; c0 < NSC; c0 += 48) {
                 uint32_t r[48];
@@ -520,7 +520,6 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                         const float e1 = fast_exp2(fmaf(__uint_as_float(r[k * 16 + u + 1]), c_l2, neg_m));
                         pe[(u >> 1) & 3] += e0 + e1;
                         pk[u >> 1] = pack_bf16x2(e0, e1);
-                        pr[(u >> 1) & 3] += sum_bf16x2(pk[u >> 1]);
                     }
                     tmem_st8(saddr + c0 / 2 + k * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5],
                              pk[6], pk[7]);
@@ -532,14 +531,13 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             // the sink seeds both sums: exp(sink - m)
             const float s0 = (sink_l2 == -INFINITY) ? 0.f : fast_exp2(sink_l2 - m);
             const float l_exact = s0 + ((pe[0] + pe[1]) + (pe[2] + pe[3]));
-            const float l_round = s0 + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
 
-            // epilogue: O = (P V) / l_round, LSE = m + log2(l_exact)
+            // epilogue: O = (P V) / l_exact, LSE = m + log2(l_exact)
             if (!warp_wait(&bars[PV_DONE + wg], (n >> 1) & 1, abort))
                 break;
             tc_fence_after();
             const bool valid = l < p.L;
-            const float inv_l = p.out_mul / l_round; // the value scale (fused RoPE) rides on 1 / l
+            const float inv_l = p.out_mul / l_exact; // the value scale (fused RoPE) rides on 1 / l
             __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.o) + (int64_t)it.b * p.o_sb +
                                   (int64_t)l * p.o_sl + (int64_t)h * p.o_sh;
 #pragma unroll 1
