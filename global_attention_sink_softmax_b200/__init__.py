@@ -49,7 +49,7 @@ EXPORTED_SYMBOLS = [
     "sinkattn_prefill_host_workspace_size", "sinkattn_prefill_host", "sinkattn_prefill_swa_rope",
 ]
 # Positions per chunk of the host-resident prefill (its copies in and out overlap chunk by chunk).
-HOST_CHUNK = 4096
+HOST_CHUNK = 1024
 # Size of the library's own split-KV workspace used by sinkattn_decode_noalloc.
 NOALLOC_WORKSPACE_BYTES = 16 << 20
 
