@@ -81,3 +81,29 @@ def test_decode_wait_gives_up_then_next_call_is_correct(limit_zero):
                               ctx_len=ctx)
     assert (o.double().cpu() - ro).abs().max().item() <= O_TOL
     assert (lse.double().cpu() - rl).abs().max().item() <= LSE_TOL
+
+
+def test_ring_decode_wait_gives_up_then_next_call_is_correct(limit_zero):
+    m = limit_zero
+    g = torch.Generator().manual_seed(7)
+    # a 4-token verify on 128-slot rings, 8 heads per KV head: the tcgen05 ring kernel, whose
+    # first waits span the Q / K / V loads and an S step
+    B, T, Hq, Hkv, cap = 3, 4, 16, 2, 128
+    q, kn, vn = rnd((B, T, Hq, 192), g), rnd((B, T, Hkv, 192), g), rnd((B, T, Hkv, 128), g)
+    kc, vc = rnd((B, cap, Hkv, 192), g), rnd((B, cap, Hkv, 128), g)
+    sink = torch.rand(Hq, generator=g) * 6
+    head = torch.tensor([0, 77, 127], dtype=torch.int32)
+    ln = torch.tensor([128, 128, 50], dtype=torch.int32)
+    args = [x.cuda() for x in (q, kn, vn, kc, vc, sink)]
+    kw = dict(window=128, ring_head=head.cuda(), ring_len=ln.cuda())
+    m.sinkattn_decode(m.KV_RING, *args, **kw)
+    torch.cuda.synchronize()
+    assert m.sinkattn_take_device_error() & 2
+    m.sinkattn_set_wait_limit_ns(10 ** 9)
+    o, lse = m.sinkattn_decode(m.KV_RING, *args, **kw)
+    torch.cuda.synchronize()
+    assert m.sinkattn_take_device_error() == 0
+    ro, rl, _ = oracle.decode(oracle.KV_RING, q, kn, vn, kc, vc, sink, 1 / math.sqrt(192), 128,
+                              ring_head=head, ring_len=ln)
+    assert (o.double().cpu() - ro).abs().max().item() <= O_TOL
+    assert (lse.double().cpu() - rl).abs().max().item() <= LSE_TOL
