@@ -23,7 +23,9 @@
 // - warp 0 takes the even units (lanes 0 .. 31) and warp 1 the odd ones (lanes 32 .. 63), on
 //   two SMSPs, so the two units in flight do not share an exponential unit (S double-buffered
 //   in TMEM, O handed over); warp 2 loads Q and K, warp 4 V, one thread of warp 3 issues the
-//   MMAs: S of the next unit goes in before P V of this one.
+//   MMAs: S of the next unit goes in before P V of this one;
+// - launched as a programmatic dependent: the next launch's CTAs are set up while this one
+//   drains, and none reads global memory before the kernels ahead of it have completed.
 //
 // Masks: slot s holds the token of age index cl = (s - head) mod 128 (0 the oldest); it is a
 // key iff first_c <= cl < n_cache, and row t sees it iff also cl >= n_cache + t - W + 1: the
