@@ -112,6 +112,36 @@ def test_ring_verify_windows(window, T):
 
 
 @pytest.mark.parametrize("T", [1, 4])
+def test_ring_decode_strided_views(T):
+    """The tensor-core ring kernel on views: Q, K_new and V_new sliced out of one fused
+    projection buffer per token (strided heads and tokens), the ring caches slices of wider
+    per-slot buffers; results must equal the oracle on the same values."""
+    g = torch.Generator().manual_seed(41 + T)
+    B, Hq, Hkv, cap = 3, 16, 2, 128
+    width = Hq * 192 + Hkv * 192 + Hkv * 128 + 64
+    qkv = torch.randn(B, T, width, generator=g).to(torch.bfloat16).cuda()
+    o1, o2 = Hq * 192, (Hq + Hkv) * 192
+    q = qkv[:, :, :o1].view(B, T, Hq, 192)
+    kn = qkv[:, :, o1:o2].view(B, T, Hkv, 192)
+    vn = qkv[:, :, o2:o2 + Hkv * 128].view(B, T, Hkv, 128)
+    kwide = torch.randn(B, cap, Hkv, 256, generator=g).to(torch.bfloat16).cuda()
+    vwide = torch.randn(B, cap, Hkv, 192, generator=g).to(torch.bfloat16).cuda()
+    kc, vc = kwide[..., :192], vwide[..., :128]
+    assert not q.is_contiguous() and not kc.is_contiguous()
+    sink = make_sink(Hq, g, "mixed")
+    head = torch.tensor([3, 127, 64], dtype=torch.int32)
+    ln = torch.tensor([128, 100, 128], dtype=torch.int32)
+    o, lse = sa.sinkattn_decode(sa.KV_RING, q, kn, vn, kc, vc, sink.cuda(), window=128,
+                                ring_head=head.cuda(), ring_len=ln.cuda())
+    torch.cuda.synchronize()
+    d = dict(q=q.cpu(), k_new=kn.cpu(), v_new=vn.cpu(), k_cache=kc.cpu(), v_cache=vc.cpu(),
+             sink=sink, ring_head=head, ring_len=ln)
+    ro, rl, _ = oracle_decode(sa.KV_RING, d, 128)
+    assert_close(o, ro, lse, rl, f"ring views T{T}")
+    assert sa.sinkattn_take_device_error() == 0
+
+
+@pytest.mark.parametrize("T", [1, 4])
 @pytest.mark.parametrize("ctx", [[0, 1, 63, 64], [65, 127, 128, 129], [1000, 5000, 3, 4093]])
 def test_contig_decode(T, ctx):
     g = torch.Generator().manual_seed(sum(ctx) + T)
