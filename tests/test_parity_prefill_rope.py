@@ -84,6 +84,29 @@ def test_fused_rope_prefill(B, L, Hq, Hkv, window, pos0, base_hi):
     assert sa.sinkattn_take_device_error() == 0
 
 
+@pytest.mark.parametrize("rope_dim", [16, 32, 48])
+def test_fused_rope_prefill_rope_widths(rope_dim):
+    """Narrower rotary widths (one to three of the four 8-pair chunks a rotator lane holds) and
+    the GA theta: LSE bit for bit against the pass then the prefill, O against the oracle."""
+    B, L, Hq, Hkv, window, pos0 = 2, 333, 16, 2, 128, 1000
+    q, k, v, s = rand_qkv(B, L, Hq, Hkv, seed=7 * rope_dim)
+    qd, kd, vd, sd = q.cuda(), k.cuda(), v.cuda(), s.cuda()
+    theta = sa.ROPE_THETA_GA
+    o, lse = sa.sinkattn_prefill_swa_rope(qd, kd, vd, sd, window, theta=theta, rope_dim=rope_dim,
+                                          pos0=pos0)
+    q2, k2, v2 = qd.clone(), kd.clone(), vd.clone()
+    sa.sinkattn_rope_qkv(q2, k2, v2, theta=theta, rope_dim=rope_dim, pos0=pos0)
+    o2, lse2 = sa.sinkattn_prefill_swa(q2, k2, v2, sd, window)
+    torch.cuda.synchronize()
+    assert torch.equal(lse, lse2)
+    pos = positions(B, L, pos0, None)
+    rq = oracle.rope(q, pos, theta, rope_dim).to(torch.bfloat16)
+    rk = oracle.rope(k, pos, theta, rope_dim).to(torch.bfloat16)
+    ro, rl, _ = oracle.prefill(rq, rk, v, s, 1 / math.sqrt(192), window)
+    assert_close(o, ro * sa.V_SCALE, lse.permute(0, 2, 1), rl, f"fused rope width {rope_dim}")
+    assert sa.sinkattn_take_device_error() == 0
+
+
 def test_fused_rope_prefill_full_size_sampled():
     """The headline workload (B=2, L=32768, 64 Q / 8 KV, W=128) with the SWA layers' RoPE:
     LSE bit for bit against the pass then the prefill; O against the oracle on sampled rows."""
