@@ -109,7 +109,8 @@ class PrefillRunner:
         self.launches = 1
         # the kernel the library dispatches this workload to
         packed = w.window > 0 and w.Hq // w.Hkv == 8 and w.window <= 128 and w.prefix == 0
-        self.kernel = "prefill_swa_packed_kernel" if packed else "prefill_band_kernel"
+        self.kernel = ("prefill_swa_packed_kernel" if packed else
+                       "prefill_wide_kernel" if w.window == 0 else "prefill_band_kernel")
         self.workload = w.name
         self.config = dict(B=w.B, L=w.L, Hq=w.Hq, Hkv=w.Hkv, d_qk=w.dq, d_v=w.dv,
                            window=w.window, kind="SWA" if w.window else "GA")
@@ -501,6 +502,8 @@ def measured_traffic(kernel):
     csrc = os.path.join(ROOT, "global_attention_sink_softmax_b200", "csrc")
     files = {"prefill_swa_packed_kernel": ["common.cuh", "swa_kernels.cuh"],
              "prefill_band_kernel": ["common.cuh", "prefill_kernels.cuh"],
+             "prefill_wide_kernel": ["common.cuh", "prefill_kernels.cuh",
+                                     "prefill_wide_kernels.cuh"],
              "decode_split_kernel": ["common.cuh", "decode_kernels.cuh"],
              "decode_tma_kernel": ["common.cuh", "decode_kernels.cuh",
                                    "decode_tma_kernels.cuh"],

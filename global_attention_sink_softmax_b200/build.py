@@ -14,7 +14,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsinkattn.so")
 SOURCES = ["sinkattn.cu"]
-DEPS = SOURCES + ["common.cuh", "internal.h", "prefill_kernels.cuh", "swa_kernels.cuh",
+DEPS = SOURCES + ["common.cuh", "internal.h", "prefill_kernels.cuh", "prefill_wide_kernels.cuh",
+                  "swa_kernels.cuh",
                   "decode_kernels.cuh", "decode_tma_kernels.cuh", "decode_umma_kernels.cuh",
                   "decode_ring_kernels.cuh", "decode_ring_umma_kernels.cuh", "rope_kernels.cuh", "decode_fp8_kernels.cuh",
                   "decode_fp8_tma_kernels.cuh", "backward_kernels.cuh"]

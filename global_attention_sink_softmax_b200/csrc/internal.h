@@ -33,6 +33,12 @@ cudaError_t launch_prefill_band(const CUtensorMap &tmQ, const CUtensorMap &tmK,
                                 const CUtensorMap &tmV, const CUtensorMap &tmKp,
                                 const CUtensorMap &tmVp, const PrefillParams &p,
                                 cudaStream_t stream);
+// Full-causal prefill (window 0), same maps and parameters: two softmax warpgroups per CTA
+// sharing 256-key tiles.
+cudaError_t launch_prefill_wide(const CUtensorMap &tmQ, const CUtensorMap &tmK,
+                                const CUtensorMap &tmV, const CUtensorMap &tmKp,
+                                const CUtensorMap &tmVp, const PrefillParams &p,
+                                cudaStream_t stream);
 
 // SWA prefill, GQA-packed persistent kernel: item = (b, kv head, block of P = 128 / G positions)
 // Partial RoPE applied to Q and K as they land in shared memory (rope_dim <= 64: the rotary

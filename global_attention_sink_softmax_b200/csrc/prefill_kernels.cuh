@@ -79,6 +79,15 @@ enum Bar {
 };
 } // namespace pf
 
+// max(a, b, c) in one instruction (the three-input form of max.f32, sm_100 and later): the row
+// maximum over 128 scores takes 64 of them instead of 128.
+SA_DEV float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Where key tile j (positions 128 j .. 128 j + 127) of sequence b comes from: the K / V tensors
 // at (row, block) = (position, sequence), or, for a paged prefix, a page of the pool below the
 // prefix (a page id outside the pool reads zeros) and the chunk's own tensors above it.
@@ -312,8 +321,9 @@ __global__ void __launch_bounds__(pf::THREADS, 1)
                         sr[e] = __float_as_uint(-INFINITY);
             }
 #pragma unroll
-            for (int e = 0; e < 128; ++e)
-                mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[e]));
+            for (int e = 0; e < 128; e += 2)
+                mx8[(e >> 1) & 7] =
+                    fmax3(mx8[(e >> 1) & 7], __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
             float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
             mx *= c_l2;

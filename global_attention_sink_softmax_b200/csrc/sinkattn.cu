@@ -19,6 +19,7 @@
 #include "backward_kernels.cuh"
 #include "internal.h"
 #include "prefill_kernels.cuh"
+#include "prefill_wide_kernels.cuh"
 #include "rope_kernels.cuh"
 #include "swa_kernels.cuh"
 
@@ -305,7 +306,9 @@ int run_prefill(const sinkattn_prefill_args *a, int window, int prefix, void *st
     p.page_size = paged ? paged->page_size : 0;
     p.max_pages = paged ? paged->max_pages : 0;
     p.num_pages = paged ? paged->num_pages : 0;
-    const cudaError_t e = launch_prefill_band(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream);
+    const cudaError_t e = (window == 0)
+                              ? launch_prefill_wide(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream)
+                              : launch_prefill_band(tq, tk, tv, tkp, tvp, p, (cudaStream_t)stream);
     return e == cudaSuccess ? SINKATTN_OK : SINKATTN_ERR_CUDA;
 }
 

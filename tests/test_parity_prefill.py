@@ -72,6 +72,19 @@ def test_ga_prefill_shapes(B, L, Hq, Hkv):
     check_full(q, k, v, s, 0, f"ga B{B} L{L} {Hq}/{Hkv}")
 
 
+@pytest.mark.parametrize("B,L,Hq,Hkv,growth", [
+    (1, 1000, 8, 1, 1 / 32), (2, 777, 4, 2, 1 / 16), (1, 1500, 16, 1, -1 / 32),
+])
+def test_ga_prefill_growing_scores(B, L, Hq, Hkv, growth):
+    """Scores that rise (or fall) steadily with the key position: one query dim is 8 and the
+    same key dim is growth x position, so a row's maximum climbs by tens of log2 units across its
+    keys and the kernel's running maximum is raised (and O rescaled) many times over."""
+    q, k, v, s = rand_inputs(B, L, Hq, Hkv, seed=int(L / abs(growth)))
+    q[..., 0] = 8.0
+    k[..., 0] = (torch.arange(L, dtype=torch.float32) * growth).view(1, L, 1).to(torch.bfloat16)
+    check_full(q, k, v, s, 0, f"ga growing B{B} L{L} {Hq}/{Hkv} x{growth}")
+
+
 @pytest.mark.parametrize("mode", ["none", "neginf", "rand"])
 @pytest.mark.parametrize("window", [0, 128])
 def test_sink_modes(mode, window):
