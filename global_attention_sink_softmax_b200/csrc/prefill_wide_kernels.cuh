@@ -5,12 +5,14 @@
 //     O_i = sum_{j <= i} exp(a_ij - m_i) v_j / (exp(sink_h - m_i) + sum_{j <= i} exp(a_ij - m_i)).
 // What changes is how a CTA walks its keys. One CTA still owns 128 query rows of one head, but it
 // takes the keys 256 at a time: the two 128-key halves of a pair go to two softmax warpgroups that
-// run at the same time, so each SMSP holds two softmax warps (the band kernel has one, and its
-// softmax, not the tensor pipe, sets its pace).
+// run at the same time, so each SMSP holds two softmax warps (the band kernel has one), and S
+// takes half as many UMMA instructions per key.
 //
 // Per pair t (keys 256 t .. 256 t + 255; the last pair may have its upper half past the diagonal,
 // in which case that half is neither loaded nor multiplied):
-//   S = Q [K_0 K_1]^T   one M128 N256 K16 x 12 chain, half x into TMEM columns 128 x
+//   S = Q [K_0 K_1]^T   one M128 N256 K16 x 12 chain, half x into TMEM columns 128 x (the two K
+//                       halves interleave by 64-dim region in shared memory, so the 256 keys of
+//                       a region form one K-major operand)
 //   row max             each warpgroup over its half, then swapped through shared memory so both
 //                       use the same running max m (and rescale O by the same factor)
 //   P_x = 2^(S_x c - m) bf16 pairs into TMEM columns 256 + 64 x (P has its own columns: S's can
