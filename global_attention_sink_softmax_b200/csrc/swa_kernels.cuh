@@ -13,13 +13,15 @@
 // The grid is one persistent CTA per SM walking a contiguous run of items (positions fastest).
 // Consecutive items of one (sequence, KV head) share all but P of their span's keys, so K and V
 // sit in shared-memory rings of 16-key chunks and each item loads only its new chunk, one item
-// ahead (the first item of a run loads the whole span); S is split into two MMAs where the span
-// wraps around the ring. Q is double-buffered and streams one item ahead. S is double-buffered
-// in tensor memory; two warpgroups own one S buffer each and work on consecutive items at the
-// same time. Each reads its row of S (48 columns per TMEM round trip), writes P (bf16) back over
-// it, so P.V takes its A operand straight from tensor memory, then reads O (128 columns), frees
-// it for the other warpgroup's P.V and writes O / l and LSE. Loops are kept rolled so the code
-// of the four warp roles fits the SM's instruction caches.
+// ahead (the first item of a run loads the whole span). S is computed over the whole ring in
+// slot order, one M128 N160 chain (10 slots of 16 keys; the slot outside the span is masked), so
+// a span that wraps around the ring costs no extra MMAs. Q is double-buffered and streams one
+// item ahead. S is double-buffered in tensor memory; two warpgroups own one S buffer each and
+// work on consecutive items at the same time. Each reads its row of S (three 16-column chunks per
+// TMEM round trip, the span's chunks in slot order), writes P (bf16) back over it (slot s's P in
+// the 8 columns at 8 s, over scores already read), so P.V takes its A operand straight from tensor
+// memory, then reads O (128 columns), frees it for the other warpgroup's P.V and writes O / l and
+// LSE. Loops are kept rolled so the code of the four warp roles fits the SM's instruction caches.
 //
 // Specialised for the 144-key span of G = 8 query heads per KV head (P = 16) and W <= 128.
 //
@@ -45,7 +47,7 @@ constexpr int Q_BYTES = 3 * Q_REGION;
 constexpr int CHUNK = 16 * ROW;   // one 16-key chunk of one 64-dim region
 constexpr int NSC = 144;          // key span: P + W - 1 rounded up to 16 (G = 8, W <= 128)
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_O = 384;  // S buffer i at i * NSC; P of that item overwrites its first NSC/2
+constexpr uint32_t TMEM_O = 384;  // S buffer i at i * 16 R (R ring slots); P of that item over it
 
 enum Bar {
     Q_FULL = 0,   // + Q buffer
@@ -77,6 +79,8 @@ __host__ __device__ constexpr bool counted_by_rope_warps(int i)
 // K and V rings: R = NSC / 16 + P / 16 chunks of 16 keys per 64-dim region (the span plus the
 // chunks the next item adds, so those load while the current span is still in use).
 __host__ __device__ constexpr int ring_chunks(int p) { return NSC / 16 + p / 16; }
+// two S buffers of 16 R columns (S over the whole ring) below O
+static_assert(2 * 16 * ring_chunks(16) <= (int)TMEM_O, "S buffers fit below O in tensor memory");
 __host__ __device__ constexpr int k_bytes(int p) { return 3 * ring_chunks(p) * CHUNK; }
 __host__ __device__ constexpr int v_bytes(int p) { return 2 * ring_chunks(p) * CHUNK; }
 __host__ __device__ constexpr int off_k() { return 2 * Q_BYTES; }
@@ -153,12 +157,12 @@ __device__ __noinline__ void swa_rope_span(uint8_t *kring, int ks, int L, int64_
     }
 }
 
-// Loads 3 chunks of 16 columns of a row (one TMEM round trip).
-SA_DEV void swa_ld48(uint32_t taddr, uint32_t (&r)[48])
+// Loads the 16-column chunks of ring slots s0, s1, s2 of a row of S (one TMEM round trip).
+SA_DEV void swa_ld48(uint32_t taddr, int s0, int s1, int s2, uint32_t (&r)[48])
 {
-    tmem_ld16(taddr + 0, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
-    tmem_ld16(taddr + 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
-    tmem_ld16(taddr + 32, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
+    tmem_ld16(taddr + s0 * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+    tmem_ld16(taddr + s1 * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[16]));
+    tmem_ld16(taddr + s2 * 16, *reinterpret_cast<uint32_t(*)[16]>(&r[32]));
     tmem_ld_wait();
 #pragma unroll
     for (int i = 0; i < 48; i += 8)
@@ -166,16 +170,24 @@ SA_DEV void swa_ld48(uint32_t taddr, uint32_t (&r)[48])
                      "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])::"memory");
 }
 
-// -inf outside [lo, hi] for columns c0 .. c0 + 47 (skipped when all are inside)
-SA_DEV void swa_mask48(uint32_t (&r)[48], int c0, int lo, int hi)
+// -inf outside span offsets [lo, hi] for three chunks whose first keys sit at span offsets k0, k1,
+// k2 (skipped when all are inside)
+SA_DEV void swa_mask48(uint32_t (&r)[48], int k0, int k1, int k2, int lo, int hi)
 {
-    if (c0 >= lo && c0 + 47 <= hi)
+    if (min(k0, min(k1, k2)) >= lo && max(k0, max(k1, k2)) + 15 <= hi)
         return;
 #pragma unroll
-    for (int u = 0; u < 48; ++u)
-        if (c0 + u < lo || c0 + u > hi)
+    for (int u = 0; u < 48; ++u) {
+        const int k = (u < 16 ? k0 : u < 32 ? k1 : k2) + (u & 15);
+        if (k < lo || k > hi)
             r[u] = __float_as_uint(-INFINITY);
+    }
 }
+
+// The i-th chunk of the span in ring-slot order (i = 0 .. SC - 1): every slot but `out`, the one
+// the span leaves out; its offset in the span is 16 ((slot - base) mod R).
+SA_DEV int swa_span_slot(int i, int out) { return i + (i >= out ? 1 : 0); }
+SA_DEV int swa_span_off(int slot, int base, int R) { return 16 * (slot >= base ? slot - base : slot + R - base); }
 
 __global__ void __launch_bounds__(sw::THREADS, 1)
     prefill_swa_packed_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -309,9 +321,11 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             int base_s = 0;
             int base_even = 0, base_odd = 0; // ring slot of the span's first key, per item parity
             int pblk = (it0 % p.n_pblk) - 1; // position block of the last item issued
-            // S of item n into S buffer n & 1 (warpgroup n & 1). The span is ring slots
-            // base .. base + SC - 1: one MMA per k-step, or two where it wraps. A CTA's items
-            // are consecutive, so the position block and the ring base advance without division.
+            // S of item n into S buffer n & 1 (warpgroup n & 1), over all R ring slots in slot
+            // order (one N = 16 R MMA per k-step, whether or not the span wraps; the slot outside
+            // the span is masked by the softmax). A CTA's items are consecutive, so the position
+            // block and the ring base advance without division.
+            const uint32_t idesc_s = umma_idesc_bf16(128, 16 * R, 0);
             auto issue_s = [&](int n) -> bool {
                 pblk = (pblk + 1 == p.n_pblk) ? 0 : pblk + 1;
                 const int nb_ = base_s + p.P / 16;
@@ -329,20 +343,13 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                 if (n >= 2 && !mbar_wait(&bars[S_FREE + sb], ((n >> 1) - 1) & 1, abort, 1u))
                     return false;
                 tc_fence_after();
-                const int ca = min(SC, R - base_s); // chunks before the wrap
-                const int na = ca * 16, nb = NSC - na;
-                const uint32_t idesc_a = umma_idesc_bf16(128, na, 0);
-                const uint32_t idesc_b = nb > 0 ? umma_idesc_bf16(128, nb, 0) : 0u;
                 const uint64_t qd = sb ? qd1 : qd0;
-                const uint64_t ka = kd0 + (uint32_t)((base_s * CHUNK) >> 4);
-                const uint32_t d = tmem + sb * NSC;
+                const uint32_t d = tmem + sb * 16 * R;
 #pragma unroll 1
                 for (int kk = 0; kk < 12; ++kk) {
                     const uint32_t qo = (uint32_t)((kk >> 2) * Q_REGION + (kk & 3) * 32) >> 4;
                     const uint32_t ko = (kk >> 2) * region16 + (((kk & 3) * 32) >> 4);
-                    umma_ss(d, qd + qo, ka + ko, idesc_a, kk > 0);
-                    if (nb > 0)
-                        umma_ss(d + na, qd + qo, kd0 + ko, idesc_b, kk > 0);
+                    umma_ss(d, qd + qo, kd0 + ko, idesc_s, kk > 0);
                 }
                 umma_commit(&bars[S_FULL + sb]);
                 umma_commit(&bars[Q_EMPTY + sb]);
@@ -362,13 +369,13 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                 if (n >= 1 && !mbar_wait(&bars[O_FREE], (n - 1) & 1, abort, 1u))
                     break;
                 tc_fence_after();
-                const uint32_t pt = tmem + (n & 1) * NSC; // P: 16 keys per 8 columns
+                const uint32_t pt = tmem + (n & 1) * 16 * R; // P of slot s: 8 columns at 8 s
 #pragma unroll 1
                 for (int kk = 0; kk < SC; ++kk) {
                     int slot = base_pv + kk;
                     slot = slot >= R ? slot - R : slot;
-                    umma_ts(tmem + TMEM_O, pt + kk * 8, vd0 + (uint32_t)((slot * CHUNK) >> 4), idesc_o,
-                            kk > 0);
+                    umma_ts(tmem + TMEM_O, pt + slot * 8, vd0 + (uint32_t)((slot * CHUNK) >> 4),
+                            idesc_o, kk > 0);
                 }
                 umma_commit(&bars[PV_DONE + (n & 1)]);
                 umma_commit(&bars[V_EMPTY + (n & 1)]);
@@ -478,23 +485,30 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             const SwaItem it = swa_item(p, it0 + n, n == 0);
             const int l = it.p0 + l_local;
             const int h = it.g * p.G + h_local;
-            // visible columns: ks + c in [max(l - W + 1, 0), l]
+            // visible span offsets: ks + c in [max(l - W + 1, 0), l]
             const int hi = l - it.ks;
             const int lo = max(l - p.W + 1, 0) - it.ks;
+            // ring slot of the span's first chunk (the issuer's base for this item) and the slot
+            // the span leaves out
+            const int base = (min(n, it.p0 / p.P) * A) % R;
+            const int out = (base + SC) % R;
             const float sink_l2 = p.sink ? p.sink[h] * kLog2e : -INFINITY;
             if (!warp_wait(&bars[S_FULL + wg], (n >> 1) & 1, abort))
                 break;
             tc_fence_after();
-            // Row max, then P, in groups of 48 columns per TMEM round trip. The loops stay
-            // rolled: the kernel's code must fit the instruction caches of an SM that runs
-            // four different warp roles.
-            const uint32_t saddr = tmem + lane_addr + wg * NSC;
+            // Row max, then P, three of the span's chunks (in slot order) per TMEM round trip.
+            // The loops stay rolled: the kernel's code must fit the instruction caches of an SM
+            // that runs four different warp roles.
+            const uint32_t saddr = tmem + lane_addr + wg * 16 * R;
             float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-            for (int c0 = 0; c0 < NSC; c0 += 48) {
+            for (int i0 = 0; i0 < SC; i0 += 3) {
+                const int s0 = swa_span_slot(i0, out), s1 = swa_span_slot(i0 + 1, out),
+                          s2 = swa_span_slot(i0 + 2, out);
                 uint32_t r[48];
-                swa_ld48(saddr + c0, r);
-                swa_mask48(r, c0, lo, hi);
+                swa_ld48(saddr, s0, s1, s2, r);
+                swa_mask48(r, swa_span_off(s0, base, R), swa_span_off(s1, base, R),
+                           swa_span_off(s2, base, R), lo, hi);
 #pragma unroll
                 for (int u = 0; u < 48; ++u)
                     mx4[u & 3] = fmaxf(mx4[u & 3], __uint_as_float(r[u]));
@@ -507,10 +521,13 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
             // normalises O and gives LSE
             float pe[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-            for (int c0 = 0; c0 < NSC; c0 += 48) {
+            for (int i0 = 0; i0 < SC; i0 += 3) {
+                const int s0 = swa_span_slot(i0, out), s1 = swa_span_slot(i0 + 1, out),
+                          s2 = swa_span_slot(i0 + 2, out);
                 uint32_t r[48];
-                swa_ld48(saddr + c0, r);
-                swa_mask48(r, c0, lo, hi);
+                swa_ld48(saddr, s0, s1, s2, r);
+                swa_mask48(r, swa_span_off(s0, base, R), swa_span_off(s1, base, R),
+                           swa_span_off(s2, base, R), lo, hi);
 #pragma unroll
                 for (int k = 0; k < 3; ++k) {
                     uint32_t pk[8];
@@ -521,8 +538,10 @@ __global__ void __launch_bounds__(sw::THREADS, 1)
                         pe[(u >> 1) & 3] += e0 + e1;
                         pk[u >> 1] = pack_bf16x2(e0, e1);
                     }
-                    tmem_st8(saddr + c0 / 2 + k * 8, pk[0], pk[1], pk[2], pk[3], pk[4], pk[5],
-                             pk[6], pk[7]);
+                    // P of slot s over S columns 8 s .. 8 s + 7, scores of slot s / 2 <= s,
+                    // already read (slots go in increasing order)
+                    tmem_st8(saddr + (k == 0 ? s0 : k == 1 ? s1 : s2) * 8, pk[0], pk[1], pk[2],
+                             pk[3], pk[4], pk[5], pk[6], pk[7]);
                 }
             }
             tmem_st_wait();
